@@ -1,0 +1,245 @@
+"""fp64 CPU oracle for query-aware sparse attention over a long KV cache.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package.  It shares no code with the CUDA library
+(``long_context_sparse_spa_b200``); both sides meet only in the seeded inputs of
+``synth``.
+
+The arithmetic lives in ``spa_oracle.cpp`` (plain C++ in double precision, one unit at a
+time).  This module marshals numpy arrays into it and loops over units.  Where a float
+decides an integer (the ranking behind top-k / top-p), the decode and prefill drivers
+round the fp64 scores to binary32 first, because the CUDA path ranks binary32 scores:
+both sides then take that decision in the same precision.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from typing import Dict, Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_dbl = ctypes.c_double
+_p = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.orc_abi_version.restype = _int
+        L.orc_block_stats.argtypes = [_p, _i64, _int, _int, _p, _p]
+        L.orc_lowrank_scores.argtypes = [_p, _int, _p, _i64, _int, _int, _dbl, _p]
+        L.orc_taylor_scores.argtypes = [_p, _int, _p, _p, _i64, _int, _dbl, _int, _p]
+        L.orc_rank_order.argtypes = [_p, _i64, _p]
+        L.orc_select_topk.argtypes = [_p, _i64, _i64, _i64, _i64, _p]
+        L.orc_select_topk.restype = _i64
+        L.orc_select_topp.argtypes = [_p, _i64, _dbl, _i64, _i64, _p, _p, _p]
+        L.orc_select_topp.restype = _i64
+        L.orc_sparse_attention.argtypes = [_p, _int, _p, _p, _i64, _int, _p, _i64, _int, _dbl, _p, _p]
+        L.orc_dense_probs.argtypes = [_p, _int, _p, _i64, _int, _dbl, _p]
+        L.orc_prefill_unit.argtypes = [_p, _p, _int, _int, _int, _int, _p, _p, _p, _i64, _i64, _dbl,
+                                       _i64, _i64, _dbl, _int, _p, _p]
+        L.orc_prefill_unit.restype = _i64
+        _LIB = L
+    return _LIB
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data
+
+
+def as_ranked(scores: np.ndarray) -> np.ndarray:
+    """Scores as the ranking sees them: rounded to binary32, widened back to float64."""
+    return np.asarray(scores, np.float64).astype(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------- per-unit
+def block_stats(K: np.ndarray, block: int) -> Tuple[np.ndarray, np.ndarray]:
+    """K [N, d] bf16 bits -> (mean, var) [N // block, d] float64 (population variance)."""
+    K = _c(K, np.uint16)
+    N, d = K.shape
+    nb = N // block
+    mean = np.empty((nb, d)); var = np.empty((nb, d))
+    lib().orc_block_stats(_ptr(K), N, d, block, _ptr(mean), _ptr(var))
+    return mean, var
+
+
+def lowrank_scores(qidx: np.ndarray, kidx: np.ndarray, collapse: bool, scale: float) -> np.ndarray:
+    """qidx [G, r], kidx [N, r] bf16 bits -> scores [N] (collapse) or [G, N], float64."""
+    qidx = _c(qidx, np.uint16); kidx = _c(kidx, np.uint16)
+    G, r = qidx.shape
+    N = kidx.shape[0]
+    out = np.empty(N if collapse else (G, N))
+    lib().orc_lowrank_scores(_ptr(qidx), G, _ptr(kidx), N, r, int(collapse), float(scale), _ptr(out))
+    return out
+
+
+def taylor_scores(q: np.ndarray, mean: np.ndarray, var: np.ndarray, scale: float, collapse: bool) -> np.ndarray:
+    """q [G, d] bf16 bits, mean/var [nb, d] -> Taylor block scores t (linear), [nb] or [G, nb]."""
+    q = _c(q, np.uint16); mean = _c(mean, np.float64); var = _c(var, np.float64)
+    G, d = q.shape
+    nb = mean.shape[0]
+    out = np.empty(nb if collapse else (G, nb))
+    lib().orc_taylor_scores(_ptr(q), G, _ptr(mean), _ptr(var), nb, d, float(scale), int(collapse), _ptr(out))
+    return out
+
+
+def rank_order(s: np.ndarray) -> np.ndarray:
+    s = _c(s, np.float64)
+    order = np.empty(s.size, np.int64)
+    lib().orc_rank_order(_ptr(s), s.size, _ptr(order))
+    return order
+
+
+def select_topk(s: np.ndarray, k: int, sink: int, window: int) -> np.ndarray:
+    s = _c(s, np.float64)
+    idx = np.empty(max(1, s.size), np.int32)
+    n = lib().orc_select_topk(_ptr(s), s.size, k, sink, window, _ptr(idx))
+    return idx[:n].copy()
+
+
+def select_topp(s: np.ndarray, p: float, sink: int, window: int) -> Tuple[np.ndarray, float, int]:
+    """-> (ascending support, index mass of the support, length of the ranked prefix)."""
+    s = _c(s, np.float64)
+    idx = np.empty(max(1, s.size), np.int32)
+    mass = ctypes.c_double(0.0); cut = ctypes.c_int64(0)
+    n = lib().orc_select_topp(_ptr(s), s.size, float(p), sink, window, _ptr(idx),
+                              ctypes.addressof(mass), ctypes.addressof(cut))
+    if n < 0:
+        raise ValueError("top-p needs 0 < p <= 1 and a non-empty score row")
+    return idx[:n].copy(), mass.value, cut.value
+
+
+def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, sm_scale: float,
+                     unit_tokens: int = 1) -> Tuple[np.ndarray, np.ndarray]:
+    """q [G, d], K/V [N, d] bf16 bits, idx support -> (out [G, d], lse [G]) float64."""
+    q = _c(q, np.uint16); K = _c(K, np.uint16); V = _c(V, np.uint16); idx = _c(idx, np.int32)
+    G, d = q.shape
+    out = np.empty((G, d)); lse = np.empty(G)
+    lib().orc_sparse_attention(_ptr(q), G, _ptr(K), _ptr(V), K.shape[0], d, _ptr(idx), idx.size,
+                               unit_tokens, float(sm_scale), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def dense_probs(q: np.ndarray, K: np.ndarray, sm_scale: float) -> np.ndarray:
+    q = _c(q, np.uint16); K = _c(K, np.uint16)
+    P = np.empty(K.shape[0])
+    lib().orc_dense_probs(_ptr(q), q.shape[0], _ptr(K), K.shape[0], q.shape[1], float(sm_scale), _ptr(P))
+    return P
+
+
+def prefill_unit(qblk, qidx_blk, K, V, kidx, t0: int, idx_scale: float, k: int, sink: int,
+                 sm_scale: float, rank_f32: bool = True) -> Tuple[np.ndarray, np.ndarray]:
+    """One (query block, kv head) unit of the shared-support prefill -> (support, out [bq, G, d])."""
+    qblk = _c(qblk, np.uint16); qidx_blk = _c(qidx_blk, np.uint16)
+    K = _c(K, np.uint16); V = _c(V, np.uint16); kidx = _c(kidx, np.uint16)
+    bq, G, d = qblk.shape
+    r = qidx_blk.shape[2]
+    support = np.empty(max(1, min(t0, k + sink)), np.int32)
+    out = np.empty((bq, G, d))
+    n = lib().orc_prefill_unit(_ptr(qblk), _ptr(qidx_blk), bq, G, d, r, _ptr(K), _ptr(V), _ptr(kidx),
+                               K.shape[0], t0, float(idx_scale), k, sink, float(sm_scale), int(rank_f32),
+                               _ptr(support), _ptr(out))
+    if n < 0:
+        raise ValueError("query block outside the cache")
+    return support[:n].copy(), out
+
+
+# --------------------------------------------------------------------------- drivers
+def f32(x: float) -> float:
+    """A scalar parameter as the CUDA path receives it (binary32), widened to double."""
+    return float(np.float32(x))
+
+
+def decode_units(cfg) -> List[Tuple[int, int]]:
+    """(b, head) pairs of a decode workload, in unit order u = b * heads + head."""
+    heads = cfg.Hq if cfg.collapse == "head" else cfg.Hkv
+    return [(b, h) for b in range(cfg.B) for h in range(heads)]
+
+
+def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.ndarray, np.ndarray]] = None,
+                with_output: bool = True) -> Dict[str, object]:
+    """The sparse decode path of one unit: scores -> support -> attention.
+
+    Returns scores (float64, as computed), the ranked scores (binary32-rounded; for
+    Taylor scores their natural log), the support, the index mass (top-p), the output
+    [heads, d] and lse [heads] of the query heads sharing the support.
+    """
+    b, h = decode_units(cfg)[u]
+    G = cfg.G
+    if cfg.collapse == "head":
+        g, heads = h // G, slice(h, h + 1)
+    else:
+        g, heads = h, slice(h * G, (h + 1) * G)
+    res: Dict[str, object] = {"b": b, "g": g}
+    if cfg.score == "lowrank":
+        s = lowrank_scores(x["q_idx"][b, heads], x["Kidx"][b, g], cfg.collapse == "group", f32(cfg.score_scale))
+        ranked = as_ranked(s)
+    else:
+        mean, var = stats if stats is not None else block_stats(x["K"][b, g], cfg.block)
+        t = taylor_scores(x["q"][b, heads], mean, var, f32(cfg.score_scale), True)
+        s = t
+        ranked = as_ranked(np.log(t))
+    res["scores"] = s
+    res["ranked"] = ranked
+    if cfg.select == "topk":
+        idx = select_topk(ranked, cfg.topk, cfg.sink, cfg.window)
+        res["index_mass"] = None
+    else:
+        idx, mass, cut = select_topp(ranked, f32(cfg.topp), cfg.sink, cfg.window)
+        res["index_mass"] = mass
+        res["cut"] = cut
+    res["idx"] = idx
+    if with_output:
+        out, lse = sparse_attention(x["q"][b, heads], x["K"][b, g], x["V"][b, g], idx, f32(cfg.sm_scale),
+                                    cfg.block)
+        res["out"] = out
+        res["lse"] = lse
+    return res
+
+
+def decode(cfg, x: Dict[str, np.ndarray], units: Optional[Sequence[int]] = None, threads: int = 1,
+           with_output: bool = True) -> List[Dict[str, object]]:
+    """decode_unit over several units, optionally on a thread pool (the C calls release the GIL)."""
+    todo = list(range(cfg.U)) if units is None else list(units)
+    if threads <= 1:
+        return [decode_unit(cfg, x, u, with_output=with_output) for u in todo]
+    with ThreadPoolExecutor(threads) as ex:
+        return list(ex.map(lambda u: decode_unit(cfg, x, u, with_output=with_output), todo))
+
+
+def captured_mass(cfg, x: Dict[str, np.ndarray], u: int, idx: np.ndarray) -> float:
+    """Dense head-averaged attention mass on the support [OGS-2.1 P_{l,t}]."""
+    b, h = decode_units(cfg)[u]
+    G = cfg.G
+    if cfg.collapse == "head":
+        g, heads = h // G, slice(h, h + 1)
+    else:
+        g, heads = h, slice(h * G, (h + 1) * G)
+    P = dense_probs(x["q"][b, heads], x["K"][b, g], f32(cfg.sm_scale))
+    rows = (np.asarray(idx, np.int64)[:, None] * cfg.block + np.arange(cfg.block)[None, :]).ravel()
+    return float(P[rows[rows < cfg.N]].sum())
+
+
+def prefill_block(cfg, x: Dict[str, np.ndarray], j: int, g: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Unit (query block j, kv head g) of a shared-support prefill -> (support, out [bq, G, d])."""
+    G, bq = cfg.G, cfg.bq
+    rows = slice(j * bq, (j + 1) * bq)
+    heads = slice(g * G, (g + 1) * G)
+    t0 = cfg.q_start + j * bq
+    return prefill_unit(x["Q"][rows, heads], x["q_idx"][rows, heads], x["K"][g], x["V"][g], x["Kidx"][g],
+                        t0, f32(cfg.score_scale), cfg.topk, cfg.sink, f32(cfg.sm_scale))

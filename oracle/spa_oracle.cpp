@@ -1,0 +1,326 @@
+// Plain, slow, fp64 CPU oracle for query-aware sparse attention over a long KV cache.
+//
+// TEST INFRASTRUCTURE.  Only the tests, the smoke check and the bench's CPU-baseline
+// leg use this library.  It shares no code, header, table or helper with the CUDA
+// library; both sides meet only in the seeded inputs.
+//
+// Every routine works on ONE unit (one batch entry and one kv head, or one query
+// head) at a time, in double precision, and follows the definitions on the method
+// pages literally: no blocking, fusion or reordering beyond what a definition states.
+// bf16 inputs are widened exactly to double.
+//
+// Passages followed (page title, section):
+//   [RTP-2]  "Full Attention Strikes Back" (RTPurbo), Methodology 2: r=16 low-rank
+//            projector on q and k, relevance scored in that subspace.
+//   [RTP-3]  RTPurbo, Methodology 3: dynamic top-p -- accumulate attention mass in
+//            the low-rank space until the cumulative threshold p is reached.
+//   [RTP-1]  RTPurbo, Methodology 1: local heads keep an attention sink and a sliding
+//            window; every support here keeps both.
+//   [OGS-2.1] "Oracle-Guided Sparse Prefill", section 2.1: head-averaged attention
+//            mass P_{l,t}; top-k support; attention recomputed with the original
+//            Q, K, V restricted to the support; b_sel = 1 or 64.
+//   [OGS-2.2] same page, section 2.2: head-collapsed indexer, one shared scoring
+//            channel per GQA group.
+//   [SPLA-2.1] "SPLA", section 2.1: block score exp(q^T kbar)(1 + 1/2 q^T Cov(k) q)
+//            with Cov(k) replaced by its diagonal.
+//
+// Parity pins (tests/test_oracle.py): dense attention and masked attention against
+// torch's fp64 scaled_dot_product_attention, top-k against numpy's lexsort, top-p
+// against brute force over all subsets, block statistics against numpy mean/var,
+// the Taylor score's zero-variance identity and fourth-order agreement on
+// axis-symmetric blocks, and the prefill path against dense causal attention.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <numeric>
+#include <vector>
+
+namespace {
+
+inline double widen_bf16(uint16_t h) {
+    uint32_t u = static_cast<uint32_t>(h) << 16;
+    float f;
+    std::memcpy(&f, &u, sizeof f);
+    return static_cast<double>(f);
+}
+
+// Order of positions by score, highest first; equal scores by ascending position
+// (the tie-break shared by top-k and top-p).
+std::vector<int64_t> rank_order(const double* s, int64_t M) {
+    std::vector<int64_t> order(M);
+    std::iota(order.begin(), order.end(), int64_t{0});
+    std::sort(order.begin(), order.end(), [s](int64_t a, int64_t b) {
+        if (s[a] != s[b]) return s[a] > s[b];
+        return a < b;
+    });
+    return order;
+}
+
+// Forced positions [RTP-1]: the sink [0, sink) and the window [M - window, M).
+void mark_forced(std::vector<char>& keep, int64_t M, int64_t sink, int64_t window) {
+    for (int64_t n = 0; n < std::min(sink, M); ++n) keep[n] = 1;
+    for (int64_t n = std::max<int64_t>(0, M - window); n < M; ++n) keep[n] = 1;
+}
+
+int64_t emit_ascending(const std::vector<char>& keep, int32_t* idx) {
+    int64_t c = 0;
+    for (int64_t n = 0; n < static_cast<int64_t>(keep.size()); ++n)
+        if (keep[n]) idx[c++] = static_cast<int32_t>(n);
+    return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+int orc_abi_version() { return 1; }
+
+// a1 -- per-block mean and diagonal (population) variance of K [SPLA-2.1].
+// K: [N, d] bf16 of one (batch, kv head); only the nb = N / block full blocks count.
+// mean, var: [nb, d].  Variance divides by the block size: the score is an
+// expectation over the block's own tokens.
+void orc_block_stats(const uint16_t* K, int64_t N, int d, int block, double* mean, double* var) {
+    const int64_t nb = N / block;
+    std::vector<double> acc(d);
+    for (int64_t b = 0; b < nb; ++b) {
+        std::fill(acc.begin(), acc.end(), 0.0);
+        for (int t = 0; t < block; ++t)
+            for (int i = 0; i < d; ++i) acc[i] += widen_bf16(K[(b * block + t) * d + i]);
+        for (int i = 0; i < d; ++i) mean[b * d + i] = acc[i] / block;
+        std::fill(acc.begin(), acc.end(), 0.0);
+        for (int t = 0; t < block; ++t)
+            for (int i = 0; i < d; ++i) {
+                const double e = widen_bf16(K[(b * block + t) * d + i]) - mean[b * d + i];
+                acc[i] += e * e;
+            }
+        for (int i = 0; i < d; ++i) var[b * d + i] = acc[i] / block;
+    }
+}
+
+// a2 -- low-rank index scores [RTP-2], head-collapsed when asked [OGS-2.2].
+// qidx: [G, r] bf16 index queries of the G query heads sharing this kv head;
+// kidx: [N, r] bf16 index keys.
+// collapse = 0: out [G, N], out[h, n] = scale * qidx_h . kidx_n
+// collapse = 1: out [N], scored with the mean index query over the G heads
+//               (heads summed in order 0..G-1, then divided by G), which is the
+//               average of the G heads' scores.
+void orc_lowrank_scores(const uint16_t* qidx, int G, const uint16_t* kidx, int64_t N, int r,
+                        int collapse, double scale, double* out) {
+    const int nq = collapse ? 1 : G;
+    std::vector<double> qv(static_cast<size_t>(nq) * r, 0.0);
+    if (collapse) {
+        for (int h = 0; h < G; ++h)
+            for (int j = 0; j < r; ++j) qv[j] += widen_bf16(qidx[h * r + j]);
+        for (int j = 0; j < r; ++j) qv[j] /= G;
+    } else {
+        for (int h = 0; h < G; ++h)
+            for (int j = 0; j < r; ++j) qv[h * r + j] = widen_bf16(qidx[h * r + j]);
+    }
+    for (int h = 0; h < nq; ++h)
+        for (int64_t n = 0; n < N; ++n) {
+            double dot = 0.0;
+            for (int j = 0; j < r; ++j) dot += qv[h * r + j] * widen_bf16(kidx[n * r + j]);
+            out[h * N + n] = scale * dot;
+        }
+}
+
+// a3 -- second-order Taylor block score with diagonal covariance [SPLA-2.1]:
+//   t_{h,b} = exp(q'_h . kbar_b) * (1 + 1/2 * sum_i q'_{h,i}^2 var_{b,i}),  q' = scale * q.
+// q: [G, d] bf16; mean, var: [nb, d].
+// collapse = 0: out [G, nb]; collapse = 1: out [nb] = mean over the G heads of t_{h,b}.
+void orc_taylor_scores(const uint16_t* q, int G, const double* mean, const double* var, int64_t nb,
+                       int d, double scale, int collapse, double* out) {
+    std::vector<double> qp(static_cast<size_t>(G) * d);
+    for (int h = 0; h < G; ++h)
+        for (int i = 0; i < d; ++i) qp[h * d + i] = scale * widen_bf16(q[h * d + i]);
+    for (int64_t b = 0; b < nb; ++b) {
+        double sum_heads = 0.0;
+        for (int h = 0; h < G; ++h) {
+            double lin = 0.0, quad = 0.0;
+            for (int i = 0; i < d; ++i) {
+                lin += qp[h * d + i] * mean[b * d + i];
+                quad += qp[h * d + i] * qp[h * d + i] * var[b * d + i];
+            }
+            const double t = std::exp(lin) * (1.0 + 0.5 * quad);
+            if (collapse) sum_heads += t;
+            else out[h * nb + b] = t;
+        }
+        if (collapse) out[b] = sum_heads / G;
+    }
+}
+
+// Positions sorted by (score desc, position asc); order: [M].
+void orc_rank_order(const double* s, int64_t M, int64_t* order) {
+    const std::vector<int64_t> o = rank_order(s, M);
+    std::copy(o.begin(), o.end(), order);
+}
+
+// a5/a6 -- exact top-k [OGS-2.1] united with the forced sink and window [RTP-1].
+// The ranking runs over all M positions; the k best (ties by ascending position) are
+// kept, then the sink [0, sink) and window [M - window, M) are added.  idx receives
+// the support in ascending order (room for min(M, k + sink + window) entries).
+// Returns the support size.
+int64_t orc_select_topk(const double* s, int64_t M, int64_t k, int64_t sink, int64_t window,
+                        int32_t* idx) {
+    const std::vector<int64_t> order = rank_order(s, M);
+    std::vector<char> keep(M, 0);
+    for (int64_t i = 0; i < std::min(k, M); ++i) keep[order[i]] = 1;
+    mark_forced(keep, M, sink, window);
+    return emit_ascending(keep, idx);
+}
+
+// a4-a6 -- dynamic top-p [RTP-3] united with the forced sink and window [RTP-1].
+// pi_n = exp(s_n - m) / Z is the softmax of the scores over all M positions
+// (m = max score, Z summed in rank order).  The ranked part is the shortest prefix of
+// the rank order whose cumulative mass reaches p * Z ("reaches" read as >=).  The
+// sink and window are then added.  idx receives the ascending support (room for M).
+// index_mass (optional) = sum of pi_n over the whole support; cut (optional) = length
+// of the ranked prefix.  Requires 0 < p <= 1; returns -1 otherwise.
+int64_t orc_select_topp(const double* s, int64_t M, double p, int64_t sink, int64_t window,
+                        int32_t* idx, double* index_mass, int64_t* cut) {
+    if (!(p > 0.0 && p <= 1.0) || M <= 0) return -1;
+    const std::vector<int64_t> order = rank_order(s, M);
+    const double m = s[order[0]];
+    std::vector<double> e(M);
+    double Z = 0.0;
+    for (int64_t i = 0; i < M; ++i) {
+        e[i] = std::exp(s[order[i]] - m);
+        Z += e[i];
+    }
+    const double target = p * Z;
+    int64_t c = 0;
+    double cum = 0.0;
+    while (c < M) {
+        cum += e[c];
+        ++c;
+        if (cum >= target) break;
+    }
+    std::vector<char> keep(M, 0);
+    for (int64_t i = 0; i < c; ++i) keep[order[i]] = 1;
+    mark_forced(keep, M, sink, window);
+    if (index_mass) {
+        double kept = 0.0;
+        for (int64_t n = 0; n < M; ++n)
+            if (keep[n]) kept += std::exp(s[n] - m);
+        *index_mass = kept / Z;
+    }
+    if (cut) *cut = c;
+    return emit_ascending(keep, idx);
+}
+
+// a7/a8 -- exact softmax attention recomputed on a support [OGS-2.1].
+// q: [G, d] bf16 (the query heads that share this support); K, V: [N, d] bf16 rows of
+// one kv head.  The support lists cnt entries; entry i stands for the rows
+// [idx[i] * unit_tokens, idx[i] * unit_tokens + unit_tokens) (unit_tokens = 1 for
+// token supports, the block size for block supports), in any order.
+// out: [G, d]; lse: [G], lse_h = log sum_{rows} exp(sm_scale * q_h . k_row).
+// An empty support gives out = 0 and lse = -inf.
+void orc_sparse_attention(const uint16_t* q, int G, const uint16_t* K, const uint16_t* V, int64_t N,
+                          int d, const int32_t* idx, int64_t cnt, int unit_tokens, double sm_scale,
+                          double* out, double* lse) {
+    std::vector<int64_t> rows;
+    rows.reserve(static_cast<size_t>(cnt) * unit_tokens);
+    for (int64_t i = 0; i < cnt; ++i)
+        for (int t = 0; t < unit_tokens; ++t) {
+            const int64_t row = static_cast<int64_t>(idx[i]) * unit_tokens + t;
+            if (row >= 0 && row < N) rows.push_back(row);
+        }
+    std::vector<double> logit(rows.size());
+    for (int h = 0; h < G; ++h) {
+        double* o = out + static_cast<int64_t>(h) * d;
+        std::fill(o, o + d, 0.0);
+        if (rows.empty()) {
+            if (lse) lse[h] = -std::numeric_limits<double>::infinity();
+            continue;
+        }
+        double mx = -std::numeric_limits<double>::infinity();
+        for (size_t j = 0; j < rows.size(); ++j) {
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i)
+                dot += widen_bf16(q[h * d + i]) * widen_bf16(K[rows[j] * d + i]);
+            logit[j] = sm_scale * dot;
+            mx = std::max(mx, logit[j]);
+        }
+        double Z = 0.0;
+        for (size_t j = 0; j < rows.size(); ++j) {
+            const double w = std::exp(logit[j] - mx);
+            Z += w;
+            for (int i = 0; i < d; ++i) o[i] += w * widen_bf16(V[rows[j] * d + i]);
+        }
+        for (int i = 0; i < d; ++i) o[i] /= Z;
+        if (lse) lse[h] = mx + std::log(Z);
+    }
+}
+
+// Dense head-averaged attention distribution P [OGS-2.1]:
+// P[n] = (1/G) sum_h softmax_n(sm_scale * q_h . k_n) over all N rows.  Used for the
+// captured-mass metric sum_{n in S} P[n]; with G = 1 it is one head's distribution.
+void orc_dense_probs(const uint16_t* q, int G, const uint16_t* K, int64_t N, int d, double sm_scale,
+                     double* P) {
+    std::fill(P, P + N, 0.0);
+    std::vector<double> logit(N);
+    for (int h = 0; h < G; ++h) {
+        double mx = -std::numeric_limits<double>::infinity();
+        for (int64_t n = 0; n < N; ++n) {
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i) dot += widen_bf16(q[h * d + i]) * widen_bf16(K[n * d + i]);
+            logit[n] = sm_scale * dot;
+            mx = std::max(mx, logit[n]);
+        }
+        double Z = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            logit[n] = std::exp(logit[n] - mx);
+            Z += logit[n];
+        }
+        for (int64_t n = 0; n < N; ++n) P[n] += logit[n] / Z / G;
+    }
+}
+
+// a9 -- selection-block-shared sparse prefill for one (query block, kv head) unit
+// [OGS-2.1 b_sel = bq, OGS-2.2 head-collapsed indexer].
+// qblk: [bq, G, d] bf16 queries of the block (positions t0 .. t0+bq-1) for the G query
+// heads of the kv head; qidx_blk: [bq, G, r] their index queries.  K, V: [N, d];
+// kidx: [N, r] of the kv head.
+// 1. index query = mean of qidx_blk over the bq queries and G heads (summed in
+//    (query, head) order, divided by bq*G);
+// 2. scores s_n = idx_scale * index_query . kidx_n over the candidates n in [0, t0)
+//    (rounded to binary32 when rank_f32 != 0, the precision a binary32 ranking sees);
+// 3. support = exact top-k of those scores united with the sink [0, sink)
+//    (written ascending to support, room for min(t0, k + sink)); returns its size;
+// 4. each query t0+i and head h attends, with the original q/K/V, to the support
+//    plus its own block's causal prefix [t0, t0+i]: out [bq, G, d].
+int64_t orc_prefill_unit(const uint16_t* qblk, const uint16_t* qidx_blk, int bq, int G, int d, int r,
+                         const uint16_t* K, const uint16_t* V, const uint16_t* kidx, int64_t N,
+                         int64_t t0, double idx_scale, int64_t k, int64_t sink, double sm_scale,
+                         int rank_f32, int32_t* support, double* out) {
+    if (t0 < 0 || t0 + bq > N) return -1;
+    std::vector<double> qhat(r, 0.0);
+    for (int i = 0; i < bq; ++i)
+        for (int h = 0; h < G; ++h)
+            for (int j = 0; j < r; ++j) qhat[j] += widen_bf16(qidx_blk[(i * G + h) * r + j]);
+    for (int j = 0; j < r; ++j) qhat[j] /= static_cast<double>(bq) * G;
+    std::vector<double> s(t0);
+    for (int64_t n = 0; n < t0; ++n) {
+        double dot = 0.0;
+        for (int j = 0; j < r; ++j) dot += qhat[j] * widen_bf16(kidx[n * r + j]);
+        s[n] = idx_scale * dot;
+        if (rank_f32) s[n] = static_cast<double>(static_cast<float>(s[n]));
+    }
+    const int64_t cnt = t0 > 0 ? orc_select_topk(s.data(), t0, k, sink, 0, support) : 0;
+
+    std::vector<int32_t> rows(support, support + cnt);
+    for (int i = 0; i < bq; ++i) {
+        rows.resize(cnt);
+        for (int j = 0; j <= i; ++j) rows.push_back(static_cast<int32_t>(t0 + j));
+        for (int h = 0; h < G; ++h)
+            orc_sparse_attention(qblk + (static_cast<int64_t>(i) * G + h) * d, 1, K, V, N, d, rows.data(),
+                                 static_cast<int64_t>(rows.size()), 1, sm_scale,
+                                 out + (static_cast<int64_t>(i) * G + h) * d, nullptr);
+    }
+    return cnt;
+}
+
+}  // extern "C"

@@ -1,0 +1,200 @@
+"""Workload definitions for query-aware sparse attention over a long KV cache.
+
+Each workload is a seeded synthetic stand-in for the long-context benchmarks the
+method pages evaluate on (RULER, LongBench and the like are not used; none of
+their items appear here).  The shapes, the selection rule and the structure of
+the keys follow the five workloads the method is measured on:
+
+* ``c1``  tiny per-head top-k decode (d=64, N=4096, 8 single-token needles)
+* ``c2``  head-collapsed top-p decode at 64K (GQA group 8, low-frequency key
+          component, 32 needle clusters of 16 tokens)
+* ``c2_128k`` the same generator and rule at a 128K-token cache: the workload
+          the headline decode throughput is quoted on
+* ``c3``  Taylor block-score top-k decode at 128K (blocks of 64 tokens)
+* ``c4``  million-token top-p decode (256 needle clusters)
+* ``c5``  selection-block-shared sparse prefill (64 queries share a support)
+
+Cited passages (page title, section):
+* r=16 index projector applied before RoPE -- "Full Attention Strikes Back"
+  (RTPurbo), Methodology 2.
+* dynamic top-p with p=0.9 -- RTPurbo, Methodology 3.
+* attention sink + sliding window for local heads -- RTPurbo, Methodology 1.
+* selection-block-shared support b_sel=64, top-k budgets 256-2048 --
+  "Oracle-Guided Sparse Prefill", sections 2.1 and 3.1.
+* Taylor block score from block mean / diagonal variance -- "SPLA", section 2.1.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+
+# Needle amplitude for the clustered-needle generator (c2, c2_128k, c4, c5).
+# Fixed once, before any GPU timing, as the smallest value in
+# NEEDLE_AMPLITUDE_CANDIDATES for which the oracle's support of unit (b=0,
+# kv head 0) of c2 reaches a sparsity of at least 0.89 -- the 64K sparsity the
+# RTPurbo page reports (Key results, "Sparsity").  oracle/calibrate_needles.py
+# recomputes the choice and tests/test_calibration.py checks it.
+NEEDLE_AMPLITUDE_CANDIDATES = (4.0, 8.0, 12.0, 16.0, 20.0, 24.0, 32.0)
+NEEDLE_AMPLITUDE = 24.0
+CALIBRATION_SPARSITY = 0.89
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    """One decode workload: a single new query per (batch, head) against N cached tokens."""
+
+    name: str
+    seed: int
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    N: int
+    score: str            # "lowrank" (r=16 index keys) or "taylor" (block mean/var)
+    select: str           # "topk" or "topp"
+    collapse: str         # "head" (one support per query head) or "group" (per kv head)
+    sink: int             # forced leading units (tokens, or blocks in block mode)
+    window: int           # forced trailing units (tokens, or blocks in block mode)
+    r: int = 16
+    topk: int = 0
+    topp: float = 0.0
+    block: int = 1        # tokens per selection unit (64 for block-sparse decode)
+    keys: str = "gauss"   # "needles" | "clusters" | "blocks"
+    n_needles: int = 0    # single-token needles (keys == "needles")
+    n_clusters: int = 0   # needle clusters of cluster_len tokens (keys == "clusters")
+    cluster_len: int = 16
+    lowfreq_amp: float = 0.0
+    lowfreq_rank: int = 0
+    needle_amp: float = 0.0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def M(self) -> int:
+        """Number of scored units per support (tokens, or blocks)."""
+        return self.N // self.block
+
+    @property
+    def U(self) -> int:
+        """Number of supports selected per step."""
+        return self.B * (self.Hq if self.collapse == "head" else self.Hkv)
+
+    @property
+    def heads_per_unit(self) -> int:
+        return 1 if self.collapse == "head" else self.G
+
+    @property
+    def score_scale(self) -> float:
+        """Index-score scale.
+
+        Low-rank: sqrt(d)/r.  With projector entries ~ N(0, 1/d), E[P P^T] = (r/d) I,
+        so sqrt(d)/r * (q P).(k P) is an unbiased estimate of q.k/sqrt(d), the
+        attention logit, and the softmax of the index scores estimates attention
+        mass (RTPurbo, Methodology 2-3).  Taylor: q' = q/sqrt(d) (SPLA, section 2.1).
+        """
+        if self.score == "lowrank":
+            return math.sqrt(self.d) / self.r
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def cap(self) -> int:
+        """Index capacity per support."""
+        if self.select == "topk":
+            return min(self.M, self.topk + self.sink + self.window)
+        return self.M
+
+    def with_(self, **kw) -> "DecodeConfig":
+        return replace(self, **kw)
+
+
+@dataclass(frozen=True)
+class PrefillConfig:
+    """Selection-block-shared sparse prefill: one chunk of T queries at positions
+    [q_start, q_start + T) against a causal KV cache of N tokens; every block of
+    bq consecutive queries shares one support per kv head."""
+
+    name: str
+    seed: int
+    Hq: int
+    Hkv: int
+    d: int
+    N: int
+    q_start: int
+    T: int
+    r: int = 16
+    bq: int = 64
+    topk: int = 2048
+    sink: int = 4
+    n_clusters: int = 32
+    cluster_len: int = 16
+    lowfreq_amp: float = 1.5
+    lowfreq_rank: int = 4
+    needle_amp: float = 0.0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def n_blocks(self) -> int:
+        return self.T // self.bq
+
+    @property
+    def U(self) -> int:
+        return self.n_blocks * self.Hkv
+
+    @property
+    def score_scale(self) -> float:
+        return math.sqrt(self.d) / self.r
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def cap(self) -> int:
+        return self.topk + self.sink
+
+    def with_(self, **kw) -> "PrefillConfig":
+        return replace(self, **kw)
+
+
+C1 = DecodeConfig(
+    name="c1", seed=0, B=1, Hq=4, Hkv=1, d=64, N=4096, score="lowrank", select="topk",
+    collapse="head", sink=4, window=64, topk=256, keys="needles", n_needles=8, needle_amp=4.0)
+
+C2 = DecodeConfig(
+    name="c2", seed=1, B=4, Hq=32, Hkv=4, d=128, N=65536, score="lowrank", select="topp",
+    collapse="group", sink=4, window=128, topp=0.9, keys="clusters", n_clusters=32,
+    lowfreq_amp=1.5, lowfreq_rank=4, needle_amp=NEEDLE_AMPLITUDE)
+
+C2_128K = C2.with_(name="c2_128k", N=131072)
+
+C3 = DecodeConfig(
+    name="c3", seed=2, B=8, Hq=32, Hkv=8, d=128, N=131072, score="taylor", select="topk",
+    collapse="group", sink=1, window=2, topk=32, block=64, keys="blocks")
+
+C4 = C2.with_(name="c4", seed=3, B=1, N=1 << 20, window=256, n_clusters=256)
+
+C5 = PrefillConfig(
+    name="c5", seed=4, Hq=32, Hkv=8, d=128, N=32768, q_start=28672, T=4096,
+    needle_amp=NEEDLE_AMPLITUDE)
+
+DECODE_CONFIGS = {c.name: c for c in (C1, C2, C2_128K, C3, C4)}
+ALL_CONFIGS = dict(DECODE_CONFIGS, c5=C5)
+
+# Reduced shapes of the same generators, used by parity tests that compare every
+# output element against the oracle.  They span several tiles and end on a ragged tail.
+SMALL = {
+    "c1s": C1.with_(name="c1s", N=3000, topk=200),
+    "c2s": C2.with_(name="c2s", B=2, Hq=16, Hkv=2, N=9001, n_clusters=8),
+    "c3s": C3.with_(name="c3s", B=2, Hq=8, Hkv=2, N=64 * 300 + 17, topk=12),
+    "c4s": C4.with_(name="c4s", N=50_003, n_clusters=24, window=256),
+    "c5s": C5.with_(name="c5s", Hq=8, Hkv=2, N=4096, q_start=3072, T=1024, topk=512),
+}
