@@ -1,0 +1,225 @@
+/*
+ * spa.h -- C ABI of libspa.so: query-aware sparse attention over a long KV cache,
+ * hand-written CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * The path: score every cached key cheaply (low-rank r=16 index keys, or a second-order
+ * Taylor score of 64-token blocks), select a support by top-k or by a sort-free
+ * histogram top-p threshold, always keeping the attention sink and the local window,
+ * then recompute exact softmax attention on the gathered K/V rows only.
+ *
+ * Passages (page title, section):
+ *   "Full Attention Strikes Back" (RTPurbo) Methodology 1 (sink + sliding window),
+ *     2 (r=16 low-rank indexer before RoPE), 3 (dynamic top-p), 5 (sort-free
+ *     histogram threshold, bandwidth-optimised sparse decode).
+ *   "Oracle-Guided Sparse Prefill" 2.1 (top-k support, sparse recompute with the
+ *     original Q/K/V, b_sel = 1 or 64), 2.2 (head-collapsed indexer).
+ *   "SPLA" 2.1 (Taylor block score with diagonal covariance).
+ *
+ * Conventions shared by every entry point
+ *   - bf16 tensors are passed as their 16-bit patterns (uint16_t); all tensors are
+ *     dense, row-major, in the layouts stated per argument, on the current CUDA device.
+ *     bf16 input pointers must be 16-byte aligned.
+ *   - The caller owns all memory.  The library allocates nothing on the device.
+ *     Entry points that need scratch take a workspace (ws, ws_bytes) sized by the
+ *     matching spa_*_workspace_bytes() call.  A workspace must be zero-filled once
+ *     before its first use (cudaMemset); every call leaves it ready for the next one.
+ *     Calls that share a workspace must not overlap on the GPU.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call is
+ *     asynchronous: the returned status covers argument/shape validation and launch
+ *     errors only.  Conditions found on the device (a support larger than its
+ *     capacity) are OR-ed into a status word at the head of the workspace and read
+ *     with spa_read_device_status().
+ *   - Supports (idx) are ascending and duplicate-free.  Entries at and beyond
+ *     min(count[u], cap) of a row are left untouched.
+ *   - Scores are binary32.  Equal scores rank by ascending position.
+ *   - No CPU fallback exists: an unsupported shape returns SPA_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef SPA_H
+#define SPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum spa_status {
+    SPA_OK = 0,
+    SPA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, p outside (0, 1], ... */
+    SPA_ERR_UNSUPPORTED_SHAPE = 2,   /* head dim, index dim, group size or alignment not supported */
+    SPA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the spa_*_workspace_bytes() figure */
+    SPA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed (spa_last_cuda_error) */
+    SPA_ERR_TIMEOUT = 5,             /* device: a bounded wait gave up (reserved; no kernel waits today) */
+    SPA_ERR_CAPACITY = 6             /* device: a support held more than cap entries (count[u] > cap) */
+} spa_status;
+
+typedef enum spa_collapse {
+    SPA_COLLAPSE_NONE = 0,       /* one support per query head: U = B * Hq */
+    SPA_COLLAPSE_GROUP_MEAN = 1  /* one support per kv head, scored for the mean of its G query heads: U = B * Hkv */
+} spa_collapse;
+
+typedef enum spa_score_kind {
+    SPA_SCORE_LOWRANK = 0,      /* s_n = scale * qhat . Kidx_n (r = 16) */
+    SPA_SCORE_TAYLOR_BLOCK = 1  /* s_b = log t_b, t_b = mean_h exp(q'_h . mean_b)(1 + 1/2 sum_i q'_hi^2 var_bi), q' = scale * q */
+} spa_score_kind;
+
+typedef enum spa_select_kind {
+    SPA_SELECT_TOPK = 0,
+    SPA_SELECT_TOPP = 1
+} spa_select_kind;
+
+/* Human-readable name of a status code (static string). */
+const char* spa_status_string(int status);
+
+/* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
+const char* spa_last_cuda_error(void);
+
+/* ABI version of this header: 1. */
+int spa_abi_version(void);
+
+/* ------------------------------------------------------------------------------------
+ * a1. Block statistics ("SPLA" 2.1: first- and second-order block statistics, the
+ * covariance replaced by its diagonal).
+ *   K     [B, Hkv, N, d] bf16 keys.
+ *   mean  [B, Hkv, N / block, d] fp32 out: mean of each full block of `block` tokens.
+ *   var   [B, Hkv, N / block, d] fp32 out: population variance (divided by `block`).
+ * A trailing partial block (N % block tokens) is not an output.  d in {64, 128};
+ * block in {32, 64, 128}.
+ */
+spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block,
+                           float* mean, float* var, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * a2/a3. Index scores, one row of M scores per selection unit.
+ * kind = SPA_SCORE_LOWRANK ("RTPurbo" Methodology 2, head collapse "Oracle-Guided
+ * Sparse Prefill" 2.2):
+ *   q     [B, Hq, r] bf16 index queries (the projected, pre-RoPE queries), r = dim = 16
+ *   keys  [B, Hkv, M, r] bf16 index keys
+ *   var   NULL
+ *   s[u, n] = scale * qhat_u . keys[b, g, n], where qhat_u is query head h's index query
+ *   (collapse NONE, u = b*Hq + h, g = h / G) or the mean of the G index queries of kv
+ *   head g (collapse GROUP_MEAN, u = b*Hkv + g; heads summed in order, divided by G).
+ * kind = SPA_SCORE_TAYLOR_BLOCK ("SPLA" 2.1):
+ *   q     [B, Hq, d] bf16 queries, d = dim in {64, 128}
+ *   keys  [B, Hkv, M, d] fp32 block means (M blocks), var [B, Hkv, M, d] fp32 block variances
+ *   s[u, b] = log t, t = exp(q'.mean_b) * (1 + 1/2 sum_i q'_i^2 var_bi), q' = scale * q,
+ *   with t averaged over the G heads of kv head g (GROUP_MEAN) or per head (NONE).  The
+ *   log keeps the score finite for any input; it ranks blocks exactly as t does.
+ * scores [U, M] fp32 out.  G = Hq / Hkv must be an integer, G <= 16.
+ */
+spa_status spa_index_scores(int kind, const void* q, const void* keys, const float* var,
+                            int B, int Hq, int Hkv, int M, int dim, int collapse, float scale,
+                            float* scores, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * a5/a6. Exact top-k ("Oracle-Guided Sparse Prefill" 2.1) united with the forced sink
+ * and window ("RTPurbo" Methodology 1).
+ *   scores   [U, M] fp32 (row stride M); unit_len NULL or [U] int32: unit u scores only
+ *            its first unit_len[u] <= M entries (L_u = unit_len[u], else M).
+ *   The ranking runs over all L_u positions (score desc, position asc); the best k are
+ *   kept, then positions [0, sink) and [L_u - window, L_u) are added.
+ *   idx      [U, cap] int32 out (ascending); count [U] int32 out (support size; when it
+ *            exceeds cap only cap entries are written and SPA_ERR_CAPACITY is flagged).
+ *   ws       >= spa_select_workspace_bytes(U, M).
+ * The threshold is found by three shared-memory radix-histogram passes over the
+ * order-preserving 32-bit keys of the scores (11 + 11 + 10 bits), run by a thread-block
+ * cluster per unit; the result is exact.
+ */
+spa_status spa_select_topk(const float* scores, const int32_t* unit_len, int U, int M, int k,
+                           int sink, int window, int32_t* idx, int32_t* count, int cap,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * a4-a6. Dynamic top-p ("RTPurbo" Methodology 3, sort-free histogram threshold of
+ * Methodology 5), united with the sink and window.
+ *   With m = max score and e_n = exp(s_n - m), the ranked part is the shortest prefix
+ *   of the rank order whose mass reaches p * sum_n e_n (reach = >=); then [0, sink)
+ *   and [L_u - window, L_u) are added.  Masses are accumulated as 64-bit fixed-point
+ *   integers (e_n scaled by 2^40), so the cut is exact for those masses and independent
+ *   of thread order.  0 < p <= 1; L_u <= 2^23.
+ *   index_mass [U] fp32 out (optional): mass of the whole support over the total mass.
+ * Other arguments as spa_select_topk.
+ */
+spa_status spa_select_topp(const float* scores, const int32_t* unit_len, int U, int M, float p,
+                           int sink, int window, int32_t* idx, int32_t* count, int cap,
+                           float* index_mass, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of spa_select_topk / spa_select_topp. */
+size_t spa_select_workspace_bytes(int U, int M);
+
+/* ------------------------------------------------------------------------------------
+ * a7/a8. Exact softmax attention on the gathered support ("Oracle-Guided Sparse
+ * Prefill" 2.1: recompute with the original Q, K, V restricted to the support;
+ * "RTPurbo" Methodology 5: bandwidth-optimised sparse decode).
+ *   q      [B, Hq, d] bf16 decode queries; K, V [B, Hkv, N, d] bf16 cache.
+ *   idx    [U, cap] int32 supports, count [U]: rows of unit u are the first
+ *          min(count[u], cap) entries; entry i covers cache rows
+ *          [idx*unit_tokens, idx*unit_tokens + unit_tokens).
+ *   collapse NONE: U = B*Hq, unit (b, h) serves query head h of kv head h/G.
+ *   collapse GROUP_MEAN: U = B*Hkv, unit (b, g) serves the G query heads of kv head g.
+ *   out    [B, Hq, d] bf16 out; out_f32 [B, Hq, d] fp32 out (optional);
+ *   lse    [B, Hq] fp32 out (optional): log sum_rows exp(sm_scale * q . k_row).
+ *   An empty support gives out = 0 and lse = -inf.
+ * Split-KV over all SMs: every CTA takes an equal share of all units' rows, gathers
+ * them with cp.async, runs an fp32 online softmax on tensor-core tiles and emits a
+ * partial (o, m, l); the last CTA of each unit merges the partials (log-sum-exp
+ * combine).  d in {64, 128}; G <= 16 for GROUP_MEAN.  ws >= spa_attend_workspace_bytes.
+ */
+spa_status spa_sparse_attend(const uint16_t* q, const uint16_t* K, const uint16_t* V,
+                             int B, int Hq, int Hkv, int N, int d,
+                             const int32_t* idx, const int32_t* count, int cap, int collapse,
+                             int unit_tokens, float sm_scale,
+                             uint16_t* out, float* out_f32, float* lse,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of spa_sparse_attend (depends on the current device's SM count). */
+size_t spa_attend_workspace_bytes(int B, int Hq, int Hkv, int d, int collapse);
+
+/* ------------------------------------------------------------------------------------
+ * Fused decode step: scores (a2 or a3) -> selection (a4-a6) -> attention (a7/a8) in one
+ * call, with the scores kept in the workspace.
+ */
+typedef struct spa_decode_args {
+    int score_kind;          /* spa_score_kind */
+    int select_kind;         /* spa_select_kind */
+    int collapse;            /* spa_collapse */
+    int B, Hq, Hkv, N, d;
+    int r;                   /* index dim (LOWRANK), 16 */
+    int block;               /* tokens per scored unit: 1 (LOWRANK) or the block size (TAYLOR) */
+    const uint16_t* q;       /* [B, Hq, d] */
+    const uint16_t* q_idx;   /* [B, Hq, r] (LOWRANK) */
+    const uint16_t* K;       /* [B, Hkv, N, d] */
+    const uint16_t* V;       /* [B, Hkv, N, d] */
+    const uint16_t* Kidx;    /* [B, Hkv, N, r] (LOWRANK) */
+    const float* bmean;      /* [B, Hkv, N / block, d] (TAYLOR) */
+    const float* bvar;       /* [B, Hkv, N / block, d] (TAYLOR) */
+    float score_scale;       /* LOWRANK: index-score scale; TAYLOR: q' = score_scale * q */
+    float sm_scale;          /* softmax scale of the exact attention */
+    int topk;                /* SPA_SELECT_TOPK */
+    float topp;              /* SPA_SELECT_TOPP */
+    int sink, window;        /* forced leading / trailing scored units */
+    int32_t* idx;            /* [U, cap] out */
+    int32_t* count;          /* [U] out */
+    int cap;
+    float* index_mass;       /* [U] out, optional (top-p) */
+    uint16_t* out;           /* [B, Hq, d] out */
+    float* out_f32;          /* optional */
+    float* lse;              /* optional */
+} spa_decode_args;
+
+spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream);
+size_t spa_decode_workspace_bytes(const spa_decode_args* a);
+
+/* ------------------------------------------------------------------------------------
+ * Device status word of a workspace (sticky OR of SPA_ERR_* bits as (1 << code)).
+ * Synchronises `stream`, copies the word to *bits and, if reset != 0, clears it.
+ * Returns SPA_OK or SPA_ERR_CUDA.
+ */
+spa_status spa_read_device_status(void* ws, void* stream, uint32_t* bits, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPA_H */

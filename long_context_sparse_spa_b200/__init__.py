@@ -1,0 +1,212 @@
+"""Query-aware sparse attention over a long KV cache on B200 (sm_100a).
+
+Thin Python binding of ``libspa.so`` (the C ABI in ``include/spa.h``).  Every function
+here only marshals torch tensors into pointers, sizes and the current CUDA stream and
+calls the library; every step of the computation runs in the library's CUDA kernels.
+There is no fallback: if ``libspa.so`` is missing or a call fails, an exception is raised.
+
+Output tensors and workspaces are allocated here through torch (the caller's allocator);
+the library itself never allocates device memory.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK, SPA_SCORE_TAYLOR_BLOCK,
+                   SPA_SELECT_TOPK, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, check, lib, lib_path)
+
+__all__ = [
+    "SpaError", "lib", "lib_path", "block_stats", "index_scores", "select_topk", "select_topp", "sparse_attend",
+    "decode", "DecodePlan", "workspace", "read_device_status", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
+    "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SELECT_TOPK", "SPA_SELECT_TOPP",
+]
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled device workspace of nbytes (uint8)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def read_device_status(ws: torch.Tensor, reset: bool = True) -> int:
+    """Device status bits of a workspace (1 << SPA_ERR_* for each condition raised)."""
+    bits = ctypes.c_uint32(0)
+    check(lib().spa_read_device_status(ctypes.c_void_p(ws.data_ptr()), _stream(), ctypes.byref(bits), int(reset)))
+    return bits.value
+
+
+# ----------------------------------------------------------------------------- a1
+def block_stats(K: torch.Tensor, block: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K [B, Hkv, N, d] bf16 -> (mean, var) [B, Hkv, N // block, d] fp32."""
+    _need(K, torch.bfloat16, "K")
+    B, Hkv, N, d = K.shape
+    nb = N // block
+    mean = torch.empty((B, Hkv, nb, d), dtype=torch.float32, device=K.device)
+    var = torch.empty_like(mean)
+    check(lib().spa_block_stats(_ptr(K), B, Hkv, N, d, block, _ptr(mean), _ptr(var), _stream()))
+    return mean, var
+
+
+# ----------------------------------------------------------------------------- a2/a3
+def index_scores(kind: int, q: torch.Tensor, keys: torch.Tensor, var: Optional[torch.Tensor], Hkv: int,
+                 collapse: int, scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Scores [U, M] fp32.  LOWRANK: q = q_idx [B, Hq, 16] bf16, keys = Kidx [B, Hkv, M, 16] bf16.
+    TAYLOR: q [B, Hq, d] bf16, keys = block means [B, Hkv, M, d] fp32, var likewise."""
+    _need(q, torch.bfloat16, "q")
+    B, Hq, dim = q.shape
+    M = keys.shape[2]
+    if kind == SPA_SCORE_LOWRANK:
+        _need(keys, torch.bfloat16, "keys")
+    else:
+        _need(keys, torch.float32, "keys")
+        _need(var, torch.float32, "var")
+    U = B * (Hkv if collapse == SPA_COLLAPSE_GROUP_MEAN else Hq)
+    if out is None:
+        out = torch.empty((U, M), dtype=torch.float32, device=q.device)
+    check(lib().spa_index_scores(kind, _ptr(q), _ptr(keys), _ptr(var), B, Hq, Hkv, M, dim, collapse,
+                                 ctypes.c_float(scale), _ptr(out), _stream()))
+    return out
+
+
+# ----------------------------------------------------------------------------- a4-a6
+def _select_out(U: int, cap: int, device) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    idx = torch.full((U, max(cap, 1)), -1, dtype=torch.int32, device=device)
+    count = torch.zeros(U, dtype=torch.int32, device=device)
+    ws = workspace(lib().spa_select_workspace_bytes(U, 0), device)
+    return idx, count, ws
+
+
+def select_topk(scores: torch.Tensor, k: int, sink: int, window: int, cap: Optional[int] = None,
+                unit_len: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """scores [U, M] fp32 -> (idx [U, cap] int32 ascending, count [U] int32)."""
+    _need(scores, torch.float32, "scores")
+    if unit_len is not None:
+        _need(unit_len, torch.int32, "unit_len")
+    U, M = scores.shape
+    cap = min(M, k + sink + window) if cap is None else cap
+    idx, count, ws = _select_out(U, cap, scores.device)
+    check(lib().spa_select_topk(_ptr(scores), _ptr(unit_len), U, M, k, sink, window, _ptr(idx), _ptr(count), cap,
+                                _ptr(ws), ws.numel(), _stream()))
+    return idx, count
+
+
+def select_topp(scores: torch.Tensor, p: float, sink: int, window: int, cap: Optional[int] = None,
+                unit_len: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """scores [U, M] fp32 -> (idx [U, cap] int32 ascending, count [U] int32, index_mass [U] fp32)."""
+    _need(scores, torch.float32, "scores")
+    if unit_len is not None:
+        _need(unit_len, torch.int32, "unit_len")
+    U, M = scores.shape
+    cap = M if cap is None else cap
+    idx, count, ws = _select_out(U, cap, scores.device)
+    mass = torch.zeros(U, dtype=torch.float32, device=scores.device)
+    check(lib().spa_select_topp(_ptr(scores), _ptr(unit_len), U, M, ctypes.c_float(p), sink, window, _ptr(idx),
+                                _ptr(count), cap, _ptr(mass), _ptr(ws), ws.numel(), _stream()))
+    return idx, count, mass
+
+
+# ----------------------------------------------------------------------------- a7/a8
+def sparse_attend(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+                  collapse: int, sm_scale: float, unit_tokens: int = 1, ws: Optional[torch.Tensor] = None,
+                  want_f32: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor], torch.Tensor]:
+    """q [B, Hq, d], K/V [B, Hkv, N, d] bf16; idx [U, cap], count [U] int32 ->
+    (out [B, Hq, d] bf16, out_f32 [B, Hq, d] or None, lse [B, Hq] fp32)."""
+    for t, n in ((q, "q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n)
+    _need(idx, torch.int32, "idx")
+    _need(count, torch.int32, "count")
+    B, Hq, d = q.shape
+    _, Hkv, N, _ = K.shape
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    out32 = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device) if want_f32 else None
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(lib().spa_attend_workspace_bytes(B, Hq, Hkv, d, collapse), q.device)
+    check(lib().spa_sparse_attend(_ptr(q), _ptr(K), _ptr(V), B, Hq, Hkv, N, d, _ptr(idx), _ptr(count),
+                                  idx.shape[1], collapse, unit_tokens, ctypes.c_float(sm_scale), _ptr(out),
+                                  _ptr(out32), _ptr(lse), _ptr(ws), ws.numel(), _stream()))
+    return out, out32, lse
+
+
+# ----------------------------------------------------------------------------- fused decode
+@dataclass
+class DecodePlan:
+    """Arguments, outputs and workspace of one fused decode step, built once and reused."""
+
+    args: SpaDecodeArgs
+    ws: torch.Tensor
+    idx: torch.Tensor
+    count: torch.Tensor
+    index_mass: Optional[torch.Tensor]
+    out: torch.Tensor
+    out_f32: Optional[torch.Tensor]
+    lse: Optional[torch.Tensor]
+    keep: tuple   # tensors the pointers refer to
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        check(lib().spa_decode(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
+                               _stream(stream)))
+
+
+def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor, K: torch.Tensor,
+           V: torch.Tensor, q_idx: Optional[torch.Tensor] = None, Kidx: Optional[torch.Tensor] = None,
+           bmean: Optional[torch.Tensor] = None, bvar: Optional[torch.Tensor] = None, block: int = 1,
+           score_scale: float, sm_scale: float, topk: int = 0, topp: float = 0.0, sink: int = 0,
+           window: int = 0, cap: Optional[int] = None, want_f32: bool = True, want_lse: bool = True,
+           run: bool = True) -> DecodePlan:
+    """Build (and by default run) a fused decode step; see spa_decode in include/spa.h."""
+    for t, n in ((q, "q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, d = q.shape
+    _, Hkv, N, _ = K.shape
+    U = B * (Hkv if collapse == SPA_COLLAPSE_GROUP_MEAN else Hq)
+    M = N // block
+    if cap is None:
+        cap = min(M, topk + sink + window) if select_kind == SPA_SELECT_TOPK else M
+    dev = q.device
+    idx = torch.full((U, max(cap, 1)), -1, dtype=torch.int32, device=dev)
+    count = torch.zeros(U, dtype=torch.int32, device=dev)
+    mass = torch.zeros(U, dtype=torch.float32, device=dev) if select_kind == SPA_SELECT_TOPP else None
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    out32 = torch.empty((B, Hq, d), dtype=torch.float32, device=dev) if want_f32 else None
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if want_lse else None
+    a = SpaDecodeArgs()
+    a.score_kind, a.select_kind, a.collapse = score_kind, select_kind, collapse
+    a.B, a.Hq, a.Hkv, a.N, a.d = B, Hq, Hkv, N, d
+    a.r = q_idx.shape[-1] if q_idx is not None else 16
+    a.block = block
+    a.q, a.K, a.V = _ptr(q), _ptr(K), _ptr(V)
+    a.q_idx, a.Kidx = _ptr(q_idx), _ptr(Kidx)
+    a.bmean, a.bvar = _ptr(bmean), _ptr(bvar)
+    a.score_scale, a.sm_scale = score_scale, sm_scale
+    a.topk, a.topp, a.sink, a.window = topk, topp, sink, window
+    a.idx, a.count, a.cap = _ptr(idx), _ptr(count), cap
+    a.index_mass = _ptr(mass)
+    a.out, a.out_f32, a.lse = _ptr(out), _ptr(out32), _ptr(lse)
+    ws = workspace(lib().spa_decode_workspace_bytes(ctypes.byref(a)), dev)
+    plan = DecodePlan(a, ws, idx, count, mass, out, out32, lse, (q, K, V, q_idx, Kidx, bmean, bvar))
+    if run:
+        plan.run()
+    return plan

@@ -1,0 +1,282 @@
+// Host side of the C ABI declared in include/spa.h: argument validation, workspace
+// layout and kernel launches.  No entry point allocates device memory.
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.cuh"
+
+namespace spa {
+
+namespace {
+thread_local std::string g_last_cuda_error;
+std::mutex g_info_mu;
+std::vector<DeviceInfo> g_info;
+}  // namespace
+
+spa_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
+    return SPA_ERR_CUDA;
+}
+
+const DeviceInfo& device_info() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_info_mu);
+    if (int(g_info.size()) <= dev) g_info.resize(dev + 1);
+    DeviceInfo& d = g_info[dev];
+    if (d.device < 0) {
+        cudaDeviceProp prop{};
+        if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess) {
+            d.num_sms = prop.multiProcessorCount;
+            d.max_smem_optin = int(prop.sharedMemPerBlockOptin);
+            d.cc_major = prop.major;
+            d.cc_minor = prop.minor;
+        } else {
+            d.num_sms = 148;
+            d.max_smem_optin = 232448;
+        }
+        d.device = dev;
+    }
+    return d;
+}
+
+namespace {
+
+inline bool bad_dims(int B, int Hq, int Hkv) { return B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0; }
+
+size_t decode_scores_bytes(const spa_decode_args* a) {
+    const int U = a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->B * a->Hkv : a->B * a->Hq;
+    const int M = a->score_kind == SPA_SCORE_TAYLOR_BLOCK ? a->N / (a->block > 0 ? a->block : 1) : a->N;
+    return align_up(size_t(U) * size_t(M) * 4, 256);
+}
+
+}  // namespace
+}  // namespace spa
+
+using namespace spa;
+
+extern "C" {
+
+const char* spa_status_string(int s) {
+    switch (s) {
+        case SPA_OK: return "SPA_OK";
+        case SPA_ERR_INVALID_ARG: return "SPA_ERR_INVALID_ARG";
+        case SPA_ERR_UNSUPPORTED_SHAPE: return "SPA_ERR_UNSUPPORTED_SHAPE";
+        case SPA_ERR_WORKSPACE_TOO_SMALL: return "SPA_ERR_WORKSPACE_TOO_SMALL";
+        case SPA_ERR_CUDA: return "SPA_ERR_CUDA";
+        case SPA_ERR_TIMEOUT: return "SPA_ERR_TIMEOUT";
+        case SPA_ERR_CAPACITY: return "SPA_ERR_CAPACITY";
+        default: return "SPA_ERR_UNKNOWN";
+    }
+}
+
+const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+int spa_abi_version(void) { return 1; }
+
+spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean, float* var,
+                           void* stream) {
+    if (B < 0 || Hkv <= 0 || N < 0 || block <= 0) return SPA_ERR_INVALID_ARG;
+    if (B == 0 || N / block == 0) return SPA_OK;
+    if (!K || !mean || !var) return SPA_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || (block != 32 && block != 64 && block != 128)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(K) || !aligned16(mean) || !aligned16(var)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    return launch_block_stats(K, B, Hkv, N, d, block, mean, var, static_cast<cudaStream_t>(stream));
+}
+
+spa_status spa_index_scores(int kind, const void* q, const void* keys, const float* var, int B, int Hq, int Hkv,
+                            int M, int dim, int collapse, float scale, float* scores, void* stream) {
+    if (bad_dims(B, Hq, Hkv) || M < 0) return SPA_ERR_INVALID_ARG;
+    if (collapse != SPA_COLLAPSE_NONE && collapse != SPA_COLLAPSE_GROUP_MEAN) return SPA_ERR_INVALID_ARG;
+    if (B == 0 || M == 0) return SPA_OK;
+    if (!q || !keys || !scores) return SPA_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    if (G > 16) return SPA_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == SPA_SCORE_LOWRANK) {
+        if (dim != 16) return SPA_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(q) || !aligned16(keys)) return SPA_ERR_UNSUPPORTED_SHAPE;
+        return launch_lowrank_scores(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(keys), B, Hq, Hkv,
+                                     M, collapse, scale, scores, nullptr, 0, st);
+    }
+    if (kind == SPA_SCORE_TAYLOR_BLOCK) {
+        if (!var) return SPA_ERR_INVALID_ARG;
+        if (dim != 64 && dim != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(keys) || !aligned16(var)) return SPA_ERR_UNSUPPORTED_SHAPE;
+        return launch_taylor_scores(static_cast<const uint16_t*>(q), static_cast<const float*>(keys), var, B, Hq,
+                                    Hkv, M, dim, collapse, scale, scores, nullptr, 0, st);
+    }
+    return SPA_ERR_INVALID_ARG;
+}
+
+size_t spa_select_workspace_bytes(int U, int M) {
+    (void)U;
+    (void)M;
+    return kWsHeader;
+}
+
+static spa_status select_common(const float* scores, const int32_t* unit_len, int U, int M, int sink, int window,
+                                int32_t* idx, int32_t* count, int cap, void* ws, size_t ws_bytes) {
+    if (U < 0 || M < 0 || sink < 0 || window < 0 || cap < 0) return SPA_ERR_INVALID_ARG;
+    if (U > 65535) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (U == 0) return SPA_OK;
+    if (!scores || !idx || !count || !ws) return SPA_ERR_INVALID_ARG;
+    if (ws_bytes < spa_select_workspace_bytes(U, M)) return SPA_ERR_WORKSPACE_TOO_SMALL;
+    (void)unit_len;
+    return SPA_OK;
+}
+
+spa_status spa_select_topk(const float* scores, const int32_t* unit_len, int U, int M, int k, int sink, int window,
+                           int32_t* idx, int32_t* count, int cap, void* ws, size_t ws_bytes, void* stream) {
+    spa_status s = select_common(scores, unit_len, U, M, sink, window, idx, count, cap, ws, ws_bytes);
+    if (s != SPA_OK || U == 0) return s;
+    if (k < 0) return SPA_ERR_INVALID_ARG;
+    SelectParams p{scores, unit_len, U, M, k, 0.f, sink, window, idx, count, cap, nullptr,
+                   static_cast<uint32_t*>(ws)};
+    return launch_select(p, false, static_cast<cudaStream_t>(stream));
+}
+
+spa_status spa_select_topp(const float* scores, const int32_t* unit_len, int U, int M, float p, int sink,
+                           int window, int32_t* idx, int32_t* count, int cap, float* index_mass, void* ws,
+                           size_t ws_bytes, void* stream) {
+    spa_status s = select_common(scores, unit_len, U, M, sink, window, idx, count, cap, ws, ws_bytes);
+    if (s != SPA_OK || U == 0) return s;
+    if (!(p > 0.f && p <= 1.f)) return SPA_ERR_INVALID_ARG;
+    if (M > (1 << 23)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    SelectParams sp{scores, unit_len, U, M, 0, p, sink, window, idx, count, cap, index_mass,
+                    static_cast<uint32_t*>(ws)};
+    return launch_select(sp, true, static_cast<cudaStream_t>(stream));
+}
+
+size_t spa_attend_workspace_bytes(int B, int Hq, int Hkv, int d, int collapse) {
+    if (bad_dims(B, Hq, Hkv)) return 0;
+    const int U = collapse == SPA_COLLAPSE_GROUP_MEAN ? B * Hkv : B * Hq;
+    const int nh = collapse == SPA_COLLAPSE_GROUP_MEAN ? Hq / Hkv : 1;
+    return kWsHeader + attend_scratch_bytes(U, nh, d);
+}
+
+static spa_status attend_params(const uint16_t* q, const uint16_t* K, const uint16_t* V, int B, int Hq, int Hkv,
+                                int N, int d, const int32_t* idx, const int32_t* count, int cap, int collapse,
+                                int unit_tokens, float sm_scale, uint16_t* out, float* out_f32, float* lse,
+                                void* ws, size_t ws_bytes, AttendParams& p) {
+    if (bad_dims(B, Hq, Hkv) || N < 0 || cap < 0 || unit_tokens <= 0) return SPA_ERR_INVALID_ARG;
+    if (collapse != SPA_COLLAPSE_NONE && collapse != SPA_COLLAPSE_GROUP_MEAN) return SPA_ERR_INVALID_ARG;
+    if (!q || !K || !V || !idx || !count || !out || !ws) return SPA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (collapse == SPA_COLLAPSE_GROUP_MEAN && Hq / Hkv > 16) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (ws_bytes < spa_attend_workspace_bytes(B, Hq, Hkv, d, collapse)) return SPA_ERR_WORKSPACE_TOO_SMALL;
+    const int U = collapse == SPA_COLLAPSE_GROUP_MEAN ? B * Hkv : B * Hq;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p = AttendParams{};
+    p.q = q; p.K = K; p.V = V;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.d = d;
+    p.idx = idx; p.count = count; p.cap = cap; p.collapse = collapse; p.unit_tokens = unit_tokens;
+    p.sm_scale = sm_scale; p.out = out; p.out_f32 = out_f32; p.lse = lse;
+    p.status = reinterpret_cast<uint32_t*>(w);
+    p.tickets = reinterpret_cast<int*>(w + kWsHeader);
+    p.partials = reinterpret_cast<float*>(w + kWsHeader + align_up(size_t(U) * 4, 256));
+    return SPA_OK;
+}
+
+spa_status spa_sparse_attend(const uint16_t* q, const uint16_t* K, const uint16_t* V, int B, int Hq, int Hkv, int N,
+                             int d, const int32_t* idx, const int32_t* count, int cap, int collapse,
+                             int unit_tokens, float sm_scale, uint16_t* out, float* out_f32, float* lse, void* ws,
+                             size_t ws_bytes, void* stream) {
+    if (B == 0) return SPA_OK;
+    AttendParams p;
+    spa_status s = attend_params(q, K, V, B, Hq, Hkv, N, d, idx, count, cap, collapse, unit_tokens, sm_scale, out,
+                                 out_f32, lse, ws, ws_bytes, p);
+    if (s != SPA_OK) return s;
+    return launch_attend(p, static_cast<cudaStream_t>(stream));
+}
+
+size_t spa_decode_workspace_bytes(const spa_decode_args* a) {
+    if (!a || bad_dims(a->B, a->Hq, a->Hkv)) return 0;
+    return kWsHeader + decode_scores_bytes(a) + attend_scratch_bytes(
+        a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->B * a->Hkv : a->B * a->Hq,
+        a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->Hq / a->Hkv : 1, a->d);
+}
+
+spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream) {
+    if (!a || !ws) return SPA_ERR_INVALID_ARG;
+    if (bad_dims(a->B, a->Hq, a->Hkv) || a->N < 0) return SPA_ERR_INVALID_ARG;
+    if (a->B == 0) return SPA_OK;
+    if (ws_bytes < spa_decode_workspace_bytes(a)) return SPA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool group = a->collapse == SPA_COLLAPSE_GROUP_MEAN;
+    if (!group && a->collapse != SPA_COLLAPSE_NONE) return SPA_ERR_INVALID_ARG;
+    const int U = group ? a->B * a->Hkv : a->B * a->Hq;
+    const bool taylor = a->score_kind == SPA_SCORE_TAYLOR_BLOCK;
+    if (!taylor && a->score_kind != SPA_SCORE_LOWRANK) return SPA_ERR_INVALID_ARG;
+    const int block = taylor ? a->block : 1;
+    if (block <= 0 || (!taylor && a->block > 1)) return SPA_ERR_INVALID_ARG;
+    const int M = a->N / block;
+    if (U > 65535) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (a->select_kind == SPA_SELECT_TOPP) {
+        if (!(a->topp > 0.f && a->topp <= 1.f)) return SPA_ERR_INVALID_ARG;
+        if (M > (1 << 23)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    } else if (a->select_kind == SPA_SELECT_TOPK) {
+        if (a->topk < 0) return SPA_ERR_INVALID_ARG;
+    } else {
+        return SPA_ERR_INVALID_ARG;
+    }
+    if (a->sink < 0 || a->window < 0 || a->cap < 0) return SPA_ERR_INVALID_ARG;
+    if (taylor) {
+        if (!a->bmean || !a->bvar) return SPA_ERR_INVALID_ARG;
+        if (a->d != 64 && a->d != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(a->bmean) || !aligned16(a->bvar)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    } else {
+        if (!a->q_idx || !a->Kidx) return SPA_ERR_INVALID_ARG;
+        if (a->r != 16) return SPA_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(a->q_idx) || !aligned16(a->Kidx)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    }
+
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    uint32_t* status = reinterpret_cast<uint32_t*>(w);
+    float* scores = reinterpret_cast<float*>(w + kWsHeader);
+    uint8_t* attend_ws = w + kWsHeader + decode_scores_bytes(a);
+
+    // attention parameters first: they validate q/K/V/idx/out and carve the workspace
+    AttendParams ap;
+    spa_status s = attend_params(a->q, a->K, a->V, a->B, a->Hq, a->Hkv, a->N, a->d, a->idx, a->count, a->cap,
+                                 a->collapse, block, a->sm_scale, a->out, a->out_f32, a->lse, ws,
+                                 size_t(-1), ap);
+    if (s != SPA_OK) return s;
+    ap.tickets = reinterpret_cast<int*>(attend_ws);
+    ap.partials = reinterpret_cast<float*>(attend_ws + align_up(size_t(U) * 4, 256));
+
+    // 1. scores (the scoring kernel also zeroes the attention tickets)
+    if (taylor) {
+        s = launch_taylor_scores(a->q, a->bmean, a->bvar, a->B, a->Hq, a->Hkv, M, a->d, a->collapse,
+                                 a->score_scale, scores, ap.tickets, U, st);
+    } else {
+        s = launch_lowrank_scores(a->q_idx, a->Kidx, a->B, a->Hq, a->Hkv, M, a->collapse, a->score_scale, scores,
+                                  ap.tickets, U, st);
+    }
+    if (s != SPA_OK) return s;
+
+    // 2. selection
+    SelectParams sp{scores, nullptr, U, M, a->topk, a->topp, a->sink, a->window, a->idx, a->count, a->cap,
+                    a->index_mass, status};
+    s = launch_select(sp, a->select_kind == SPA_SELECT_TOPP, st);
+    if (s != SPA_OK) return s;
+
+    // 3. attention on the gathered rows
+    return launch_attend(ap, st);
+}
+
+spa_status spa_read_device_status(void* ws, void* stream, uint32_t* bits, int reset) {
+    if (!ws || !bits) return SPA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SPA_CUDA_TRY(cudaMemcpyAsync(bits, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, st));
+    SPA_CUDA_TRY(cudaStreamSynchronize(st));
+    if (reset) {
+        SPA_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(uint32_t), st));
+        SPA_CUDA_TRY(cudaStreamSynchronize(st));
+    }
+    return SPA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,349 @@
+// Streaming score kernels: low-rank index scores ("Full Attention Strikes Back"
+// (RTPurbo), Methodology 2; head collapse per "Oracle-Guided Sparse Prefill" 2.2),
+// Taylor block scores and block statistics ("SPLA" 2.1).
+//
+// All three are HBM-bound streams with a few flops per byte: they are written for
+// coalesced 128-bit loads, enough bytes in flight per SM and grids sized in multiples
+// of the SM count.  Reductions run in a fixed order, so results are bit-reproducible.
+#include "internal.cuh"
+
+namespace spa {
+namespace {
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ============================================================================ low-rank
+// One work item = (kv unit, chunk of kChunk rows).  Two lanes share a 32-byte index-key
+// row: each loads one 16-byte half (8 bf16) and the halves are joined with one
+// warp shuffle.  Each thread keeps kUnroll rows of loads in flight.
+constexpr int kLrThreads = 256;
+constexpr int kLrUnroll = 4;
+constexpr int kLrChunk = 4096;
+
+template <int NQ>
+__global__ void __launch_bounds__(kLrThreads)
+lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict__ kidx, int Hq, int Hkv,
+                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items,
+                      int* zero_ptr, int zero_count) {
+    if (zero_ptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_ptr[i] = 0;
+
+    const int G = Hq / Hkv;
+    const int half = threadIdx.x & 1;          // which 8 of the 16 index dims this lane holds
+    const int pair = threadIdx.x >> 1;         // row slot within a pass
+    constexpr int kRowsPerPass = kLrThreads / 2;
+
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int kvu = item / chunks_per_unit;        // b * Hkv + g
+        const int chunk = item - kvu * chunks_per_unit;
+        const int b = kvu / Hkv, g = kvu - b * Hkv;
+
+        // Index query (8 dims of it) per query vector, fp32.
+        float qv[NQ][8];
+        const uint16_t* qbase = qidx + (size_t(b) * Hq + size_t(g) * G) * 16 + half * 8;
+        if (NQ == 1) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int h = 0; h < G; ++h) {             // heads summed in order 0..G-1
+                const uint4 w = *reinterpret_cast<const uint4*>(qbase + size_t(h) * 16);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[2 * j] += bf_lo(ws[j]);
+                    acc[2 * j + 1] += bf_hi(ws[j]);
+                }
+            }
+            const float fg = float(G);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) qv[0][j] = acc[j] / fg;
+        } else {
+#pragma unroll
+            for (int h = 0; h < NQ; ++h) {
+                const uint4 w = *reinterpret_cast<const uint4*>(qbase + size_t(h) * 16);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    qv[h][2 * j] = bf_lo(ws[j]);
+                    qv[h][2 * j + 1] = bf_hi(ws[j]);
+                }
+            }
+        }
+
+        const int n0 = chunk * kLrChunk;
+        const int n1 = min(M, n0 + kLrChunk);
+        const uint4* krow = kidx + size_t(kvu) * M * 2 + half;
+        float* out_base = NQ == 1 ? scores + size_t(kvu) * M : scores + (size_t(b) * Hq + size_t(g) * G) * M;
+
+        for (int nb = n0 + pair; nb < n1; nb += kRowsPerPass * kLrUnroll) {
+            uint4 w[kLrUnroll];
+#pragma unroll
+            for (int i = 0; i < kLrUnroll; ++i) {
+                const int n = nb + i * kRowsPerPass;
+                w[i] = n < n1 ? __ldg(krow + size_t(n) * 2) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < kLrUnroll; ++i) {
+                const int n = nb + i * kRowsPerPass;
+                const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+                for (int h = 0; h < NQ; ++h) {
+                    float part = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        part = fmaf(qv[h][2 * j], bf_lo(ws[j]), part);
+                        part = fmaf(qv[h][2 * j + 1], bf_hi(ws[j]), part);
+                    }
+                    const float other = __shfl_xor_sync(0xffffffffu, part, 1);
+                    const float dot = half ? other + part : part + other;   // low half + high half
+                    if (!half && n < n1) out_base[size_t(h) * M + n] = scale * dot;
+                }
+            }
+        }
+    }
+}
+
+// ============================================================================ Taylor
+// One work item = (kv unit, chunk of kTyChunk blocks).  Eight lanes share a block: each
+// holds D/8 dims of the block mean and variance (float4 loads) and the partial sums
+// a_h = q'_h . mean and c_h = sum q'_h^2 var for the G heads are joined by three
+// xor-shuffles.  q' = scale * q lives in shared memory.
+constexpr int kTyThreads = 256;
+constexpr int kTyChunk = 256;
+
+template <int D, int G>
+__global__ void __launch_bounds__(kTyThreads)
+taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ mean, const float4* __restrict__ var,
+                     int Hq, int Hkv, int M, int collapse, float scale, float* __restrict__ scores,
+                     int chunks_per_unit, int n_items, int* zero_ptr, int zero_count) {
+    if (zero_ptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_ptr[i] = 0;
+    __shared__ float qs[G][D];
+    constexpr int kPer = D / 8;          // dims per lane
+    constexpr int kVec = kPer / 4;       // float4 loads per lane per tensor
+    const int lane8 = threadIdx.x & 7;
+    const int slot = threadIdx.x >> 3;   // block slot within a pass
+    constexpr int kSlots = kTyThreads / 8;
+    int cur_kvu = -1;
+
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int kvu = item / chunks_per_unit;
+        const int chunk = item - kvu * chunks_per_unit;
+        const int b = kvu / Hkv, g = kvu - b * Hkv;
+        if (kvu != cur_kvu) {
+            __syncthreads();
+            for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+                const uint16_t h = q[(size_t(b) * Hq + size_t(g) * G + i / D) * D + (i % D)];
+                qs[i / D][i % D] = scale * __uint_as_float(uint32_t(h) << 16);
+            }
+            __syncthreads();
+            cur_kvu = kvu;
+        }
+        const int b0 = chunk * kTyChunk;
+        const int b1 = min(M, b0 + kTyChunk);
+        for (int pass = b0; pass < b1; pass += kSlots) {   // same trip count for every lane
+            const int blk = pass + slot;
+            const bool live = blk < b1;
+            float a[G], c[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) a[h] = c[h] = 0.f;
+            if (live) {
+                const size_t base = (size_t(kvu) * M + blk) * (D / 4);
+#pragma unroll
+                for (int v = 0; v < kVec; ++v) {
+                    // lane8 owns dims {4*(lane8 + 8*v) .. +3}: 8 lanes read 128 contiguous bytes
+                    const int f4 = lane8 + 8 * v;
+                    const float4 mu = __ldg(mean + base + f4);
+                    const float4 vr = __ldg(var + base + f4);
+                    const float mus[4] = {mu.x, mu.y, mu.z, mu.w};
+                    const float vrs[4] = {vr.x, vr.y, vr.z, vr.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 4 * f4 + e;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float qp = qs[h][i];
+                            a[h] = fmaf(qp, mus[e], a[h]);
+                            c[h] = fmaf(qp * qp, vrs[e], c[h]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = 4; off >= 1; off >>= 1) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    a[h] += __shfl_xor_sync(0xffffffffu, a[h], off);
+                    c[h] += __shfl_xor_sync(0xffffffffu, c[h], off);
+                }
+            }
+            if (!live) continue;
+            if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
+                if (lane8 == 0) {
+                    float mx = a[0];
+#pragma unroll
+                    for (int h = 1; h < G; ++h) mx = fmaxf(mx, a[h]);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) acc += expf(a[h] - mx) * (1.f + 0.5f * c[h]);
+                    scores[size_t(kvu) * M + blk] = mx + logf(acc / float(G));
+                }
+            } else {
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    if ((h & 7) == lane8)
+                        scores[(size_t(b) * Hq + size_t(g) * G + h) * M + blk] = a[h] + log1pf(0.5f * c[h]);
+            }
+        }
+    }
+}
+
+// ============================================================================ block stats
+// One CTA of 128 threads per 64-token (or 32/128) block at a time: thread t holds 8
+// dims (one 16-byte chunk) of BLOCK*D/1024 rows in registers, so the two passes (mean,
+// then squared deviations) read HBM once.
+template <int D, int BLOCK>
+__global__ void __launch_bounds__(128)
+block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, float* __restrict__ mean,
+                   float* __restrict__ var) {
+    constexpr int DV = D / 8;                 // 16-byte chunks per row
+    constexpr int PH = 128 / DV;              // row phases
+    constexpr int RPT = BLOCK / PH;           // rows per thread
+    static_assert(RPT * PH == BLOCK, "block must be a multiple of the row phases");
+    __shared__ float red[PH][D];
+    __shared__ float mu_s[D];
+    const int c = threadIdx.x % DV;
+    const int ph = threadIdx.x / DV;
+
+    for (int blk = blockIdx.x; blk < n_blocks; blk += gridDim.x) {
+        const int unit = blk / nb_per_unit;
+        const int j = blk - unit * nb_per_unit;
+        const uint4* base = K + (size_t(unit) * N + size_t(j) * BLOCK) * DV + c;
+        uint4 w[RPT];
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) w[i] = __ldg(base + size_t(ph + i * PH) * DV);
+        float s[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s[2 * e] += bf_lo(ws[e]);
+                s[2 * e + 1] += bf_hi(ws[e]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[ph][c * 8 + e] = s[e];
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float t = 0.f;
+#pragma unroll
+            for (int p = 0; p < PH; ++p) t += red[p][threadIdx.x];
+            const float m = t / float(BLOCK);
+            mu_s[threadIdx.x] = m;
+            mean[size_t(blk) * D + threadIdx.x] = m;
+        }
+        __syncthreads();
+        float mv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { mv[e] = mu_s[c * 8 + e]; s[e] = 0.f; }
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float d0 = bf_lo(ws[e]) - mv[2 * e];
+                const float d1 = bf_hi(ws[e]) - mv[2 * e + 1];
+                s[2 * e] = fmaf(d0, d0, s[2 * e]);
+                s[2 * e + 1] = fmaf(d1, d1, s[2 * e + 1]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[ph][c * 8 + e] = s[e];
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float t = 0.f;
+#pragma unroll
+            for (int p = 0; p < PH; ++p) t += red[p][threadIdx.x];
+            var[size_t(blk) * D + threadIdx.x] = t / float(BLOCK);
+        }
+        __syncthreads();
+    }
+}
+
+int grid_for(int items, int per_sm) {
+    const int cap = device_info().num_sms * per_sm;
+    return items < cap ? (items > 0 ? items : 1) : cap;
+}
+
+}  // namespace
+
+spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
+                                 int collapse, float scale, float* scores, int* zero_ptr, int zero_count,
+                                 cudaStream_t st) {
+    const int G = Hq / Hkv;
+    const int chunks = (M + kLrChunk - 1) / kLrChunk;
+    const int items = B * Hkv * chunks;
+    const int grid = grid_for(items, 8);
+    const uint4* k4 = reinterpret_cast<const uint4*>(kidx);
+    if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
+        lowrank_scores_kernel<1><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores, chunks, items,
+                                                                zero_ptr, zero_count);
+    } else {
+        switch (G) {
+#define SPA_LR_CASE(n) \
+    case n: lowrank_scores_kernel<n><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores, chunks, items, zero_ptr, zero_count); break;
+            SPA_LR_CASE(1) SPA_LR_CASE(2) SPA_LR_CASE(4) SPA_LR_CASE(8) SPA_LR_CASE(16)
+#undef SPA_LR_CASE
+            default: return SPA_ERR_UNSUPPORTED_SHAPE;
+        }
+    }
+    SPA_CUDA_TRY(cudaGetLastError());
+    return SPA_OK;
+}
+
+spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
+                                int M, int d, int collapse, float scale, float* scores, int* zero_ptr,
+                                int zero_count, cudaStream_t st) {
+    const int G = Hq / Hkv;
+    const int chunks = (M + kTyChunk - 1) / kTyChunk;
+    const int items = B * Hkv * chunks;
+    const int grid = grid_for(items, 8);
+    const float4* m4 = reinterpret_cast<const float4*>(mean);
+    const float4* v4 = reinterpret_cast<const float4*>(var);
+#define SPA_TY_CASE(D, GG)                                                                                  \
+    if (d == D && G == GG) {                                                                               \
+        taylor_scores_kernel<D, GG><<<grid, kTyThreads, 0, st>>>(q, m4, v4, Hq, Hkv, M, collapse, scale, scores, \
+                                                                  chunks, items, zero_ptr, zero_count);   \
+        SPA_CUDA_TRY(cudaGetLastError());                                                                  \
+        return SPA_OK;                                                                                     \
+    }
+    SPA_TY_CASE(64, 1) SPA_TY_CASE(64, 2) SPA_TY_CASE(64, 4) SPA_TY_CASE(64, 8) SPA_TY_CASE(64, 16)
+    SPA_TY_CASE(128, 1) SPA_TY_CASE(128, 2) SPA_TY_CASE(128, 4) SPA_TY_CASE(128, 8) SPA_TY_CASE(128, 16)
+#undef SPA_TY_CASE
+    return SPA_ERR_UNSUPPORTED_SHAPE;
+}
+
+spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean,
+                              float* var, cudaStream_t st) {
+    const int nb = N / block;
+    const int n_blocks = B * Hkv * nb;
+    if (n_blocks == 0) return SPA_OK;
+    const int grid = grid_for(n_blocks, 16);
+    const uint4* k4 = reinterpret_cast<const uint4*>(K);
+#define SPA_BS_CASE(D, BL)                                                                       \
+    if (d == D && block == BL) {                                                                \
+        block_stats_kernel<D, BL><<<grid, 128, 0, st>>>(k4, n_blocks, nb, N, mean, var);        \
+        SPA_CUDA_TRY(cudaGetLastError());                                                       \
+        return SPA_OK;                                                                          \
+    }
+    SPA_BS_CASE(64, 32) SPA_BS_CASE(64, 64) SPA_BS_CASE(64, 128)
+    SPA_BS_CASE(128, 32) SPA_BS_CASE(128, 64) SPA_BS_CASE(128, 128)
+#undef SPA_BS_CASE
+    return SPA_ERR_UNSUPPORTED_SHAPE;
+}
+
+}  // namespace spa

@@ -1,0 +1,78 @@
+"""The C-ABI library loads, exports every entry point include/spa.h declares, and rejects
+bad arguments on the host (no GPU needed: validation precedes any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_sparse_spa_b200 as spa
+from long_context_sparse_spa_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(spa_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    L = spa.lib()
+    declared = _declared()
+    assert declared, "no declarations found"
+    for name in sorted(declared):
+        assert hasattr(L, name), f"{name} missing from libspa.so"
+        assert name in _abi.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_status_strings_and_version():
+    L = spa.lib()
+    assert L.spa_abi_version() == 1
+    assert L.spa_status_string(_abi.SPA_ERR_CAPACITY) == b"SPA_ERR_CAPACITY"
+    assert L.spa_status_string(99) == b"SPA_ERR_UNKNOWN"
+
+
+def test_host_validation():
+    L = spa.lib()
+    P = ctypes.c_void_p(16)   # never dereferenced: every call below fails validation first
+    # negative sizes
+    assert L.spa_select_topk(P, None, -1, 10, 1, 0, 0, P, P, 1, P, 256, None) == _abi.SPA_ERR_INVALID_ARG
+    # workspace too small
+    assert L.spa_select_topk(P, None, 2, 10, 1, 0, 0, P, P, 1, P, 8, None) == _abi.SPA_ERR_WORKSPACE_TOO_SMALL
+    # p outside (0, 1]
+    assert L.spa_select_topp(P, None, 2, 10, ctypes.c_float(0.0), 0, 0, P, P, 10, None, P, 256, None) == \
+        _abi.SPA_ERR_INVALID_ARG
+    assert L.spa_select_topp(P, None, 2, 10, ctypes.c_float(1.5), 0, 0, P, P, 10, None, P, 256, None) == \
+        _abi.SPA_ERR_INVALID_ARG
+    # unsupported index dim / head dim / group size
+    assert L.spa_index_scores(0, P, P, None, 1, 4, 1, 10, 32, 0, ctypes.c_float(1.0), P, None) == \
+        _abi.SPA_ERR_UNSUPPORTED_SHAPE
+    assert L.spa_index_scores(0, P, P, None, 1, 64, 2, 10, 16, 1, ctypes.c_float(1.0), P, None) == \
+        _abi.SPA_ERR_UNSUPPORTED_SHAPE
+    assert L.spa_block_stats(P, 1, 1, 128, 96, 64, P, P, None) == _abi.SPA_ERR_UNSUPPORTED_SHAPE
+    # misaligned bf16 pointer
+    assert L.spa_block_stats(ctypes.c_void_p(18), 1, 1, 128, 128, 64, P, P, None) == _abi.SPA_ERR_UNSUPPORTED_SHAPE
+    # Hq not a multiple of Hkv
+    assert L.spa_sparse_attend(P, P, P, 1, 6, 4, 100, 128, P, P, 1, 1, 1, ctypes.c_float(1.0), P, None, None,
+                               P, 1 << 30, None) == _abi.SPA_ERR_INVALID_ARG
+    # empty problems are no-ops
+    assert L.spa_select_topk(None, None, 0, 10, 1, 0, 0, None, None, 1, None, 0, None) == _abi.SPA_OK
+    assert L.spa_block_stats(None, 0, 1, 128, 128, 64, None, None, None) == _abi.SPA_OK
+
+
+def test_decode_validation():
+    a = _abi.SpaDecodeArgs()
+    a.B, a.Hq, a.Hkv, a.N, a.d, a.r, a.block = 1, 8, 1, 1000, 128, 16, 1
+    a.select_kind = _abi.SPA_SELECT_TOPP
+    a.topp = 0.0
+    L = spa.lib()
+    need = L.spa_decode_workspace_bytes(ctypes.byref(a))
+    assert need > 1000 * 4
+    assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(16), 10, None) == _abi.SPA_ERR_WORKSPACE_TOO_SMALL
+    assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(16), need, None) == _abi.SPA_ERR_INVALID_ARG

@@ -1,0 +1,95 @@
+"""Fused decode (spa_decode: scores -> selection -> attention) against the fp64 oracle.
+
+Small workloads compare every output; the full-size workloads compare every support and
+every output too (the oracle's sparse path is cheap enough), run in the launch
+configuration the bench times.  Captured mass and sparsity are reported per workload.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from parity import (MASS_TIE_REL, OUT_TOL, check_outputs, compare_support, dev, dev_bf16, topk_band, topp_band)
+from synth import C1, C2, C2_128K, C3, C4, SMALL, decode_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import long_context_sparse_spa_b200 as spa  # noqa: E402
+
+
+def run_gpu(cfg, x):
+    lowrank = cfg.score == "lowrank"
+    kw = dict(
+        score_kind=spa.SPA_SCORE_LOWRANK if lowrank else spa.SPA_SCORE_TAYLOR_BLOCK,
+        select_kind=spa.SPA_SELECT_TOPK if cfg.select == "topk" else spa.SPA_SELECT_TOPP,
+        collapse=spa.SPA_COLLAPSE_GROUP_MEAN if cfg.collapse == "group" else spa.SPA_COLLAPSE_NONE,
+        q=dev_bf16(x["q"]), K=dev_bf16(x["K"]), V=dev_bf16(x["V"]), block=cfg.block,
+        score_scale=oracle.f32(cfg.score_scale), sm_scale=oracle.f32(cfg.sm_scale),
+        topk=cfg.topk, topp=cfg.topp, sink=cfg.sink, window=cfg.window, cap=cfg.cap)
+    if lowrank:
+        kw.update(q_idx=dev_bf16(x["q_idx"]), Kidx=dev_bf16(x["Kidx"]))
+    else:
+        mean, var = spa.block_stats(kw["K"], cfg.block)   # off the per-step path: once per filled block
+        kw.update(bmean=mean, bvar=var)
+    plan = spa.decode(**kw)
+    torch.cuda.synchronize()
+    assert spa.read_device_status(plan.ws) == 0
+    res = dict(idx=plan.idx.cpu().numpy(), count=plan.count.cpu().numpy(),
+               out=plan.out.view(torch.int16).cpu().numpy().view(np.uint16), out32=plan.out_f32.cpu().numpy(),
+               lse=plan.lse.cpu().numpy(),
+               mass=plan.index_mass.cpu().numpy() if plan.index_mass is not None else None)
+    del plan, kw
+    torch.cuda.empty_cache()
+    return res
+
+
+def check_decode(cfg, report_mass=False):
+    x = decode_inputs(cfg)
+    g = run_gpu(cfg, x)
+    G = cfg.G
+    ties = 0
+    worst = 0.0
+    sparsity, captured = [], []
+    for u, (b, h) in enumerate(oracle.decode_units(cfg)):
+        r = oracle.decode_unit(cfg, x, u)   # the oracle computes its own (fp64) block statistics
+        s = r["ranked"]
+        band = topk_band(s, cfg.topk) if cfg.select == "topk" else topp_band(s, oracle.f32(cfg.topp))
+        got = g["idx"][u, :g["count"][u]]
+        d = compare_support(got, r["idx"], band, f"{cfg.name} unit {u}")
+        ties += d
+        heads = slice(h, h + 1) if cfg.collapse == "head" else slice(h * G, (h + 1) * G)
+        if d == 0:
+            worst = max(worst, check_outputs(g["out"][b, heads], g["out32"][b, heads], r["out"],
+                                             f"{cfg.name} unit {u}"))
+            np.testing.assert_allclose(g["lse"][b, heads], r["lse"], rtol=2e-6, atol=2e-6)
+            if g["mass"] is not None:
+                assert abs(g["mass"][u] - r["index_mass"]) <= 4 * MASS_TIE_REL + 1e-6
+        else:
+            print(f"{cfg.name} unit {u}: {d} tie differences; output compared on the oracle's rerun of "
+                  "the GPU's ranked prefix is not asserted")
+        sparsity.append(1 - got.size / cfg.M)
+        if report_mass and u < 4:
+            captured.append(oracle.captured_mass(cfg, x, u, got))
+    msg = f"{cfg.name}: max|err| {worst:.2e}, tie differences {ties}, sparsity mean {np.mean(sparsity):.4f}"
+    if captured:
+        msg += f", captured mass (first units) {np.round(captured, 4).tolist()}"
+    print(msg)
+    return worst
+
+
+@pytest.mark.parametrize("name", ["c1s", "c2s", "c3s", "c4s"])
+def test_decode_small(name):
+    check_decode(SMALL[name])
+
+
+def test_decode_c1():
+    check_decode(C1, report_mass=True)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [C2, C2_128K, C3, C4], ids=lambda c: c.name)
+def test_decode_full_size(cfg):
+    check_decode(cfg, report_mass=True)
