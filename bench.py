@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Sparse-decode benchmark on B200: the fused top-p decode step at a 128K-token KV cache.
+
+One step = one pass of the whole decode path (low-rank index scores over all cached keys
+-> histogram top-p selection with sink and window -> exact attention on the gathered K/V
+rows -> log-sum-exp combine) for a batch of B=4 sequences x 32 query heads (8 per kv
+head), N = 131072 cached tokens, d = 128, r = 16, p = 0.9, sink 4, window 128.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spa|reference]
+
+Prints ONE JSON line on rank 0.  ``value`` is the whole-job decode throughput in query
+heads per second; the L2 is flushed (256 MiB write) before every step and each step is
+timed on the device with CUDA events; the multi-GPU figure divides the units all ranks
+processed by the max over ranks of the device time.  ``--impl reference`` times the fp64
+CPU oracle on the same workload (rank 0 only).  Extra detail goes to stderr.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import DECODE_CONFIGS, decode_inputs  # noqa: E402
+
+METRIC = "sparse-decode queries/s (query heads per second), 128K-token KV cache"
+UNIT = "queries/s"
+L2_FLUSH_BYTES = 256 << 20
+KV_ROW_BYTES = lambda d: 2 * d * 2          # K + V row, bf16
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
+    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = 3000 if a.impl == "spa" else 20
+    if a.warmup is None:
+        a.warmup = 50 if a.impl == "spa" else 3
+    return a
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: {cfg.select} decode, {cfg.score} scores, collapse={cfg.collapse}, B={cfg.B} Hq={cfg.Hq} "
+            f"Hkv={cfg.Hkv} d={cfg.d} r={cfg.r} N={cfg.N} p={cfg.topp} k={cfg.topk} sink={cfg.sink} "
+            f"window={cfg.window}")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (profiles/traffic.tsv: kernel, workload, bytes, source sha256 prefix)."""
+    path = os.path.join(ROOT, "profiles", "traffic.tsv")
+    src = os.path.join(ROOT, "long_context_sparse_spa_b200", "csrc", "attend.cu" if kernel == "attend" else
+                       ("scores.cu" if kernel == "scores" else "select.cu"))
+    if not os.path.exists(path) or not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        f = line.strip().split("\t")
+        if len(f) == 4 and f[0] == kernel and f[1] == workload and f[3] == sha:
+            return float(f[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                x = [c.strip() for c in line.split(",")]
+                if len(x) >= 9:
+                    rows.append(x)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(cfg, x, seconds: float):
+    """The fp64 oracle's sparse path (scores -> selection -> attention), as it stands, on the
+    host cores: units of the same workload cycled until the time budget is spent."""
+    import oracle
+
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    units = list(range(cfg.U))
+    done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:      # whole rounds over all units
+        oracle.decode(cfg, x, units=units, threads=cores)
+        done += len(units)
+    dt = time.perf_counter() - t0
+    return {"value": done * cfg.heads_per_unit / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} units (one kv head of one sequence each, {cfg.heads_per_unit} query heads) of "
+                      f"{cfg.name}, fp64 oracle, {dt:.1f} s"}
+
+
+# ============================================================================ reference arm
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = DECODE_CONFIGS[a.config]
+    import oracle
+
+    x = decode_inputs(cfg)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    # one step = one unit (a kv head of one sequence: its index scores over all N keys,
+    # the top-p cut and exact attention for its query heads), cycling over the units
+    for i in range(a.warmup):
+        oracle.decode_unit(cfg, x, i % cfg.U)
+    t0 = time.perf_counter()
+    for i in range(a.steps):
+        oracle.decode_unit(cfg, x, i % cfg.U)
+    dt = time.perf_counter() - t0
+    value = a.steps * cfg.heads_per_unit / dt
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_desc(cfg), "sample": "one unit per step, cycling over the units"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{a.steps} units of {cfg.name}, one per step, single thread "
+                                       f"({cores} cores available)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ============================================================================ our arm
+def run_spa(a):
+    import torch
+    import torch.distributed as dist
+
+    import long_context_sparse_spa_b200 as spa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != a.gpus:
+        log(f"note: --gpus {a.gpus} but WORLD_SIZE {world}; using WORLD_SIZE")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    base = DECODE_CONFIGS[a.config]
+    # weak scaling: every rank holds its own B sequences (a shard of a global batch of world*B)
+    cfg_global = base.with_(B=base.B * world)
+    t = time.perf_counter()
+    x = decode_inputs(cfg_global, batch=(rank * base.B, (rank + 1) * base.B))
+    log(f"[rank {rank}] inputs generated in {time.perf_counter() - t:.1f} s")
+
+    def up(arr):
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
+
+    cfg = base
+    lowrank = cfg.score == "lowrank"
+    dq, dK, dV = up(x["q"]), up(x["K"]), up(x["V"])
+    kw = dict(score_kind=spa.SPA_SCORE_LOWRANK if lowrank else spa.SPA_SCORE_TAYLOR_BLOCK,
+              select_kind=spa.SPA_SELECT_TOPP if cfg.select == "topp" else spa.SPA_SELECT_TOPK,
+              collapse=spa.SPA_COLLAPSE_GROUP_MEAN if cfg.collapse == "group" else spa.SPA_COLLAPSE_NONE,
+              q=dq, K=dK, V=dV, block=cfg.block, score_scale=float(np.float32(cfg.score_scale)),
+              sm_scale=float(np.float32(cfg.sm_scale)), topk=cfg.topk, topp=cfg.topp, sink=cfg.sink,
+              window=cfg.window, cap=cfg.cap, want_f32=False, want_lse=False, run=False)
+    if lowrank:
+        dqi, dKi = up(x["q_idx"]), up(x["Kidx"])
+        kw.update(q_idx=dqi, Kidx=dKi)
+    else:
+        bm, bv = spa.block_stats(dK, cfg.block)      # once per filled block, off the per-step path
+        kw.update(bmean=bm, bvar=bv)
+    plan = spa.decode(**kw)
+    wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+
+    def flush_l2():
+        # write a buffer larger than L2, then read another one so that the dirty lines are
+        # written back here and not during the next timed step
+        wbuf.zero_()
+        rbuf.sum()
+
+    for _ in range(a.warmup):
+        flush_l2()
+        plan.run()
+    torch.cuda.synchronize()
+    assert spa.read_device_status(plan.ws) == 0, "device status raised during warm-up"
+    counts = plan.count.cpu().numpy().astype(np.int64)
+    rows = int(counts.sum()) * cfg.block
+    M = cfg.N // cfg.block
+    sparsity = 1.0 - counts.sum() / (cfg.U * M)
+
+    # ---- timed region: K steps, L2 flushed before each, per-kernel events inside each step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    for e4 in ev:
+        for e in e4:
+            e.record()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    for i in range(a.steps):
+        flush_l2()
+        plan.run_timed(ev[i])
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = np.array([ev[i][0].elapsed_time(ev[i][3]) for i in range(a.steps)])
+    k_ms = {name: np.array([ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(a.steps)])
+            for j, name in enumerate(("scores", "select", "attend"))}
+    dev_s = float(step_ms.sum()) / 1e3
+    t_max = dev_s
+    if world > 1:
+        tt = torch.tensor([dev_s], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    queries = cfg.B * cfg.Hq * a.steps * world
+    value = queries / t_max
+
+    # ---- algorithmic bytes (what the chosen support must move)
+    d = cfg.d
+    if lowrank:
+        score_bytes = cfg.B * cfg.Hkv * cfg.N * cfg.r * 2 + cfg.B * cfg.Hq * cfg.r * 2
+    else:
+        score_bytes = 2 * cfg.B * cfg.Hkv * M * d * 4 + cfg.B * cfg.Hq * d * 2
+    attend_bytes = rows * KV_ROW_BYTES(d) + 2 * cfg.B * cfg.Hq * d * 2
+    step_bytes = score_bytes + attend_bytes
+    peak, peak_kind = peaks()
+    mean_ms = {k: float(v.mean()) for k, v in k_ms.items()}
+    kbytes = {"scores": score_bytes, "attend": attend_bytes, "select": 0}
+    dom = max(("scores", "attend"), key=lambda k: mean_ms[k])
+    achieved = kbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": peak_kind,
+                "traffic": recorded_traffic(dom, cfg.name),
+                "step_achieved": step_bytes / (float(step_ms.mean()) * 1e-3) / 1e9,
+                "step_frac": step_bytes / (float(step_ms.mean()) * 1e-3) / 1e9 / peak}
+    roofline["algorithmic_bytes_per_launch"] = kbytes[dom]
+
+    # ---- end to end through the public API with host buffers
+    n_e2e = min(a.steps, 200)
+    hq = x["q"].view(np.int16)
+    pin_q = torch.from_numpy(np.ascontiguousarray(hq)).pin_memory()
+    h2d = pin_q.numel() * 2
+    pin_qi = None
+    if lowrank:
+        pin_qi = torch.from_numpy(np.ascontiguousarray(x["q_idx"].view(np.int16))).pin_memory()
+        h2d += pin_qi.numel() * 2
+    out_h = torch.empty(plan.out.shape, dtype=torch.bfloat16).pin_memory()
+    cnt_h = torch.empty(plan.count.shape, dtype=torch.int32).pin_memory()
+    d2h = out_h.numel() * 2 + cnt_h.numel() * 4
+    e2e_ms = []
+    for i in range(n_e2e + 3):
+        flush_l2()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        dq.view(torch.int16).copy_(pin_q, non_blocking=True)
+        if pin_qi is not None:
+            dqi.view(torch.int16).copy_(pin_qi, non_blocking=True)
+        plan.run()
+        out_h.copy_(plan.out, non_blocking=True)
+        cnt_h.copy_(plan.count, non_blocking=True)
+        s1.record()
+        s1.synchronize()
+        if i >= 3:
+            e2e_ms.append(s0.elapsed_time(s1))
+    e2e_local = float(np.sum(e2e_ms)) / 1e3
+    if world > 1:
+        tt = torch.tensor([e2e_local], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_local = float(tt.item())
+    e2e_value = cfg.B * cfg.Hq * n_e2e * world / e2e_local
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": float(step_ms.mean()), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "seq_len": cfg.N,
+                       "parallelism": f"dp{world} (independent sequence shards, no collective on the data path)",
+                       "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
+                       "support_rows_per_step": rows, "sparsity": round(float(sparsity), 4),
+                       "algorithmic_bytes_per_step": step_bytes},
+            "roofline": roofline,
+            "kernels_ms": {k: round(v, 5) for k, v in mean_ms.items()},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": float(np.mean(e2e_ms))},
+            "gpu_launches": 3 * a.steps,
+            "clocks": clocks,
+            "wall_s_timed_region": w1 - w0,
+        }
+        if not a.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(cfg, x, a.cpu_seconds)
+        elif world > 1:
+            line["cpu_baseline"] = None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_spa(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -211,6 +211,12 @@ typedef struct spa_decode_args {
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream);
 size_t spa_decode_workspace_bytes(const spa_decode_args* a);
 
+/* spa_decode that also records four caller-created cudaEvent_t on `stream`: events[0]
+ * before the scoring kernel, events[1] after it, events[2] after the selection kernel and
+ * events[3] after the attention kernel, so a caller can time each kernel inside a real step. */
+spa_status spa_decode_timed(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
+                            void* const* events);
+
 /* ------------------------------------------------------------------------------------
  * Device status word of a workspace (sticky OR of SPA_ERR_* bits as (1 << code)).
  * Synchronises `stream`, copies the word to *bits and, if reset != 0, clears it.

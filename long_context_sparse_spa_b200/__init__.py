@@ -169,6 +169,13 @@ class DecodePlan:
         check(lib().spa_decode(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
                                _stream(stream)))
 
+    def run_timed(self, events, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """run() recording four torch.cuda.Event (enable_timing=True, already recorded once so that
+        they exist) before scoring, after scoring, after selection and after attention."""
+        handles = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        check(lib().spa_decode_timed(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()),
+                                     self.ws.numel(), _stream(stream), handles))
+
 
 def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor, K: torch.Tensor,
            V: torch.Tensor, q_idx: Optional[torch.Tensor] = None, Kidx: Optional[torch.Tensor] = None,

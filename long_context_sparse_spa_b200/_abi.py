@@ -58,6 +58,7 @@ SIGNATURES = {
     "spa_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spa_decode": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p]),
     "spa_decode_workspace_bytes": (_sz, [ctypes.POINTER(SpaDecodeArgs)]),
+    "spa_decode_timed": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p, ctypes.POINTER(_p)]),
     "spa_read_device_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32), _i]),
 }
 

@@ -98,22 +98,21 @@ spa_status spa_index_scores(int kind, const void* q, const void* keys, const flo
         if (dim != 16) return SPA_ERR_UNSUPPORTED_SHAPE;
         if (!aligned16(q) || !aligned16(keys)) return SPA_ERR_UNSUPPORTED_SHAPE;
         return launch_lowrank_scores(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(keys), B, Hq, Hkv,
-                                     M, collapse, scale, scores, nullptr, 0, st);
+                                     M, collapse, scale, scores, nullptr, false, st);
     }
     if (kind == SPA_SCORE_TAYLOR_BLOCK) {
         if (!var) return SPA_ERR_INVALID_ARG;
         if (dim != 64 && dim != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
         if (!aligned16(keys) || !aligned16(var)) return SPA_ERR_UNSUPPORTED_SHAPE;
         return launch_taylor_scores(static_cast<const uint16_t*>(q), static_cast<const float*>(keys), var, B, Hq,
-                                    Hkv, M, dim, collapse, scale, scores, nullptr, 0, st);
+                                    Hkv, M, dim, collapse, scale, scores, st);
     }
     return SPA_ERR_INVALID_ARG;
 }
 
 size_t spa_select_workspace_bytes(int U, int M) {
-    (void)U;
     (void)M;
-    return kWsHeader;
+    return U < 0 ? 0 : kWsHeader + select_scratch_bytes(U);
 }
 
 static spa_status select_common(const float* scores, const int32_t* unit_len, int U, int M, int sink, int window,
@@ -132,9 +131,12 @@ spa_status spa_select_topk(const float* scores, const int32_t* unit_len, int U, 
     spa_status s = select_common(scores, unit_len, U, M, sink, window, idx, count, cap, ws, ws_bytes);
     if (s != SPA_OK || U == 0) return s;
     if (k < 0) return SPA_ERR_INVALID_ARG;
-    SelectParams p{scores, unit_len, U, M, k, 0.f, sink, window, idx, count, cap, nullptr,
-                   static_cast<uint32_t*>(ws)};
-    return launch_select(p, false, static_cast<cudaStream_t>(stream));
+    SelectParams p{hist0_carve(static_cast<uint8_t*>(ws) + kWsHeader, U), scores, unit_len, U, M, k, 0.f, sink,
+                   window, idx, count, cap, nullptr, static_cast<uint32_t*>(ws)};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = launch_hist0(p, false, st);
+    if (s != SPA_OK) return s;
+    return launch_select(p, false, st);
 }
 
 spa_status spa_select_topp(const float* scores, const int32_t* unit_len, int U, int M, float p, int sink,
@@ -144,9 +146,12 @@ spa_status spa_select_topp(const float* scores, const int32_t* unit_len, int U, 
     if (s != SPA_OK || U == 0) return s;
     if (!(p > 0.f && p <= 1.f)) return SPA_ERR_INVALID_ARG;
     if (M > (1 << 23)) return SPA_ERR_UNSUPPORTED_SHAPE;
-    SelectParams sp{scores, unit_len, U, M, 0, p, sink, window, idx, count, cap, index_mass,
-                    static_cast<uint32_t*>(ws)};
-    return launch_select(sp, true, static_cast<cudaStream_t>(stream));
+    SelectParams sp{hist0_carve(static_cast<uint8_t*>(ws) + kWsHeader, U), scores, unit_len, U, M, 0, p, sink,
+                    window, idx, count, cap, index_mass, static_cast<uint32_t*>(ws)};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = launch_hist0(sp, true, st);
+    if (s != SPA_OK) return s;
+    return launch_select(sp, true, st);
 }
 
 size_t spa_attend_workspace_bytes(int B, int Hq, int Hkv, int d, int collapse) {
@@ -175,8 +180,8 @@ static spa_status attend_params(const uint16_t* q, const uint16_t* K, const uint
     p.idx = idx; p.count = count; p.cap = cap; p.collapse = collapse; p.unit_tokens = unit_tokens;
     p.sm_scale = sm_scale; p.out = out; p.out_f32 = out_f32; p.lse = lse;
     p.status = reinterpret_cast<uint32_t*>(w);
-    p.tickets = reinterpret_cast<int*>(w + kWsHeader);
-    p.partials = reinterpret_cast<float*>(w + kWsHeader + align_up(size_t(U) * 4, 256));
+    p.unit_ctas = reinterpret_cast<int*>(w + kWsHeader);
+    p.partials = reinterpret_cast<float*>(w + kWsHeader + align_up(size_t(U) * 8, 256));
     return SPA_OK;
 }
 
@@ -194,12 +199,28 @@ spa_status spa_sparse_attend(const uint16_t* q, const uint16_t* K, const uint16_
 
 size_t spa_decode_workspace_bytes(const spa_decode_args* a) {
     if (!a || bad_dims(a->B, a->Hq, a->Hkv)) return 0;
-    return kWsHeader + decode_scores_bytes(a) + attend_scratch_bytes(
-        a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->B * a->Hkv : a->B * a->Hq,
-        a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->Hq / a->Hkv : 1, a->d);
+    const int U = a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->B * a->Hkv : a->B * a->Hq;
+    return kWsHeader + decode_scores_bytes(a) + select_scratch_bytes(U) +
+           attend_scratch_bytes(U, a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->Hq / a->Hkv : 1, a->d);
 }
 
+static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
+                              void* const* events);
+
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream) {
+    return decode_impl(a, ws, ws_bytes, stream, nullptr);
+}
+
+spa_status spa_decode_timed(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
+                            void* const* events) {
+    if (!events) return SPA_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i)
+        if (!events[i]) return SPA_ERR_INVALID_ARG;
+    return decode_impl(a, ws, ws_bytes, stream, events);
+}
+
+static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
+                              void* const* events) {
     if (!a || !ws) return SPA_ERR_INVALID_ARG;
     if (bad_dims(a->B, a->Hq, a->Hkv) || a->N < 0) return SPA_ERR_INVALID_ARG;
     if (a->B == 0) return SPA_OK;
@@ -236,7 +257,12 @@ spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void*
     uint8_t* w = static_cast<uint8_t*>(ws);
     uint32_t* status = reinterpret_cast<uint32_t*>(w);
     float* scores = reinterpret_cast<float*>(w + kWsHeader);
-    uint8_t* attend_ws = w + kWsHeader + decode_scores_bytes(a);
+    const Hist0 hist = hist0_carve(w + kWsHeader + decode_scores_bytes(a), U);
+    uint8_t* attend_ws = w + kWsHeader + decode_scores_bytes(a) + select_scratch_bytes(U);
+    const bool topp = a->select_kind == SPA_SELECT_TOPP;
+    // the level-0 selection histogram is built inside the scoring kernel when it produces
+    // one score row per kv head (low-rank, GROUP_MEAN); otherwise by a histogram kernel
+    const bool fused_hist = !taylor && group;
 
     // attention parameters first: they validate q/K/V/idx/out and carve the workspace
     AttendParams ap;
@@ -244,27 +270,38 @@ spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void*
                                  a->collapse, block, a->sm_scale, a->out, a->out_f32, a->lse, ws,
                                  size_t(-1), ap);
     if (s != SPA_OK) return s;
-    ap.tickets = reinterpret_cast<int*>(attend_ws);
-    ap.partials = reinterpret_cast<float*>(attend_ws + align_up(size_t(U) * 4, 256));
+    ap.unit_ctas = reinterpret_cast<int*>(attend_ws);
+    ap.partials = reinterpret_cast<float*>(attend_ws + align_up(size_t(U) * 8, 256));
 
-    // 1. scores (the scoring kernel also zeroes the attention tickets)
+    auto mark = [&](int i) -> spa_status {
+        if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st));
+        return SPA_OK;
+    };
+
+    // 1. scores
+    if ((s = mark(0)) != SPA_OK) return s;
     if (taylor) {
         s = launch_taylor_scores(a->q, a->bmean, a->bvar, a->B, a->Hq, a->Hkv, M, a->d, a->collapse,
-                                 a->score_scale, scores, ap.tickets, U, st);
+                                 a->score_scale, scores, st);
     } else {
         s = launch_lowrank_scores(a->q_idx, a->Kidx, a->B, a->Hq, a->Hkv, M, a->collapse, a->score_scale, scores,
-                                  ap.tickets, U, st);
+                                  fused_hist ? &hist : nullptr, topp, st);
     }
     if (s != SPA_OK) return s;
 
     // 2. selection
-    SelectParams sp{scores, nullptr, U, M, a->topk, a->topp, a->sink, a->window, a->idx, a->count, a->cap,
+    SelectParams sp{hist, scores, nullptr, U, M, a->topk, a->topp, a->sink, a->window, a->idx, a->count, a->cap,
                     a->index_mass, status};
-    s = launch_select(sp, a->select_kind == SPA_SELECT_TOPP, st);
+    if (!fused_hist && (s = launch_hist0(sp, topp, st)) != SPA_OK) return s;
+    if ((s = mark(1)) != SPA_OK) return s;
+    s = launch_select(sp, topp, st);
     if (s != SPA_OK) return s;
+    if ((s = mark(2)) != SPA_OK) return s;
 
     // 3. attention on the gathered rows
-    return launch_attend(ap, st);
+    s = launch_attend(ap, st);
+    if (s != SPA_OK) return s;
+    return mark(3);
 }
 
 spa_status spa_read_device_status(void* ws, void* stream, uint32_t* bits, int reset) {

@@ -21,8 +21,9 @@
 //   CUDA cores its 8 flops per byte would bound the kernel well below HBM speed.
 //
 // At the end of its share of a unit a CTA merges its warps' (m, l, o) in shared memory.
-// A CTA holding a whole unit writes the output; otherwise it stores a partial, and the
-// last CTA to finish the unit (atomic ticket) merges the partials and writes the output.
+// A CTA holding a whole unit writes the output; otherwise it stores a partial (o, m, l),
+// and a second kernel, one CTA per (unit, head) with eight warps splitting the unit's
+// partials, merges them in a fixed order (log-sum-exp combine) and writes the output.
 #include "internal.cuh"
 
 namespace spa {
@@ -119,7 +120,6 @@ attend_kernel(AttendParams p, int U, int nh) {
     int* s_prefix = reinterpret_cast<int*>(smem);                            // [U + 1]
     uint8_t* ring = smem + align_up(size_t(U + 1) * 4, 128);
     __shared__ uint32_t s_vmask[kAtWarps][kStages];
-    __shared__ int s_last;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gq = lane >> 2, cq = lane & 3;   // mma fragment coordinates
@@ -155,10 +155,13 @@ attend_kernel(AttendParams p, int U, int nh) {
     if (tid == 0) s_prefix[U] = running;
     __syncthreads();
     const long long TT = running;
-    const int G = gridDim.x, cta = blockIdx.x;
+    const int cta = blockIdx.x;
+    // Tiles are split over G = min(grid, TT) CTAs so that every range is non-empty (the
+    // partial accounting counts CTAs); the rest only serve empty supports.
+    const int G = int(TT < (long long)gridDim.x ? TT : (long long)gridDim.x);
 
     // ---- empty supports: out = 0, lse = -inf
-    for (int u = cta; u < U; u += G) {
+    for (int u = cta; u < U; u += gridDim.x) {
         if (s_prefix[u + 1] != s_prefix[u]) continue;
         const UnitGeom ug = unit_geom(p, u, nh);
         for (int i = tid; i < nh * D; i += kAtThreads) {
@@ -169,8 +172,22 @@ attend_kernel(AttendParams p, int U, int nh) {
         }
     }
 
+    // CTA range of every unit, for the combine kernel: (first, last) CTA, or (-1, -1)
+    // when one CTA (or none) produced the whole output
+    if (cta == 0) {
+        for (int v = tid; v < U; v += kAtThreads) {
+            int lo = -1, hi = -1;
+            if (s_prefix[v + 1] > s_prefix[v]) {
+                lo = tile_owner(s_prefix[v], TT, G);
+                hi = tile_owner(s_prefix[v + 1] - 1, TT, G);
+                if (lo == hi) lo = hi = -1;
+            }
+            p.unit_ctas[2 * v] = lo;
+            p.unit_ctas[2 * v + 1] = hi;
+        }
+    }
+    if (cta >= G) return;
     const long long t0 = TT * cta / G, t1 = TT * (cta + 1) / G;
-    if (t0 >= t1) return;
 
     // first unit of the range: last u with prefix[u] <= t0 (empty units are skipped)
     int u;
@@ -388,47 +405,68 @@ attend_kernel(AttendParams p, int U, int nh) {
                 }
             }
         }
-        if (!whole) {
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) {
-                const int c_lo = tile_owner(s_prefix[u], TT, G);
-                const int c_hi = tile_owner(s_prefix[u + 1] - 1, TT, G);
-                const int ticket = atomicAdd(&p.tickets[u], 1);
-                s_last = ticket == c_hi - c_lo;
-                if (s_last) p.tickets[u] = 0;
-            }
-            __syncthreads();
-            if (s_last) {
-                __threadfence();
-                const int c_lo = tile_owner(s_prefix[u], TT, G);
-                const int c_hi = tile_owner(s_prefix[u + 1] - 1, TT, G);
-                for (int i = tid; i < nh * D; i += kAtThreads) {
-                    const int row = i / D, col = i - row * D;
-                    float M = -INFINITY;
-                    for (int c = c_lo; c <= c_hi; ++c)
-                        M = fmaxf(M, __ldcg(p.partials + (size_t(u + c) * nh + row) * (D + 2) + D));
-                    const float Mr = M == -INFINITY ? 0.f : M;
-                    float L = 0.f, O = 0.f;
-                    for (int c = c_lo; c <= c_hi; ++c) {
-                        const float* pp = p.partials + (size_t(u + c) * nh + row) * (D + 2);
-                        const float sc = exp2f(__ldcg(pp + D) - Mr);
-                        L += __ldcg(pp + D + 1) * sc;
-                        O += __ldcg(pp + col) * sc;
-                    }
-                    const size_t o = (size_t(ug.b) * p.Hq + ug.h0 + row) * D + col;
-                    const float val = L > 0.f ? O / L : 0.f;
-                    const __nv_bfloat16 bv = __float2bfloat16_rn(val);
-                    p.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
-                    if (p.out_f32) p.out_f32[o] = val;
-                    if (p.lse && col == 0)
-                        p.lse[size_t(ug.b) * p.Hq + ug.h0 + row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-                }
-            }
-        }
         __syncthreads();   // rings are reused by the next segment
         x = seg_end;
     }
+}
+
+// Log-sum-exp combine of the partials of every unit split over several CTAs.
+// grid (U, heads per unit), 256 threads: warp w merges partials c_lo + w, c_lo + w + 8, ...
+// online (running max, rescaled sums); the eight warp results are merged in warp order.
+template <int D>
+__global__ void __launch_bounds__(256)
+combine_kernel(AttendParams p, int nh) {
+    constexpr int CPL = D / 32;    // columns per lane
+    const int u = blockIdx.x, row = blockIdx.y;
+    const int c_lo = p.unit_ctas[2 * u], c_hi = p.unit_ctas[2 * u + 1];
+    if (c_lo < 0 || row >= nh) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float M = -INFINITY, L = 0.f, O[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) O[j] = 0.f;
+    for (int c = c_lo + warp; c <= c_hi; c += 8) {
+        const float* pp = p.partials + (size_t(u + c) * nh + row) * (D + 2);
+        const float m = __ldcg(pp + D), l = __ldcg(pp + D + 1);
+        float v[CPL];
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) v[j] = __ldcg(pp + lane * CPL + j);
+        const float Mn = fmaxf(M, m);
+        if (Mn == -INFINITY) continue;
+        const float a = exp2f(M - Mn), b = exp2f(m - Mn);
+        L = L * a + l * b;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) O[j] = O[j] * a + v[j] * b;
+        M = Mn;
+    }
+    __shared__ float sM[8], sL[8], sO[8][D];
+    if (lane == 0) { sM[warp] = M; sL[warp] = L; }
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) sO[warp][lane * CPL + j] = O[j];
+    __syncthreads();
+    if (warp != 0) return;
+    float Mt = -INFINITY;
+    for (int w = 0; w < 8; ++w) Mt = fmaxf(Mt, sM[w]);
+    const float Mr = Mt == -INFINITY ? 0.f : Mt;
+    float Lt = 0.f, Ot[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) Ot[j] = 0.f;
+    for (int w = 0; w < 8; ++w) {
+        const float sc = exp2f(sM[w] - Mr);
+        Lt += sL[w] * sc;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) Ot[j] += sO[w][lane * CPL + j] * sc;
+    }
+    const UnitGeom ug = unit_geom(p, u, nh);
+    const size_t ob = (size_t(ug.b) * p.Hq + ug.h0 + row) * D;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        const float val = Lt > 0.f ? Ot[j] / Lt : 0.f;
+        const __nv_bfloat16 bv = __float2bfloat16_rn(val);
+        p.out[ob + lane * CPL + j] = *reinterpret_cast<const uint16_t*>(&bv);
+        if (p.out_f32) p.out_f32[ob + lane * CPL + j] = val;
+    }
+    if (p.lse && lane == 0)
+        p.lse[size_t(ug.b) * p.Hq + ug.h0 + row] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
 }
 
 template <int D>
@@ -441,9 +479,9 @@ size_t attend_smem(int U) {
 int attend_grid() { return device_info().num_sms * 2; }
 
 size_t attend_scratch_bytes(int U, int heads_per_unit, int d) {
-    const size_t tickets = align_up(size_t(U) * 4, 256);
+    const size_t meta = align_up(size_t(U) * 8, 256);
     const size_t partials = size_t(U + attend_grid()) * heads_per_unit * (d + 2) * 4;
-    return tickets + align_up(partials, 256);
+    return meta + align_up(partials, 256);
 }
 
 spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
@@ -456,10 +494,14 @@ spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
         const size_t sm = attend_smem<128>(U);
         SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));
         attend_kernel<128><<<grid, kAtThreads, sm, st>>>(p, U, nh);
+        SPA_CUDA_TRY(cudaGetLastError());
+        combine_kernel<128><<<dim3(U, nh), 256, 0, st>>>(p, nh);
     } else if (p.d == 64) {
         const size_t sm = attend_smem<64>(U);
         SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));
         attend_kernel<64><<<grid, kAtThreads, sm, st>>>(p, U, nh);
+        SPA_CUDA_TRY(cudaGetLastError());
+        combine_kernel<64><<<dim3(U, nh), 256, 0, st>>>(p, nh);
     } else {
         return SPA_ERR_UNSUPPORTED_SHAPE;
     }

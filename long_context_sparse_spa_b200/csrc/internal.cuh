@@ -50,23 +50,62 @@ __device__ __forceinline__ float key_score(uint32_t k) {
     return __uint_as_float(u);
 }
 
+// ------------------------------------------------------------------ level-0 selection histogram
+// Per unit: 2048 bins over the top 11 bits of the score keys.  Each bin holds its count
+// and a 64-bit fixed-point mass sum_n round(2^40 exp(s_n - r_b)), where r_b is the largest
+// score a key of bin b can hold, so the sums need no knowledge of the unit's maximum and
+// are exact integers whatever the order of accumulation; plus the unit's largest key.
+// Producers (the fused scoring kernel, or the histogram kernel) add into it; the selection
+// kernel reads it and zeroes it again for the next call.
+constexpr int kHistBins = 2048;
+constexpr float kMassScale = 1099511627776.0f;   // 2^40
+
+struct Hist0 {
+    uint32_t* cnt;                 // [U][2048]
+    unsigned long long* mass;      // [U][2048]
+    uint32_t* max_key;             // [U]
+};
+inline size_t hist0_bytes(int U) {
+    return align_up(size_t(U) * kHistBins * 4, 256) + align_up(size_t(U) * kHistBins * 8, 256) +
+           align_up(size_t(U) * 4, 256);
+}
+inline Hist0 hist0_carve(void* base, int U) {
+    uint8_t* b = static_cast<uint8_t*>(base);
+    Hist0 h;
+    h.cnt = reinterpret_cast<uint32_t*>(b);
+    b += align_up(size_t(U) * kHistBins * 4, 256);
+    h.mass = reinterpret_cast<unsigned long long*>(b);
+    b += align_up(size_t(U) * kHistBins * 8, 256);
+    h.max_key = reinterpret_cast<uint32_t*>(b);
+    return h;
+}
+// largest score a key of level-0 bin b can hold (bin 2047 holds only +inf/NaN patterns)
+__device__ __forceinline__ float bin_top_score(uint32_t b) {
+    return b >= 2047u ? 3.402823466e38f : key_score(((b + 1u) << 21) - 1u);
+}
+__device__ __forceinline__ unsigned long long fixed_mass(float s, float ref) {
+    return __float2ull_rn(expf(s - ref) * kMassScale);
+}
+
 __device__ __forceinline__ void raise_status(uint32_t* status, int code) {
     if (status) atomicOr(status, 1u << code);
 }
 
 // ------------------------------------------------------------------ launchers
 // scores.cu
+// hist (optional, GROUP_MEAN only): also accumulate the level-0 histogram of the scores;
+// with_mass adds the fixed-point masses (top-p), else counts only.
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
-                                 int collapse, float scale, float* scores, int* zero_ptr, int zero_count,
+                                 int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
                                  cudaStream_t st);
 spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
-                                int M, int d, int collapse, float scale, float* scores, int* zero_ptr,
-                                int zero_count, cudaStream_t st);
+                                int M, int d, int collapse, float scale, float* scores, cudaStream_t st);
 spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean,
                               float* var, cudaStream_t st);
 
 // select.cu
 struct SelectParams {
+    Hist0 hist;        // level-0 histogram (filled by launch_hist0 or the fused scorer)
     const float* scores;
     const int32_t* unit_len;
     int U, M;
@@ -79,7 +118,9 @@ struct SelectParams {
     float* index_mass;
     uint32_t* status;
 };
+spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st);
 spa_status launch_select(const SelectParams& p, bool topp, cudaStream_t st);
+size_t select_scratch_bytes(int U);
 
 // attend.cu
 struct AttendParams {
@@ -97,11 +138,11 @@ struct AttendParams {
     float* out_f32;
     float* lse;
     // workspace pieces
-    int* tickets;      // [U], zero on entry; left zero on exit
+    int* unit_ctas;    // [U][2]: first and last CTA of a unit split over several CTAs, else -1
     float* partials;   // [(U + grid) * heads_per_unit * (d + 2)]
     uint32_t* status;
 };
-size_t attend_scratch_bytes(int U, int heads_per_unit, int d);   // tickets + partials
+size_t attend_scratch_bytes(int U, int heads_per_unit, int d);   // unit CTA ranges + partials
 int attend_grid();
 spa_status launch_attend(const AttendParams& p, cudaStream_t st);
 

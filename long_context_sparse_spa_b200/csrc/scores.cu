@@ -14,30 +14,42 @@ __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w <<
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // ============================================================================ low-rank
-// One work item = (kv unit, chunk of kChunk rows).  Two lanes share a 32-byte index-key
+// One work item = (kv unit, chunk of kLrChunk rows).  Two lanes share a 32-byte index-key
 // row: each loads one 16-byte half (8 bf16) and the halves are joined with one
-// warp shuffle.  Each thread keeps kUnroll rows of loads in flight.
+// warp shuffle.  Each thread keeps kLrUnroll rows of loads in flight.
+// With HIST (one score per row, GROUP_MEAN), the CTA also histograms its scores into the
+// level-0 selection histogram (shared-memory bins flushed to global with integer atomics,
+// so the result does not depend on the order of accumulation).
 constexpr int kLrThreads = 256;
-constexpr int kLrUnroll = 4;
+constexpr int kLrUnroll = 8;
 constexpr int kLrChunk = 4096;
 
-template <int NQ>
+template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
 lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict__ kidx, int Hq, int Hkv,
-                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items,
-                      int* zero_ptr, int zero_count) {
-    if (zero_ptr && blockIdx.x == 0)
-        for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_ptr[i] = 0;
-
+                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items, Hist0 hist) {
     const int G = Hq / Hkv;
     const int half = threadIdx.x & 1;          // which 8 of the 16 index dims this lane holds
     const int pair = threadIdx.x >> 1;         // row slot within a pass
     constexpr int kRowsPerPass = kLrThreads / 2;
+    constexpr int kHb = HIST ? kHistBins : 1;
+    __shared__ uint32_t h_cnt[kHb];
+    __shared__ unsigned long long h_mass[MASS ? kHb : 1];
+    __shared__ uint32_t h_max;
 
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int kvu = item / chunks_per_unit;        // b * Hkv + g
         const int chunk = item - kvu * chunks_per_unit;
         const int b = kvu / Hkv, g = kvu - b * Hkv;
+        if (HIST) {
+            for (int i = threadIdx.x; i < kHistBins; i += kLrThreads) {
+                h_cnt[i] = 0;
+                if (MASS) h_mass[i] = 0;
+            }
+            if (threadIdx.x == 0) h_max = 0;
+            __syncthreads();
+        }
+        uint32_t my_max = 0;
 
         // Index query (8 dims of it) per query vector, fp32.
         float qv[NQ][8];
@@ -97,9 +109,36 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
                     }
                     const float other = __shfl_xor_sync(0xffffffffu, part, 1);
                     const float dot = half ? other + part : part + other;   // low half + high half
-                    if (!half && n < n1) out_base[size_t(h) * M + n] = scale * dot;
+                    if (!half && n < n1) {
+                        const float sc = scale * dot;
+                        out_base[size_t(h) * M + n] = sc;
+                        if (HIST) {
+                            const uint32_t key = score_key(sc);
+                            const uint32_t bin = key >> 21;
+                            my_max = max(my_max, key);
+                            atomicAdd(&h_cnt[bin], 1u);
+                            if (MASS) atomicAdd(&h_mass[bin], fixed_mass(sc, bin_top_score(bin)));
+                        }
+                    }
                 }
             }
+        }
+        if (HIST) {
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, off));
+            if ((threadIdx.x & 31) == 0) atomicMax(&h_max, my_max);
+            __syncthreads();
+            uint32_t* gc = hist.cnt + size_t(kvu) * kHistBins;
+            unsigned long long* gm = hist.mass + size_t(kvu) * kHistBins;
+            for (int i = threadIdx.x; i < kHistBins; i += kLrThreads) {
+                const uint32_t c = h_cnt[i];
+                if (c) {
+                    atomicAdd(gc + i, c);
+                    if (MASS) atomicAdd(gm + i, h_mass[i]);
+                }
+            }
+            if (threadIdx.x == 0) atomicMax(hist.max_key + kvu, h_max);
+            __syncthreads();
         }
     }
 }
@@ -116,9 +155,7 @@ template <int D, int G>
 __global__ void __launch_bounds__(kTyThreads)
 taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ mean, const float4* __restrict__ var,
                      int Hq, int Hkv, int M, int collapse, float scale, float* __restrict__ scores,
-                     int chunks_per_unit, int n_items, int* zero_ptr, int zero_count) {
-    if (zero_ptr && blockIdx.x == 0)
-        for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_ptr[i] = 0;
+                     int chunks_per_unit, int n_items) {
     __shared__ float qs[G][D];
     constexpr int kPer = D / 8;          // dims per lane
     constexpr int kVec = kPer / 4;       // float4 loads per lane per tensor
@@ -282,20 +319,32 @@ int grid_for(int items, int per_sm) {
 }  // namespace
 
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
-                                 int collapse, float scale, float* scores, int* zero_ptr, int zero_count,
+                                 int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
                                  cudaStream_t st) {
     const int G = Hq / Hkv;
     const int chunks = (M + kLrChunk - 1) / kLrChunk;
     const int items = B * Hkv * chunks;
     const int grid = grid_for(items, 8);
     const uint4* k4 = reinterpret_cast<const uint4*>(kidx);
+    const Hist0 h = hist ? *hist : Hist0{nullptr, nullptr, nullptr};
     if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
-        lowrank_scores_kernel<1><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores, chunks, items,
-                                                                zero_ptr, zero_count);
+        if (hist && with_mass)
+            lowrank_scores_kernel<1, true, true><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores,
+                                                                              chunks, items, h);
+        else if (hist)
+            lowrank_scores_kernel<1, true, false><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores,
+                                                                               chunks, items, h);
+        else
+            lowrank_scores_kernel<1, false, false><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores,
+                                                                                chunks, items, h);
     } else {
+        if (hist) return SPA_ERR_INVALID_ARG;
         switch (G) {
-#define SPA_LR_CASE(n) \
-    case n: lowrank_scores_kernel<n><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores, chunks, items, zero_ptr, zero_count); break;
+#define SPA_LR_CASE(n)                                                                                          \
+    case n:                                                                                                     \
+        lowrank_scores_kernel<n, false, false><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores, \
+                                                                            chunks, items, h);                  \
+        break;
             SPA_LR_CASE(1) SPA_LR_CASE(2) SPA_LR_CASE(4) SPA_LR_CASE(8) SPA_LR_CASE(16)
 #undef SPA_LR_CASE
             default: return SPA_ERR_UNSUPPORTED_SHAPE;
@@ -306,8 +355,7 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
 }
 
 spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
-                                int M, int d, int collapse, float scale, float* scores, int* zero_ptr,
-                                int zero_count, cudaStream_t st) {
+                                int M, int d, int collapse, float scale, float* scores, cudaStream_t st) {
     const int G = Hq / Hkv;
     const int chunks = (M + kTyChunk - 1) / kTyChunk;
     const int items = B * Hkv * chunks;
@@ -317,7 +365,7 @@ spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const floa
 #define SPA_TY_CASE(D, GG)                                                                                  \
     if (d == D && G == GG) {                                                                               \
         taylor_scores_kernel<D, GG><<<grid, kTyThreads, 0, st>>>(q, m4, v4, Hq, Hkv, M, collapse, scale, scores, \
-                                                                  chunks, items, zero_ptr, zero_count);   \
+                                                                  chunks, items);                         \
         SPA_CUDA_TRY(cudaGetLastError());                                                                  \
         return SPA_OK;                                                                                     \
     }

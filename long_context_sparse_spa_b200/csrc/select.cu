@@ -5,24 +5,25 @@
 // "Oracle-Guided Sparse Prefill" 2.1 (top-k support); RTPurbo Methodology 1 (sink and
 // sliding window kept).
 //
-// One thread-block cluster of C CTAs selects one unit's support.  Each CTA owns a
-// contiguous chunk of the unit's scores, converted to order-preserving 32-bit keys and
-// held in shared memory when they fit (re-read from global/L2 otherwise).  The
-// threshold key is found by three radix-histogram levels over the key bits (11, 11 and
-// 10 bits):
-//   1. every CTA histograms (count, mass) of its elements that match the prefix so far;
-//   2. each CTA sums the peers' histograms for the bins it owns (distributed shared
-//      memory, fixed peer order);
-//   3. every CTA reads the merged bins and scans them from the top, finding the bin
-//      where the cumulative count (top-k) or mass (top-p) reaches the target.
-// After the last level the threshold key tau and the quota q of elements equal to tau
-// (taken by ascending position) are exact.  Compaction then walks the chunk in
-// ascending order per warp (ballot + popc prefix sums) and writes the support in
-// ascending order at offsets from a cluster-wide prefix of the CTA counts.
-//
-// Top-p masses are e_n = exp(s_n - m) scaled by 2^40 and rounded to 64-bit integers,
-// so every sum is exact and independent of thread order; the cut is the shortest
-// prefix with sum >= ceil(p * Z).
+// The scores are mapped to order-preserving 32-bit keys and the threshold key is found by
+// a radix descent over the key bits in three levels (11, 11 and 10 bits):
+//   level 0: a histogram of the top 11 bits, with counts and 64-bit fixed-point masses,
+//            built while the scores are produced (fused scoring kernel) or by
+//            hist0_kernel; every bin's masses are taken relative to the largest score the
+//            bin can hold, so the sums are exact integers independent of thread order and
+//            need no knowledge of the maximum.  The crossing bin B0 -- where the cumulative
+//            count reaches k, or the cumulative mass (scaled to the unit's maximum, fp64,
+//            fixed order) reaches p times the total -- is found by one block scan.
+//   levels 1, 2: one thread-block cluster of C CTAs per unit.  Each CTA holds a contiguous
+//            chunk of the unit's scores in shared memory; only elements of B0 are
+//            histogrammed (masses relative to the same bin reference, so they sum exactly to
+//            the level-0 mass of B0); the peers' histograms are merged over distributed
+//            shared memory in a fixed peer order and scanned from the top.
+// The result is the threshold key tau and the quota q of elements equal to tau, taken in
+// ascending position.  Compaction walks each warp's slice of the chunk in ascending order
+// (ballot + popc prefix) and packs the selected positions in place in shared memory; a
+// block scan and a cluster-wide prefix of the CTA counts give every list its offset in the
+// ascending support, and the lists are copied out coalesced.
 #include <cooperative_groups.h>
 
 #include "internal.cuh"
@@ -32,57 +33,52 @@ namespace cg = cooperative_groups;
 namespace spa {
 namespace {
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kMaxCluster = 8;
-constexpr float kMassScale = 1099511627776.0f;   // 2^40
+constexpr double kInvMassScale = 1.0 / 1099511627776.0;   // 2^-40
 
 using u64 = unsigned long long;
 
 struct SelShared {
-    uint32_t hist_cnt[kBins];     // local histogram of the current level
+    uint32_t hist_cnt[kBins];     // local histogram of the current level (levels 1 and 2)
     u64 hist_mass[kBins];
     uint32_t mrg_cnt[kBins];      // merged histogram of the bins this CTA owns
     u64 mrg_mass[kBins];
     uint32_t warp_u32[kSelWarps];
     u64 warp_u64[kSelWarps];
-    uint32_t cta_max_key;         // published to peers
-    uint32_t cta_sel;             // selected count of this CTA (published)
-    u64 cta_fmass;                // mass of forced-only elements (published)
-    // result of a level scan
+    double warp_f64[kSelWarps];
+    uint32_t cta_sel;             // selected count of this CTA (published to peers)
+    double cta_fmass;             // mass of forced-only elements of this CTA (published)
     uint32_t found_bin;
     uint32_t found_above_cnt;
     u64 found_above_mass;
+    double found_above_f64;
     uint32_t found_cnt;
-    u64 total_mass;
 };
 
-__device__ __forceinline__ u64 mass_of(uint32_t key, float m) {
-    return __float2ull_rn(expf(key_score(key) - m) * kMassScale);
-}
-
-// Block-wide exclusive scan of (a, b) in thread order; returns the exclusive prefix and
-// writes the block totals.
-__device__ __forceinline__ void block_exscan(uint32_t a, u64 b, uint32_t& ea, u64& eb, uint32_t& ta, u64& tb,
-                                             SelShared& sh) {
+// Block-wide exclusive scan of (a, b) in thread order; totals returned too.  Fixed order.
+template <typename TB>
+__device__ __forceinline__ void block_exscan(uint32_t a, TB b, uint32_t& ea, TB& eb, uint32_t& ta, TB& tb,
+                                             uint32_t* wa_s, TB* wb_s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t ia = a;
-    u64 ib = b;
+    TB ib = b;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const uint32_t xa = __shfl_up_sync(0xffffffffu, ia, off);
-        const u64 xb = __shfl_up_sync(0xffffffffu, ib, off);
+        const TB xb = __shfl_up_sync(0xffffffffu, ib, off);
         if (lane >= off) { ia += xa; ib += xb; }
     }
-    if (lane == 31) { sh.warp_u32[warp] = ia; sh.warp_u64[warp] = ib; }
+    if (lane == 31) { wa_s[warp] = ia; wb_s[warp] = ib; }
     __syncthreads();
     uint32_t wa = 0, sa = 0;
-    u64 wb = 0, sb = 0;
+    TB wb = 0, sb = 0;
 #pragma unroll
     for (int w = 0; w < kSelWarps; ++w) {
-        const uint32_t va = sh.warp_u32[w];
-        const u64 vb = sh.warp_u64[w];
+        const uint32_t va = wa_s[w];
+        const TB vb = wb_s[w];
         if (w < warp) { wa += va; wb += vb; }
         sa += va; sb += vb;
     }
@@ -90,11 +86,62 @@ __device__ __forceinline__ void block_exscan(uint32_t a, u64 b, uint32_t& ea, u6
     eb = wb + ib - b;
     ta = sa;
     tb = sb;
-    __syncthreads();   // warp_* may be reused by the caller's next scan
+    __syncthreads();
 }
 
+// ============================================================================ level-0 histogram
+// One work item = (unit, chunk of 4096 scores); shared-memory bins flushed with integer
+// atomics into the unit's histogram.
+constexpr int kH0Threads = 256;
+constexpr int kH0Chunk = 4096;
+
+template <bool MASS>
+__global__ void __launch_bounds__(kH0Threads)
+hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
+    __shared__ uint32_t h_cnt[kBins];
+    __shared__ u64 h_mass[MASS ? kBins : 1];
+    __shared__ uint32_t h_max;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int u = item / chunks_per_unit;
+        const int chunk = item - u * chunks_per_unit;
+        const int L = p.unit_len ? min(max(p.unit_len[u], 0), p.M) : p.M;
+        const int n0 = chunk * kH0Chunk, n1 = min(L, n0 + kH0Chunk);
+        if (n0 >= n1) continue;
+        for (int i = threadIdx.x; i < kBins; i += kH0Threads) {
+            h_cnt[i] = 0;
+            if (MASS) h_mass[i] = 0;
+        }
+        if (threadIdx.x == 0) h_max = 0;
+        __syncthreads();
+        uint32_t my_max = 0;
+        const float* row = p.scores + size_t(u) * p.M;
+        for (int n = n0 + threadIdx.x; n < n1; n += kH0Threads) {
+            const float s = __ldg(row + n);
+            const uint32_t key = score_key(s);
+            const uint32_t bin = key >> 21;
+            my_max = max(my_max, key);
+            atomicAdd(&h_cnt[bin], 1u);
+            if (MASS) atomicAdd(&h_mass[bin], fixed_mass(s, bin_top_score(bin)));
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, off));
+        if ((threadIdx.x & 31) == 0) atomicMax(&h_max, my_max);
+        __syncthreads();
+        for (int i = threadIdx.x; i < kBins; i += kH0Threads) {
+            const uint32_t c = h_cnt[i];
+            if (c) {
+                atomicAdd(p.hist.cnt + size_t(u) * kBins + i, c);
+                if (MASS) atomicAdd(p.hist.mass + size_t(u) * kBins + i, h_mass[i]);
+            }
+        }
+        if (threadIdx.x == 0) atomicMax(p.hist.max_key + u, h_max);
+        __syncthreads();
+    }
+}
+
+// ============================================================================ selection
 template <bool TOPP>
-__global__ void __launch_bounds__(kSelThreads, 1)
+__global__ void __launch_bounds__(kSelThreads, 2)
 select_kernel(SelectParams p, int chunk, int resident) {
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
@@ -104,7 +151,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
 
     extern __shared__ __align__(16) uint8_t dyn[];
     SelShared& sh = *reinterpret_cast<SelShared*>(dyn);
-    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn + align_up(sizeof(SelShared), 16));
+    float* sv = reinterpret_cast<float*>(dyn + align_up(sizeof(SelShared), 16));   // resident chunk
 
     const int L = p.unit_len ? min(max(p.unit_len[u], 0), p.M) : p.M;
     const int lo = min(L, rank * chunk);
@@ -112,65 +159,128 @@ select_kernel(SelectParams p, int chunk, int resident) {
     const int n = hi - lo;
     const float* srow = p.scores + size_t(u) * p.M + lo;
 
-    auto key_at = [&](int i) -> uint32_t { return resident ? keys[i] : score_key(__ldg(srow + i)); };
-
-    // ---- keys into shared memory, local maximum
-    uint32_t kmax = 0;
-    for (int i = tid; i < n; i += kSelThreads) {
-        const uint32_t k = score_key(__ldg(srow + i));
-        if (resident) keys[i] = k;
-        kmax = max(kmax, k);
+    // ---- the chunk into shared memory (128-bit loads when the row slice is aligned)
+    if (resident) {
+        if ((reinterpret_cast<uintptr_t>(srow) & 15) == 0) {
+            const int n4 = n >> 2;
+            const float4* s4 = reinterpret_cast<const float4*>(srow);
+            float4* d4 = reinterpret_cast<float4*>(sv);
+            int i = tid;
+            for (; i + 3 * kSelThreads < n4; i += 4 * kSelThreads) {
+                const float4 a = __ldg(s4 + i), b = __ldg(s4 + i + kSelThreads);
+                const float4 c = __ldg(s4 + i + 2 * kSelThreads), d = __ldg(s4 + i + 3 * kSelThreads);
+                d4[i] = a; d4[i + kSelThreads] = b; d4[i + 2 * kSelThreads] = c; d4[i + 3 * kSelThreads] = d;
+            }
+            for (; i < n4; i += kSelThreads) d4[i] = __ldg(s4 + i);
+            for (int j = (n4 << 2) + tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
+        } else {
+            for (int j = tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
+        }
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
-    if (lane == 0) sh.warp_u32[warp] = kmax;
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t m = 0;
-        for (int w = 0; w < kSelWarps; ++w) m = max(m, sh.warp_u32[w]);
-        sh.cta_max_key = m;
-    }
+    __syncthreads();   // the resident chunk is read by every warp below
+    auto val_at = [&](int i) -> float { return resident ? sv[i] : __ldg(srow + i); };
 
-    // ---- mode
-    // select_all: every position is selected (top-k with k >= L).
-    // select_none: only forced positions (top-k with k <= 0).
     bool select_all = false, select_none = false;
     if (!TOPP) {
         select_all = p.topk >= L;
         select_none = p.topk <= 0;
     }
-    cluster.sync();   // cta_max_key visible; keys resident
-
-    float m = 0.f;
-    if (TOPP) {
-        uint32_t gmax = 0;
-        for (int r = 0; r < C; ++r) gmax = max(gmax, *cluster.map_shared_rank(&sh.cta_max_key, r));
-        m = key_score(gmax);
-    }
-
-    uint32_t tau = 0, q = 0;              // threshold key, tie quota
-    uint32_t bin_last = 0;                // level-3 bin of tau (its local count = ties here)
-    u64 Z = 0, T = 0, cum_mass = 0, E_tau = 0;
-    uint32_t cum_cnt = 0;
     const bool thresholded = L > 0 && !select_all && !select_none;
 
+    // ---- level 0: crossing bin B0 from the unit's histogram (same result in every CTA)
+    const uint32_t* hc = p.hist.cnt + size_t(u) * kBins;
+    const u64* hm = p.hist.mass + size_t(u) * kBins;
+    const uint32_t max_key = p.hist.max_key[u];
+    const float m = key_score(max_key);
+    double Z = 0.0, T = 0.0;
+    uint32_t b0 = max_key >> 21, cum_cnt0 = 0;
+    double cum_mass0 = 0.0;
     if (thresholded) {
-        uint32_t prefix = 0;
-        for (int level = 0; level < 3; ++level) {
-            const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
-            const int nb = level == 2 ? 1024 : 2048;
-            const int pshift = shift + (level == 2 ? 10 : 11);   // bits above this level
+        if (tid == 0) {
+            sh.found_bin = b0;
+            sh.found_above_cnt = 0;
+            sh.found_above_f64 = 0.0;
+        }
+        constexpr int per = kBins / kSelThreads;   // 8 bins per thread, descending
+        uint32_t vc[per];
+        double vm[per];
+        uint32_t sc = 0;
+        double sm = 0.0;
+#pragma unroll
+        for (int j = 0; j < per; ++j) {
+            const int bin = kBins - 1 - (tid * per + j);
+            vc[j] = __ldcg(hc + bin);
+            vm[j] = 0.0;
+            if (TOPP) {
+                const u64 mb = __ldcg(hm + bin);
+                if (mb) vm[j] = double(mb) * kInvMassScale * exp(double(bin_top_score(bin)) - double(m));
+            }
+            sc += vc[j];
+            sm += vm[j];
+        }
+        uint32_t ec, tc;
+        double em, tm;
+        block_exscan<double>(sc, sm, ec, em, tc, tm, sh.warp_u32, sh.warp_f64);
+        if (TOPP) {
+            Z = tm;
+            T = double(p.topp) * Z;
+        }
+        uint32_t ac = ec;
+        double am = em;
+#pragma unroll
+        for (int j = 0; j < per; ++j) {
+            const bool hit = TOPP ? (am < T && am + vm[j] >= T)
+                                  : (ac < uint32_t(p.topk) && ac + vc[j] >= uint32_t(p.topk));
+            if (hit) {
+                sh.found_bin = uint32_t(kBins - 1 - (tid * per + j));
+                sh.found_above_cnt = ac;
+                sh.found_above_f64 = am;
+            }
+            ac += vc[j];
+            am += vm[j];
+        }
+        __syncthreads();
+        b0 = sh.found_bin;
+        cum_cnt0 = sh.found_above_cnt;
+        cum_mass0 = sh.found_above_f64;
+        __syncthreads();
+    }
+    const float r0 = bin_top_score(b0);                       // mass reference inside B0
+    const double scale0 = TOPP ? kInvMassScale * exp(double(r0) - double(m)) : 0.0;
+
+    // ---- levels 1 and 2 inside B0
+    uint32_t tau = 0, q = 0, cnt_tau = 0, bin_last = 0;
+    u64 cum_in = 0, E_tau = 0;          // mass above tau inside B0 (fixed point, relative to r0)
+    if (thresholded) {
+        uint32_t target_cnt = 0;
+        u64 target_mass = 0;
+        if (TOPP) {
+            const double need = (T - cum_mass0) / scale0;
+            const u64 hb = __ldcg(hm + b0);
+            u64 t = need <= 1.0 ? 1ull : (need >= double(hb) ? hb : u64(ceil(need)));
+            target_mass = t < 1 ? 1 : t;
+        } else {
+            target_cnt = uint32_t(p.topk) - cum_cnt0;
+        }
+        uint32_t prefix = b0;
+        uint32_t cum_c = 0;
+        u64 cum_m = 0;
+        for (int level = 1; level <= 2; ++level) {
+            const int shift = level == 1 ? 10 : 0;
+            const int nb = level == 1 ? 2048 : 1024;
+            const int pshift = level == 1 ? 21 : 10;
             for (int i = tid; i < nb; i += kSelThreads) {
                 sh.hist_cnt[i] = 0;
                 if (TOPP) sh.hist_mass[i] = 0;
             }
             __syncthreads();
             for (int i = tid; i < n; i += kSelThreads) {
-                const uint32_t k = key_at(i);
-                if (level == 0 || (k >> pshift) == prefix) {
+                const float s = val_at(i);
+                const uint32_t k = score_key(s);
+                if ((k >> pshift) == prefix) {
                     const uint32_t bin = (k >> shift) & uint32_t(nb - 1);
                     atomicAdd(&sh.hist_cnt[bin], 1u);
-                    if (TOPP) atomicAdd(&sh.hist_mass[bin], mass_of(k, m));
+                    if (TOPP) atomicAdd(&sh.hist_mass[bin], fixed_mass(s, r0));
                 }
             }
             cluster.sync();   // local histograms complete
@@ -187,14 +297,13 @@ select_kernel(SelectParams p, int chunk, int resident) {
             }
             cluster.sync();   // merged slices complete
 
-            // scan the merged bins from the top (thread t owns descending positions)
-            const int per = nb / kSelThreads;
-            uint32_t vc[4];
-            u64 vm[4];
+            const int per = nb / kSelThreads;    // 8 or 4 bins per thread, descending
+            uint32_t vc[8];
+            u64 vm[8];
             uint32_t sc = 0;
             u64 sm = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 vc[j] = 0; vm[j] = 0;
                 if (j < per) {
                     const int bin = nb - 1 - (tid * per + j);
@@ -207,20 +316,21 @@ select_kernel(SelectParams p, int chunk, int resident) {
             }
             uint32_t ec, tc;
             u64 em, tm;
-            block_exscan(sc, sm, ec, em, tc, tm, sh);
-            if (level == 0 && TOPP) {
-                Z = tm;
-                const double t = ceil(double(p.topp) * double(Z));
-                T = t >= double(Z) ? Z : (t < 1.0 ? 1ull : u64(t));
+            block_exscan<u64>(sc, sm, ec, em, tc, tm, sh.warp_u32, sh.warp_u64);
+            if (tid == 0) {   // defaults if rounding left no crossing: the last non-empty bin
+                sh.found_bin = 0;
+                sh.found_above_cnt = cum_c;
+                sh.found_above_mass = cum_m;
+                sh.found_cnt = 0;
             }
-            uint32_t ac = cum_cnt + ec;
-            u64 am = cum_mass + em;
+            __syncthreads();
+            uint32_t ac = cum_c + ec;
+            u64 am = cum_m + em;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 if (j < per) {
-                    bool hit;
-                    if (TOPP) hit = am < T && am + vm[j] >= T;
-                    else hit = ac < uint32_t(p.topk) && ac + vc[j] >= uint32_t(p.topk);
+                    const bool hit = TOPP ? (am < target_mass && am + vm[j] >= target_mass)
+                                          : (ac < target_cnt && ac + vc[j] >= target_cnt);
                     if (hit) {
                         sh.found_bin = uint32_t(nb - 1 - (tid * per + j));
                         sh.found_above_cnt = ac;
@@ -233,63 +343,66 @@ select_kernel(SelectParams p, int chunk, int resident) {
             }
             __syncthreads();
             const uint32_t fb = sh.found_bin;
-            prefix = (prefix << (level == 2 ? 10 : 11)) | fb;
-            cum_cnt = sh.found_above_cnt;
-            cum_mass = sh.found_above_mass;
+            prefix = (prefix << (level == 1 ? 11 : 10)) | fb;
+            cum_c = sh.found_above_cnt;
+            cum_m = sh.found_above_mass;
             if (level == 2) {
                 bin_last = fb;
                 tau = prefix;
-                const uint32_t cnt_tau = sh.found_cnt;
+                cnt_tau = sh.found_cnt;
+                cum_in = cum_m;
                 if (TOPP) {
-                    E_tau = mass_of(tau, m);
-                    const u64 need = T - cum_mass;
+                    E_tau = fixed_mass(key_score(tau), r0);
+                    const u64 need = target_mass > cum_m ? target_mass - cum_m : 0;
                     u64 qq = E_tau ? (need + E_tau - 1) / E_tau : u64(cnt_tau);
                     if (qq < 1) qq = 1;
                     if (qq > cnt_tau) qq = cnt_tau;
                     q = uint32_t(qq);
                 } else {
-                    q = uint32_t(p.topk) - cum_cnt;
+                    q = target_cnt - cum_c;
+                    if (q > cnt_tau) q = cnt_tau;
                 }
             }
-            __syncthreads();   // found_* may be rewritten by the next level
+            __syncthreads();
         }
     }
 
-    // ---- ties before this CTA (each CTA's level-3 local count of tau, peers in order)
-    uint32_t ties_before_cta = 0;
-    if (thresholded)
-        for (int r = 0; r < rank; ++r) ties_before_cta += *cluster.map_shared_rank(&sh.hist_cnt[bin_last], r);
-
-    // ---- compaction: warp w walks [w*seg, w*seg+seg) of the chunk in ascending order
+    // ---- compaction: warp w owns [w*seg, w*seg + seg) of the chunk, walked in ascending order
     const int seg = ((n + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
     const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
     const int window_lo = L - p.window;
-    auto forced = [&](int pos) { return pos < p.sink || pos >= window_lo; };
+    const unsigned lt_mask = (1u << lane) - 1u;
 
-    // pass 1: ties per warp -> ties before each warp
-    uint32_t wties = 0;
-    if (thresholded)
+    // ties before each warp are needed only when the quota splits the run of equal keys
+    int64_t q_warp = int64_t(q);
+    const bool split_ties = thresholded && q < cnt_tau;
+    if (split_ties) {
+        uint32_t before = 0;
+        for (int r = 0; r < rank; ++r) before += *cluster.map_shared_rank(&sh.hist_cnt[bin_last], r);
+        uint32_t wt = 0;
         for (int i0 = w0; i0 < w1; i0 += 32) {
             const int i = i0 + lane;
-            const bool tie = i < w1 && key_at(i) == tau;
-            wties += __popc(__ballot_sync(0xffffffffu, tie));
+            wt += __popc(__ballot_sync(0xffffffffu, i < w1 && score_key(val_at(i)) == tau));
         }
-    if (lane == 0) sh.warp_u32[warp] = wties;
-    __syncthreads();
-    uint32_t ties_before = ties_before_cta;
-    for (int w = 0; w < warp; ++w) ties_before += sh.warp_u32[w];
-    __syncthreads();
-    const int64_t q_warp = int64_t(q) - int64_t(ties_before);
+        if (lane == 0) sh.warp_u32[warp] = wt;
+        __syncthreads();
+        for (int w = 0; w < warp; ++w) before += sh.warp_u32[w];
+        __syncthreads();
+        q_warp = int64_t(q) - int64_t(before);
+    }
 
-    const unsigned lt_mask = (1u << lane) - 1u;
-    auto walk = [&](bool write, uint32_t base, uint32_t& nsel, u64& fmass) {
+    // one ascending walk: selected positions of warp w are packed at sv[w0 ...] in place
+    // (resident chunk), or only counted (streaming chunk, written by a second walk)
+    auto walk = [&](bool pack, bool write, uint32_t base, uint32_t& nsel, double& fmass) {
         uint32_t run_tie = 0;
         nsel = 0;
-        fmass = 0;
+        fmass = 0.0;
+        int* packed = reinterpret_cast<int*>(sv);
         for (int i0 = w0; i0 < w1; i0 += 32) {
             const int i = i0 + lane;
             const bool live = i < w1;
-            const uint32_t k = live ? key_at(i) : 0u;
+            const float s = live ? val_at(i) : 0.f;
+            const uint32_t k = score_key(s);
             const int pos = lo + i;
             bool top = false, tie = false;
             if (select_all) top = live;
@@ -298,58 +411,70 @@ select_kernel(SelectParams p, int chunk, int resident) {
                 tie = live && k == tau;
             }
             const unsigned tb = __ballot_sync(0xffffffffu, tie);
-            if (tie) top = int64_t(run_tie + __popc(tb & lt_mask)) < q_warp;
+            if (tie) top = !split_ties || int64_t(run_tie + __popc(tb & lt_mask)) < q_warp;
             run_tie += __popc(tb);
-            const bool f = live && forced(pos);
+            const bool f = live && (pos < p.sink || pos >= window_lo);
             const bool sel = top || f;
-            if (TOPP && f && !top) fmass += mass_of(k, m);
+            if (TOPP && f && !top) fmass += exp(double(s) - double(m));
             const unsigned sb = __ballot_sync(0xffffffffu, sel);
-            if (write && sel) {
-                const uint32_t at = base + nsel + __popc(sb & lt_mask);
-                if (at < uint32_t(p.cap)) p.idx[size_t(u) * p.cap + at] = pos;
+            if (sel) {
+                const uint32_t at = nsel + __popc(sb & lt_mask);
+                if (pack) packed[w0 + at] = pos;     // at <= i: never overtakes the reads
+                if (write && base + at < uint32_t(p.cap)) p.idx[size_t(u) * p.cap + base + at] = pos;
             }
             nsel += __popc(sb);
         }
-    };
-
-    // pass 2: counts per warp
-    uint32_t nsel;
-    u64 fmass;
-    walk(false, 0, nsel, fmass);
-    if (TOPP) {
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) fmass += __shfl_xor_sync(0xffffffffu, fmass, off);
-    }
-    if (lane == 0) { sh.warp_u32[warp] = nsel; sh.warp_u64[warp] = fmass; }
+    };
+
+    uint32_t nsel;
+    double fmass;
+    walk(resident != 0, false, 0, nsel, fmass);
+    if (lane == 0) { sh.warp_u32[warp] = nsel; sh.warp_f64[warp] = fmass; }
     __syncthreads();
     uint32_t sel_before_warp = 0;
     for (int w = 0; w < warp; ++w) sel_before_warp += sh.warp_u32[w];
     if (tid == 0) {
         uint32_t t = 0;
-        u64 fm = 0;
-        for (int w = 0; w < kSelWarps; ++w) { t += sh.warp_u32[w]; fm += sh.warp_u64[w]; }
+        double fm = 0.0;
+        for (int w = 0; w < kSelWarps; ++w) { t += sh.warp_u32[w]; fm += sh.warp_f64[w]; }
         sh.cta_sel = t;
         sh.cta_fmass = fm;
     }
-    cluster.sync();   // CTA counts visible to peers
+    cluster.sync();   // CTA counts visible to peers; every CTA is past its level-0 reads
     uint32_t sel_before_cta = 0, total = 0;
-    u64 fmass_total = 0;
+    double fmass_total = 0.0;
     for (int r = 0; r < C; ++r) {
         const uint32_t c = *cluster.map_shared_rank(&sh.cta_sel, r);
         if (r < rank) sel_before_cta += c;
         total += c;
         if (TOPP) fmass_total += *cluster.map_shared_rank(&sh.cta_fmass, r);
     }
+    const uint32_t base = sel_before_cta + sel_before_warp;
+    if (resident) {
+        const int* packed = reinterpret_cast<const int*>(sv);
+        for (uint32_t j = lane; j < nsel; j += 32)
+            if (base + j < uint32_t(p.cap)) p.idx[size_t(u) * p.cap + base + j] = packed[w0 + j];
+    } else {
+        walk(false, true, base, nsel, fmass);
+    }
 
-    // pass 3: write
-    walk(true, sel_before_cta + sel_before_warp, nsel, fmass);
-
-    if (rank == 0 && tid == 0) {
-        p.count[u] = int32_t(total);
-        if (total > uint32_t(p.cap)) raise_status(p.status, SPA_ERR_CAPACITY);
-        if (TOPP && p.index_mass) {
-            const u64 top_mass = thresholded ? cum_mass + u64(q) * E_tau : 0ull;
-            p.index_mass[u] = Z ? float(double(top_mass + fmass_total) / double(Z)) : 0.f;
+    if (rank == 0) {
+        // the unit's level-0 histogram is consumed: clear it for the next producer
+        for (int i = tid; i < kBins; i += kSelThreads) {
+            p.hist.cnt[size_t(u) * kBins + i] = 0;
+            p.hist.mass[size_t(u) * kBins + i] = 0;
+        }
+        if (tid == 0) {
+            p.hist.max_key[u] = 0;
+            p.count[u] = int32_t(total);
+            if (total > uint32_t(p.cap)) raise_status(p.status, SPA_ERR_CAPACITY);
+            if (TOPP && p.index_mass) {
+                double top = 0.0;
+                if (thresholded) top = cum_mass0 + double(cum_in + u64(q) * E_tau) * scale0;
+                p.index_mass[u] = Z > 0.0 ? float((top + fmass_total) / Z) : 0.f;
+            }
         }
     }
     cluster.sync();   // no CTA leaves while a peer may still read its shared memory
@@ -362,25 +487,71 @@ struct SelectConfig {
     size_t smem;
 };
 
+template <bool TOPP>
+int max_active_clusters(int C, size_t smem) {
+    // cached per (device, C, smem bucket)
+    static thread_local int cache_dev = -1;
+    static thread_local int cache[kMaxCluster + 1][4];
+    const DeviceInfo& di = device_info();
+    if (cache_dev != di.device) {
+        for (auto& row : cache)
+            for (int& v : row) v = -1;
+        cache_dev = di.device;
+    }
+    const int bucket = smem <= 48 * 1024 ? 0 : (smem <= 113 * 1024 ? 1 : (smem <= 160 * 1024 ? 2 : 3));
+    int& v = cache[C][bucket];
+    if (v < 0) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(C, 1, 1);
+        cfg.blockDim = dim3(kSelThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, select_kernel<TOPP>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        v = n;
+    }
+    return v;
+}
+
+template <bool TOPP>
 SelectConfig choose(int U, int M) {
     const DeviceInfo& di = device_info();
-    SelectConfig c{};
-    int C = 1;
-    while (C < kMaxCluster && U * C < di.num_sms) C *= 2;
-    while (C > 1 && (M + C - 1) / C < 1024) C /= 2;
-    c.C = C;
-    c.chunk = (M + C - 1) / C;
     const size_t fixed = align_up(sizeof(SelShared), 16);
-    const size_t budget = size_t(di.max_smem_optin) - fixed;
-    c.resident = size_t(c.chunk) * 4 <= budget;
-    c.smem = fixed + (c.resident ? size_t(c.chunk) * 4 : 0);
-    return c;
+    SelectConfig best{};
+    best.C = 0;
+    // largest cluster (<= 8) that keeps every unit's cluster in one wave and >= 2048 scores per CTA
+    for (int C = kMaxCluster; C >= 1; C /= 2) {
+        if (C > 1 && (M + C - 1) / C < 2048) continue;
+        const int chunk = ((M + C - 1) / C + 3) / 4 * 4;
+        size_t smem = fixed + size_t(chunk) * 4;
+        int resident = 1;
+        if (smem > size_t(di.max_smem_optin)) {
+            resident = 0;
+            smem = fixed;
+        }
+        cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        const int active = C > 1 ? max_active_clusters<TOPP>(C, smem) : U;
+        if (C == 1 || U <= active) {
+            best = SelectConfig{C, chunk, resident, smem};
+            break;
+        }
+    }
+    if (best.C == 0) best = SelectConfig{1, M, 0, fixed};
+    return best;
 }
 
 template <bool TOPP>
 spa_status launch_t(const SelectParams& p, cudaStream_t st) {
-    const SelectConfig c = choose(p.U, p.M);
-    static_assert(kBins % (kMaxCluster * 1) == 0, "bins split across the cluster");
+    const SelectConfig c = choose<TOPP>(p.U, p.M);
     SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(c.C, p.U, 1);
@@ -399,6 +570,20 @@ spa_status launch_t(const SelectParams& p, cudaStream_t st) {
 }
 
 }  // namespace
+
+size_t select_scratch_bytes(int U) { return hist0_bytes(U); }
+
+spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st) {
+    const int chunks = (p.M + kH0Chunk - 1) / kH0Chunk;
+    const int items = p.U * chunks;
+    if (items == 0) return SPA_OK;
+    const int cap = device_info().num_sms * 8;
+    const int grid = items < cap ? items : cap;
+    if (with_mass) hist0_kernel<true><<<grid, kH0Threads, 0, st>>>(p, chunks, items);
+    else hist0_kernel<false><<<grid, kH0Threads, 0, st>>>(p, chunks, items);
+    SPA_CUDA_TRY(cudaGetLastError());
+    return SPA_OK;
+}
 
 spa_status launch_select(const SelectParams& p, bool topp, cudaStream_t st) {
     return topp ? launch_t<true>(p, st) : launch_t<false>(p, st);

@@ -188,6 +188,7 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
     res: Dict[str, object] = {"b": b, "g": g}
     if cfg.score == "lowrank":
         s = lowrank_scores(x["q_idx"][b, heads], x["Kidx"][b, g], cfg.collapse == "group", f32(cfg.score_scale))
+        s = s.reshape(-1)                 # one row: the group's shared scores, or the one head's
         ranked = as_ranked(s)
     else:
         mean, var = stats if stats is not None else block_stats(x["K"][b, g], cfg.block)

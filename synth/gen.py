@@ -24,6 +24,8 @@ method only consumes its outputs).
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, Iterable, Optional, Tuple
 
 import numpy as np
@@ -35,11 +37,16 @@ BF16 = np.uint16
 
 # --------------------------------------------------------------------------- bf16 bits
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32/float64 values to bf16 (RNE) and return the uint16 bit patterns."""
-    f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    u += np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))
-    return (u >> np.uint64(16)).astype(np.uint16)
+    """Round finite float32/float64 values to bf16 (RNE) and return the uint16 bit patterns.
+
+    For finite binary32 patterns u <= 0xFF7FFFFF, u + 0x8000 cannot overflow 32 bits."""
+    u = np.array(x, dtype=np.float32, copy=True, order="C").view(np.uint32)
+    lsb = u >> np.uint32(16)
+    lsb &= np.uint32(1)
+    lsb += np.uint32(0x7FFF)
+    u += lsb
+    u >>= np.uint32(16)
+    return u.astype(np.uint16)
 
 
 def bf16_value(b: np.ndarray) -> np.ndarray:
@@ -134,26 +141,45 @@ def decode_unit_values(cfg: DecodeConfig, b: int, g: int) -> np.ndarray:
     return bf16_bits(_rng(cfg.seed, 4, b, g).standard_normal((cfg.N, cfg.d), dtype=np.float32))
 
 
-def decode_inputs(cfg: DecodeConfig, units: Optional[Iterable[Tuple[int, int]]] = None) -> Dict[str, np.ndarray]:
+def decode_inputs(cfg: DecodeConfig, units: Optional[Iterable[Tuple[int, int]]] = None,
+                  batch: Optional[Tuple[int, int]] = None, threads: int = 0) -> Dict[str, np.ndarray]:
     """All inputs of a decode workload as uint16 bf16 bit arrays.
 
     Returns q [B,Hq,d], K, V [B,Hkv,N,d] and, for low-rank scoring, q_idx [B,Hq,r],
     Kidx [B,Hkv,N,r] and the projector P.  ``units`` restricts key/value generation to
     the listed (b, g) pairs (others stay zero), for bounded samples of large workloads.
+    ``batch = (b0, b1)`` returns only batch entries b0 <= b < b1 of the workload (a data
+    shard: entry b is drawn exactly as in the full workload).  Units are generated on
+    ``threads`` threads (default: all cores); each has its own random stream, so the
+    result does not depend on the thread count.
     """
     q, q_idx, P = decode_queries(cfg)
-    B, Hkv, N, d = cfg.B, cfg.Hkv, cfg.N, cfg.d
+    b0, b1 = batch if batch is not None else (0, cfg.B)
+    q = q[b0:b1].copy()
+    q_idx = q_idx[b0:b1].copy() if q_idx is not None else None
+    B, Hkv, N, d = b1 - b0, cfg.Hkv, cfg.N, cfg.d
     K = np.zeros((B, Hkv, N, d), BF16)
     V = np.zeros((B, Hkv, N, d), BF16)
     Kidx = np.zeros((B, Hkv, N, cfg.r), BF16) if P is not None else None
     lf = lowfreq_component(cfg.seed, N, d, cfg.lowfreq_rank, cfg.lowfreq_amp) if cfg.lowfreq_rank else None
     needles = {}
-    todo = list(units) if units is not None else [(b, g) for b in range(B) for g in range(Hkv)]
-    for b, g in todo:
-        K[b, g], needles[(b, g)] = decode_unit_keys(cfg, b, g, q, lf)
-        V[b, g] = decode_unit_values(cfg, b, g)
+    todo = list(units) if units is not None else [(b, g) for b in range(b0, b1) for g in range(Hkv)]
+    qfull = decode_queries(cfg)[0]
+
+    def one(bg):
+        b, g = bg
+        K[b - b0, g], needles[(b, g)] = decode_unit_keys(cfg, b, g, qfull, lf)
+        V[b - b0, g] = decode_unit_values(cfg, b, g)
         if Kidx is not None:
-            Kidx[b, g] = _project(K[b, g], P)
+            Kidx[b - b0, g] = _project(K[b - b0, g], P)
+
+    n_threads = threads if threads > 0 else min(len(todo), os.cpu_count() or 1)
+    if n_threads <= 1:
+        for bg in todo:
+            one(bg)
+    else:
+        with ThreadPoolExecutor(n_threads) as ex:
+            list(ex.map(one, todo))
     out = {"q": q, "K": K, "V": V, "needles": needles}
     if P is not None:
         out.update(q_idx=q_idx, Kidx=Kidx, P=P)

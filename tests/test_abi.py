@@ -42,13 +42,14 @@ def test_host_validation():
     L = spa.lib()
     P = ctypes.c_void_p(16)   # never dereferenced: every call below fails validation first
     # negative sizes
-    assert L.spa_select_topk(P, None, -1, 10, 1, 0, 0, P, P, 1, P, 256, None) == _abi.SPA_ERR_INVALID_ARG
+    assert L.spa_select_topk(P, None, -1, 10, 1, 0, 0, P, P, 1, P, 1 << 30, None) == _abi.SPA_ERR_INVALID_ARG
     # workspace too small
     assert L.spa_select_topk(P, None, 2, 10, 1, 0, 0, P, P, 1, P, 8, None) == _abi.SPA_ERR_WORKSPACE_TOO_SMALL
     # p outside (0, 1]
-    assert L.spa_select_topp(P, None, 2, 10, ctypes.c_float(0.0), 0, 0, P, P, 10, None, P, 256, None) == \
+    big = 1 << 30
+    assert L.spa_select_topp(P, None, 2, 10, ctypes.c_float(0.0), 0, 0, P, P, 10, None, P, big, None) == \
         _abi.SPA_ERR_INVALID_ARG
-    assert L.spa_select_topp(P, None, 2, 10, ctypes.c_float(1.5), 0, 0, P, P, 10, None, P, 256, None) == \
+    assert L.spa_select_topp(P, None, 2, 10, ctypes.c_float(1.5), 0, 0, P, P, 10, None, P, big, None) == \
         _abi.SPA_ERR_INVALID_ARG
     # unsupported index dim / head dim / group size
     assert L.spa_index_scores(0, P, P, None, 1, 4, 1, 10, 32, 0, ctypes.c_float(1.0), P, None) == \
