@@ -12,13 +12,17 @@
 // with cp.async (16-byte copies, bounds-checked, zero-filled when the index is out of
 // range) into a private multi-stage ring in shared memory.
 //
-// Math per 16-row tile, on tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
-//   S = Q K^T with the unit's query heads as the 16 rows of Q (G <= 16 heads; unused
-//   rows are zero), an fp32 online softmax per head (exp2 with the log2(e) factor folded
-//   into the scale), then O += P V.  P is carried as the sum of two bf16 terms (hi + lo)
-//   so that the product keeps about 16 bits of each weight.  The rows of a GQA group
-//   share every K/V row loaded, which is why the step is a small dense contraction: on
-//   CUDA cores its 8 flops per byte would bound the kernel well below HBM speed.
+// Math per 16-row tile, on tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate),
+// in transposed form so that the gathered keys, not the few query heads, fill the
+// 16-row side of the tensor-core tile:
+//   S^T = K Q^T      16 keys x 8 heads per head tile (the group's G <= 16 heads, padded to 8);
+//   fp32 online softmax per head (column), exp2 with log2(e) folded into the scale;
+//   P^T is moved into the B-operand layout by two 8x8 transposes (movmatrix);
+//   O^T += V^T P^T   V^T read with transposing ldmatrix; d = 128 rows x 8 heads.
+// P is carried as the sum of two bf16 terms (hi + lo) so the product keeps about 16 bits
+// of each weight.  The heads of a GQA group share every K/V row loaded, which is why the
+// step is a small dense contraction: on CUDA cores its 8 flops per byte would bound the
+// kernel well below HBM speed.  Row indices are fetched one tile ahead of their gather.
 //
 // At the end of its share of a unit a CTA merges its warps' (m, l, o) in shared memory.
 // A CTA holding a whole unit writes the output; otherwise it stores a partial (o, m, l),
@@ -34,6 +38,7 @@ constexpr int kAtWarps = kAtThreads / 32;
 constexpr int kRows = 16;           // rows per tile (the mma N-extent of the score tile)
 constexpr int kStages = 3;          // cp.async ring depth per warp
 constexpr int kMaxUnits = 8192;
+constexpr int kWinTiles = 128;      // tiles whose row indices are staged in shared memory at once
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -61,6 +66,12 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         "{%0,%1,%2,%3};\n"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// transpose of an 8x8 b16 matrix held in mma fragment layout (one b16x2 per thread)
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
 }
 // p ~= hi + lo with hi = bf16(p), lo = bf16(p - hi)
 __device__ __forceinline__ void split_bf16(float p0, float p1, uint32_t& hi, uint32_t& lo) {
@@ -112,17 +123,18 @@ __device__ __forceinline__ int tile_owner(long long x, long long TT, int G) {
     return int(((x + 1) * G - 1) / TT);
 }
 
-template <int D>
+template <int D, int NH8>
 __global__ void __launch_bounds__(kAtThreads, 2)
 attend_kernel(AttendParams p, int U, int nh) {
     using TL = Tile<D>;
     extern __shared__ __align__(128) uint8_t smem[];
     int* s_prefix = reinterpret_cast<int*>(smem);                            // [U + 1]
-    uint8_t* ring = smem + align_up(size_t(U + 1) * 4, 128);
+    int* s_rows = reinterpret_cast<int*>(smem + align_up(size_t(U + 1) * 4, 128));   // [kWinTiles * 16]
+    uint8_t* ring = smem + align_up(size_t(U + 1) * 4, 128) + size_t(kWinTiles) * kRows * 4;
     __shared__ uint32_t s_vmask[kAtWarps][kStages];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gq = lane >> 2, cq = lane & 3;   // mma fragment coordinates
+    const int gq = lane >> 2, cq = lane & 3;   // mma fragment coordinates (row group, column pair)
     uint8_t* my_ring = ring + size_t(warp) * kStages * TL::BYTES;
 
     // ---- tile prefix over units
@@ -209,37 +221,28 @@ attend_kernel(AttendParams p, int U, int nh) {
         const int tiles_u = s_prefix[u + 1] - s_prefix[u];
         const UnitGeom ug = unit_geom(p, u, nh);
 
-        // Q fragments (rows = query heads of the unit; rows >= nh are zero)
-        uint32_t qa[TL::KSTEPS][4];
+        // Q^T as the B operand of S^T = K Q^T: b0/b1 of k-step kk, head tile nt hold
+        // q[head 8nt + gq][16kk + 2cq (+1)] and [16kk + 8 + 2cq (+1)]; heads >= nh are zero.
+        uint32_t qb[TL::KSTEPS][NH8][2];
         {
             const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
-            const size_t r0 = size_t(ug.b) * p.Hq + ug.h0 + gq;
-            const bool v0 = gq < nh, v1 = gq + 8 < nh;
 #pragma unroll
-            for (int kk = 0; kk < TL::KSTEPS; ++kk) {
-                const int col = kk * 16 + 2 * cq;
-                qa[kk][0] = v0 ? __ldg(q32 + (r0 * D + col) / 2) : 0u;
-                qa[kk][1] = v1 ? __ldg(q32 + ((r0 + 8) * D + col) / 2) : 0u;
-                qa[kk][2] = v0 ? __ldg(q32 + (r0 * D + col + 8) / 2) : 0u;
-                qa[kk][3] = v1 ? __ldg(q32 + ((r0 + 8) * D + col + 8) / 2) : 0u;
+            for (int nt = 0; nt < NH8; ++nt) {
+                const int hd = nt * 8 + gq;
+                const bool v = hd < nh;
+                const size_t r0 = size_t(ug.b) * p.Hq + ug.h0 + hd;
+#pragma unroll
+                for (int kk = 0; kk < TL::KSTEPS; ++kk) {
+                    const int col = kk * 16 + 2 * cq;
+                    qb[kk][nt][0] = v ? __ldg(q32 + (r0 * D + col) / 2) : 0u;
+                    qb[kk][nt][1] = v ? __ldg(q32 + (r0 * D + col + 8) / 2) : 0u;
+                }
             }
         }
 
-        // warp's tiles: a + warp, a + warp + 4, ...
-        const int first = a + warp;
-        const int n_my = first < bnd ? (bnd - first + kAtWarps - 1) / kAtWarps : 0;
         const int32_t* idx_u = p.idx + size_t(u) * p.cap;
         const int T = p.unit_tokens;
-
-        auto issue = [&](int j, int stage) {
-            const int tile = first + j * kAtWarps;
-            const int r = tile * kRows + (lane & 15);
-            long long row = -1;
-            if (r < ug.rows) {
-                const int e = T == 1 ? r : r / T;
-                const long long n = (long long)idx_u[e] * T + (T == 1 ? 0 : r - e * T);
-                if (n >= 0 && n < p.N) row = n;
-            }
+        auto issue = [&](long long row, int stage) {
             const uint32_t vm = __ballot_sync(0xffffffffu, row >= 0) & 0xffffu;
             if (lane == 0) s_vmask[warp][stage] = vm;
             uint8_t* st = my_ring + size_t(stage) * TL::BYTES;
@@ -258,19 +261,46 @@ attend_kernel(AttendParams p, int U, int nh) {
             }
         };
 
-        float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-        float acc[TL::NT][4];
+        // online-softmax state of heads 8nt + 2cq + e (e = 0, 1); l is this thread's partial sum
+        float m_r[NH8][2], l_r[NH8][2];
+        float acc[TL::KSTEPS][NH8][4];      // O^T: d-tile x head tile, rows d = 16dt + gq (+8)
 #pragma unroll
-        for (int i = 0; i < TL::NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        for (int nt = 0; nt < NH8; ++nt) {
+            m_r[nt][0] = m_r[nt][1] = -INFINITY;
+            l_r[nt][0] = l_r[nt][1] = 0.f;
+#pragma unroll
+            for (int dt = 0; dt < TL::KSTEPS; ++dt) acc[dt][nt][0] = acc[dt][nt][1] = acc[dt][nt][2] = acc[dt][nt][3] = 0.f;
+        }
 
+        for (int wt0 = a; wt0 < bnd; wt0 += kWinTiles) {
+        const int wt1 = min(bnd, wt0 + kWinTiles);
+        // cache rows of the window's tiles, staged once with coalesced index loads (-1: none)
+        __syncthreads();
+        for (int i = tid; i < (wt1 - wt0) * kRows; i += kAtThreads) {
+            const int r = wt0 * kRows + i;
+            int v = -1;
+            if (r < ug.rows) {
+                const int e = T == 1 ? r : r / T;
+                const long long n = (long long)__ldg(idx_u + e) * T + (T == 1 ? 0 : r - e * T);
+                v = (n >= 0 && n < p.N) ? int(n) : -1;
+            }
+            s_rows[i] = v;
+        }
+        __syncthreads();
+        // warp's tiles of the window: wt0 + warp, wt0 + warp + 4, ...
+        const int first = wt0 + warp;
+        const int n_my = first < wt1 ? (wt1 - first + kAtWarps - 1) / kAtWarps : 0;
+        auto fetch = [&](int j) -> long long {
+            return j < n_my ? (long long)s_rows[(first - wt0 + j * kAtWarps) * kRows + (lane & 15)] : -1ll;
+        };
 #pragma unroll
         for (int j = 0; j < kStages - 1; ++j) {
-            if (j < n_my) issue(j, j);
+            if (j < n_my) issue(fetch(j), j);
             cp_commit();
         }
         for (int j = 0; j < n_my; ++j) {
             const int jn = j + kStages - 1;
-            if (jn < n_my) issue(jn, jn % kStages);
+            if (jn < n_my) issue(fetch(jn), jn % kStages);
             cp_commit();
             cp_wait<kStages - 1>();
             __syncwarp();
@@ -279,101 +309,107 @@ attend_kernel(AttendParams p, int U, int nh) {
             const uint32_t kbase = smem_u32(st), vbase = kbase + kRows * D * 2;
             const uint32_t vm = s_vmask[warp][stage];
 
-            // S = Q K^T (two 8-key column tiles)
-            float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            // S^T = K Q^T: 16 keys x 8 heads per head tile
+            float s[NH8][4];
+#pragma unroll
+            for (int nt = 0; nt < NH8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < TL::KSTEPS; ++kk) {
                 const int mat = lane >> 3;
-                const int rr = (mat >> 1) * 8 + (lane & 7);
-                const int c = 2 * kk + (mat & 1);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kbase + (rr * TL::CPR + (c ^ (rr & 7))) * 16, b0, b1, b2, b3);
-                mma16816(s[0], qa[kk], b0, b1);
-                mma16816(s[1], qa[kk], b2, b3);
-            }
-            // scale, mask, online softmax (rows gq and gq + 8)
-            float tmax[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = nt * 8 + 2 * cq + (e & 1);
-                    const float v = ((vm >> key) & 1u) ? s[nt][e] * sl2 : -INFINITY;
-                    s[nt][e] = v;
-                    tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
-                }
-            float alpha[2], mref[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 1));
-                tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
-                const float mn = fmaxf(m_r[h], tmax[h]);
-                mref[h] = mn == -INFINITY ? 0.f : mn;
-                alpha[h] = exp2f(m_r[h] - mref[h]);
-                m_r[h] = mn;
-            }
-            float rs[2] = {0.f, 0.f};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float pv = exp2f(s[nt][e] - mref[e >> 1]);
-                    s[nt][e] = pv;
-                    rs[e >> 1] += pv;
-                }
-            l_r[0] = l_r[0] * alpha[0] + rs[0];
-            l_r[1] = l_r[1] * alpha[1] + rs[1];
-#pragma unroll
-            for (int i = 0; i < TL::NT; ++i) {
-                acc[i][0] *= alpha[0]; acc[i][1] *= alpha[0];
-                acc[i][2] *= alpha[1]; acc[i][3] *= alpha[1];
-            }
-            uint32_t ph[4], pl[4];
-            split_bf16(s[0][0], s[0][1], ph[0], pl[0]);
-            split_bf16(s[0][2], s[0][3], ph[1], pl[1]);
-            split_bf16(s[1][0], s[1][1], ph[2], pl[2]);
-            split_bf16(s[1][2], s[1][3], ph[3], pl[3]);
-            // O += P V
-#pragma unroll
-            for (int n2 = 0; n2 < TL::NT / 2; ++n2) {
-                const int mat = lane >> 3;
                 const int rr = (mat & 1) * 8 + (lane & 7);
-                const int c = 2 * n2 + (mat >> 1);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_t(vbase + (rr * TL::CPR + (c ^ (rr & 7))) * 16, v0, v1, v2, v3);
-                mma16816(acc[2 * n2], ph, v0, v1);
-                mma16816(acc[2 * n2], pl, v0, v1);
-                mma16816(acc[2 * n2 + 1], ph, v2, v3);
-                mma16816(acc[2 * n2 + 1], pl, v2, v3);
+                const int c = 2 * kk + (mat >> 1);
+                uint32_t a[4];
+                ldsm_x4(kbase + (rr * TL::CPR + (c ^ (rr & 7))) * 16, a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NH8; ++nt) mma16816(s[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+            }
+            // mask, scale; per-head max over the 16 keys (keys gq, gq + 8 here; xor over gq)
+            const bool kv0 = (vm >> gq) & 1u, kv1 = (vm >> (gq + 8)) & 1u;
+            uint32_t bh[NH8][2], bl[NH8][2];
+#pragma unroll
+            for (int nt = 0; nt < NH8; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float x0 = kv0 ? s[nt][e] * sl2 : -INFINITY;       // key gq
+                    const float x1 = kv1 ? s[nt][2 + e] * sl2 : -INFINITY;   // key gq + 8
+                    float tm = fmaxf(x0, x1);
+                    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+                    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+                    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+                    const float mn = fmaxf(m_r[nt][e], tm);
+                    const float mref = mn == -INFINITY ? 0.f : mn;
+                    const float alpha = exp2f(m_r[nt][e] - mref);
+                    m_r[nt][e] = mn;
+                    const float p0 = exp2f(x0 - mref), p1 = exp2f(x1 - mref);
+                    s[nt][e] = p0;
+                    s[nt][2 + e] = p1;
+                    l_r[nt][e] = l_r[nt][e] * alpha + p0 + p1;
+#pragma unroll
+                    for (int dt = 0; dt < TL::KSTEPS; ++dt) {
+                        acc[dt][nt][e] *= alpha;
+                        acc[dt][nt][2 + e] *= alpha;
+                    }
+                }
+                // P^T into B-operand layout: transpose the two 8x8 (key x head) blocks
+                uint32_t h0, l0, h1, l1;
+                split_bf16(s[nt][0], s[nt][1], h0, l0);     // key gq,     heads 2cq, 2cq+1
+                split_bf16(s[nt][2], s[nt][3], h1, l1);     // key gq + 8
+                bh[nt][0] = movm_t(h0); bh[nt][1] = movm_t(h1);
+                bl[nt][0] = movm_t(l0); bl[nt][1] = movm_t(l1);
+            }
+            // O^T += V^T P^T  (P as hi + lo bf16 terms)
+#pragma unroll
+            for (int dt = 0; dt < TL::KSTEPS; ++dt) {
+                const int mat = lane >> 3;
+                const int rr = (mat >> 1) * 8 + (lane & 7);
+                const int c = 2 * dt + (mat & 1);
+                uint32_t a[4];
+                ldsm_x4_t(vbase + (rr * TL::CPR + (c ^ (rr & 7))) * 16, a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NH8; ++nt) {
+                    mma16816(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
+                    mma16816(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                }
             }
             __syncwarp();   // this stage may be refilled after the next wait
         }
         cp_wait<0>();
+        }   // window
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            l_r[h] += __shfl_xor_sync(0xffffffffu, l_r[h], 1);
-            l_r[h] += __shfl_xor_sync(0xffffffffu, l_r[h], 2);
-        }
+        for (int nt = 0; nt < NH8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                l_r[nt][e] += __shfl_xor_sync(0xffffffffu, l_r[nt][e], 4);
+                l_r[nt][e] += __shfl_xor_sync(0xffffffffu, l_r[nt][e], 8);
+                l_r[nt][e] += __shfl_xor_sync(0xffffffffu, l_r[nt][e], 16);
+            }
 
         // ---- merge the warps: each warp parks (m, l, o) in its own ring
         __syncthreads();
         float* wbuf = reinterpret_cast<float*>(my_ring);      // m[16], l[16], o[16][D]
-        if (cq == 0) {
-            wbuf[gq] = m_r[0]; wbuf[gq + 8] = m_r[1];
-            wbuf[16 + gq] = l_r[0]; wbuf[16 + gq + 8] = l_r[1];
-        }
 #pragma unroll
-        for (int i = 0; i < TL::NT; ++i) {
-            const int col = i * 8 + 2 * cq;
-            wbuf[32 + gq * D + col] = acc[i][0];
-            wbuf[32 + gq * D + col + 1] = acc[i][1];
-            wbuf[32 + (gq + 8) * D + col] = acc[i][2];
-            wbuf[32 + (gq + 8) * D + col + 1] = acc[i][3];
+        for (int nt = 0; nt < NH8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int hd = nt * 8 + 2 * cq + e;
+                if (gq == 0) {
+                    wbuf[hd] = m_r[nt][e];
+                    wbuf[16 + hd] = l_r[nt][e];
+                }
+#pragma unroll
+                for (int dt = 0; dt < TL::KSTEPS; ++dt) {
+                    wbuf[32 + hd * D + dt * 16 + gq] = acc[dt][nt][e];
+                    wbuf[32 + hd * D + dt * 16 + gq + 8] = acc[dt][nt][2 + e];
+                }
+            }
+        if (NH8 == 1 && lane < 8) {     // heads 8..15 absent: empty state
+            wbuf[8 + lane] = -INFINITY;
+            wbuf[24 + lane] = 0.f;
         }
         __syncthreads();
         const bool whole = a == 0 && bnd == tiles_u;
         const int slot = u + cta;
-        float* part = p.partials + size_t(slot) * nh * (D + 2);
+        const size_t n_slots = size_t(U) + gridDim.x;
         for (int i = tid; i < nh * D; i += kAtThreads) {
             const int row = i / D, col = i - row * D;
             float M = -INFINITY;
@@ -398,10 +434,11 @@ attend_kernel(AttendParams p, int U, int nh) {
                 if (p.lse && col == 0)
                     p.lse[size_t(ug.b) * p.Hq + ug.h0 + row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
             } else {
-                part[row * (D + 2) + col] = O;
+                float* part = p.partials + (size_t(row) * n_slots + slot) * (D + 2);
+                part[col] = O;
                 if (col == 0) {
-                    part[row * (D + 2) + D] = M;
-                    part[row * (D + 2) + D + 1] = L;
+                    part[D] = M;
+                    part[D + 1] = L;
                 }
             }
         }
@@ -411,67 +448,93 @@ attend_kernel(AttendParams p, int U, int nh) {
 }
 
 // Log-sum-exp combine of the partials of every unit split over several CTAs.
-// grid (U, heads per unit), 256 threads: warp w merges partials c_lo + w, c_lo + w + 8, ...
-// online (running max, rescaled sums); the eight warp results are merged in warp order.
+// grid (U, heads per unit), 256 threads.  Partials are stored head-major, so the records
+// (o[D], m, l) of one (unit, head) are contiguous: they are staged into shared memory in
+// chunks with every load of a thread issued at once, then merged against the unit's
+// maximum M with a fixed assignment of records to thread groups and a fixed-order sum.
+constexpr int kCombRecs = 48;    // records staged per chunk
+
 template <int D>
 __global__ void __launch_bounds__(256)
-combine_kernel(AttendParams p, int nh) {
-    constexpr int CPL = D / 32;    // columns per lane
+combine_kernel(AttendParams p, int nh, int n_slots) {
+    constexpr int REC = D + 2;
+    constexpr int PAIRS = D / 2;                 // float2 columns
+    constexpr int GROUPS = 256 / PAIRS;          // record groups
+    constexpr int LOADS = (kCombRecs * REC / 2 + 255) / 256;
     const int u = blockIdx.x, row = blockIdx.y;
     const int c_lo = p.unit_ctas[2 * u], c_hi = p.unit_ctas[2 * u + 1];
     if (c_lo < 0 || row >= nh) return;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float M = -INFINITY, L = 0.f, O[CPL];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_c = c_hi - c_lo + 1;
+    const float* base = p.partials + (size_t(row) * n_slots + u + c_lo) * REC;
+
+    __shared__ __align__(16) float st[kCombRecs * REC];
+    __shared__ float s_red[8];
+    __shared__ float sL[GROUPS], sO[GROUPS][D];
+    float mx = -INFINITY;
+    for (int c = tid; c < n_c; c += 256) mx = fmaxf(mx, __ldcg(base + size_t(c) * REC + D));
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) O[j] = 0.f;
-    for (int c = c_lo + warp; c <= c_hi; c += 8) {
-        const float* pp = p.partials + (size_t(u + c) * nh + row) * (D + 2);
-        const float m = __ldcg(pp + D), l = __ldcg(pp + D + 1);
-        float v[CPL];
-#pragma unroll
-        for (int j = 0; j < CPL; ++j) v[j] = __ldcg(pp + lane * CPL + j);
-        const float Mn = fmaxf(M, m);
-        if (Mn == -INFINITY) continue;
-        const float a = exp2f(M - Mn), b = exp2f(m - Mn);
-        L = L * a + l * b;
-#pragma unroll
-        for (int j = 0; j < CPL; ++j) O[j] = O[j] * a + v[j] * b;
-        M = Mn;
-    }
-    __shared__ float sM[8], sL[8], sO[8][D];
-    if (lane == 0) { sM[warp] = M; sL[warp] = L; }
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) sO[warp][lane * CPL + j] = O[j];
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) s_red[warp] = mx;
     __syncthreads();
-    if (warp != 0) return;
-    float Mt = -INFINITY;
-    for (int w = 0; w < 8; ++w) Mt = fmaxf(Mt, sM[w]);
-    const float Mr = Mt == -INFINITY ? 0.f : Mt;
-    float Lt = 0.f, Ot[CPL];
+    float M = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) Ot[j] = 0.f;
-    for (int w = 0; w < 8; ++w) {
-        const float sc = exp2f(sM[w] - Mr);
-        Lt += sL[w] * sc;
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, s_red[w]);
+    const float Mr = M == -INFINITY ? 0.f : M;
+
+    const int pair = tid % PAIRS, grp = tid / PAIRS;
+    float L = 0.f, O0 = 0.f, O1 = 0.f;
+    for (int c0 = 0; c0 < n_c; c0 += kCombRecs) {
+        const int nr = min(kCombRecs, n_c - c0);
+        const int n2 = nr * REC / 2;                     // float2 count (REC is even)
+        const float2* src = reinterpret_cast<const float2*>(base + size_t(c0) * REC);
+        float2 t[LOADS];
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) Ot[j] += sO[w][lane * CPL + j] * sc;
+        for (int k = 0; k < LOADS; ++k) {
+            const int i = tid + k * 256;
+            t[k] = i < n2 ? __ldcg(src + i) : make_float2(0.f, 0.f);
+        }
+        __syncthreads();   // previous chunk consumed
+#pragma unroll
+        for (int k = 0; k < LOADS; ++k) {
+            const int i = tid + k * 256;
+            if (i < n2) reinterpret_cast<float2*>(st)[i] = t[k];
+        }
+        __syncthreads();
+        for (int r = grp; r < nr; r += GROUPS) {
+            const float* rec = st + r * REC;
+            const float sc = exp2f(rec[D] - Mr);
+            L += rec[D + 1] * sc;
+            const float2 o = reinterpret_cast<const float2*>(rec)[pair];
+            O0 += o.x * sc;
+            O1 += o.y * sc;
+        }
+    }
+    if (pair == 0) sL[grp] = L;
+    sO[grp][2 * pair] = O0;
+    sO[grp][2 * pair + 1] = O1;
+    __syncthreads();
+    if (tid >= D) return;
+    float Lt = 0.f, Ot = 0.f;
+#pragma unroll
+    for (int g = 0; g < GROUPS; ++g) {
+        Lt += sL[g];
+        Ot += sO[g][tid];
     }
     const UnitGeom ug = unit_geom(p, u, nh);
-    const size_t ob = (size_t(ug.b) * p.Hq + ug.h0 + row) * D;
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-        const float val = Lt > 0.f ? Ot[j] / Lt : 0.f;
-        const __nv_bfloat16 bv = __float2bfloat16_rn(val);
-        p.out[ob + lane * CPL + j] = *reinterpret_cast<const uint16_t*>(&bv);
-        if (p.out_f32) p.out_f32[ob + lane * CPL + j] = val;
-    }
-    if (p.lse && lane == 0)
-        p.lse[size_t(ug.b) * p.Hq + ug.h0 + row] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
+    const size_t o = (size_t(ug.b) * p.Hq + ug.h0 + row) * D + tid;
+    const float val = Lt > 0.f ? Ot / Lt : 0.f;
+    const __nv_bfloat16 bv = __float2bfloat16_rn(val);
+    p.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
+    if (p.out_f32) p.out_f32[o] = val;
+    if (p.lse && tid == 0)
+        p.lse[size_t(ug.b) * p.Hq + ug.h0 + row] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
 }
 
 template <int D>
 size_t attend_smem(int U) {
-    return align_up(size_t(U + 1) * 4, 128) + size_t(kAtWarps) * kStages * Tile<D>::BYTES;
+    return align_up(size_t(U + 1) * 4, 128) + size_t(kWinTiles) * kRows * 4 +
+           size_t(kAtWarps) * kStages * Tile<D>::BYTES;
 }
 
 }  // namespace
@@ -490,23 +553,20 @@ spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
     const int nh = p.collapse == SPA_COLLAPSE_GROUP_MEAN ? G : 1;
     if (U > kMaxUnits || nh > 16) return SPA_ERR_UNSUPPORTED_SHAPE;
     const int grid = attend_grid();
-    if (p.d == 128) {
-        const size_t sm = attend_smem<128>(U);
-        SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));
-        attend_kernel<128><<<grid, kAtThreads, sm, st>>>(p, U, nh);
-        SPA_CUDA_TRY(cudaGetLastError());
-        combine_kernel<128><<<dim3(U, nh), 256, 0, st>>>(p, nh);
-    } else if (p.d == 64) {
-        const size_t sm = attend_smem<64>(U);
-        SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));
-        attend_kernel<64><<<grid, kAtThreads, sm, st>>>(p, U, nh);
-        SPA_CUDA_TRY(cudaGetLastError());
-        combine_kernel<64><<<dim3(U, nh), 256, 0, st>>>(p, nh);
-    } else {
-        return SPA_ERR_UNSUPPORTED_SHAPE;
+#define SPA_AT_CASE(DD, H8)                                                                                    \
+    if (p.d == DD && (nh + 7) / 8 == H8) {                                                                    \
+        const size_t sm = attend_smem<DD>(U);                                                                 \
+        SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<DD, H8>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                          int(sm)));                                                          \
+        attend_kernel<DD, H8><<<grid, kAtThreads, sm, st>>>(p, U, nh);                                        \
+        SPA_CUDA_TRY(cudaGetLastError());                                                                     \
+        combine_kernel<DD><<<dim3(U, nh), 256, 0, st>>>(p, nh, U + grid);                                     \
+        SPA_CUDA_TRY(cudaGetLastError());                                                                     \
+        return SPA_OK;                                                                                        \
     }
-    SPA_CUDA_TRY(cudaGetLastError());
-    return SPA_OK;
+    SPA_AT_CASE(128, 1) SPA_AT_CASE(128, 2) SPA_AT_CASE(64, 1) SPA_AT_CASE(64, 2)
+#undef SPA_AT_CASE
+    return SPA_ERR_UNSUPPORTED_SHAPE;
 }
 
 }  // namespace spa

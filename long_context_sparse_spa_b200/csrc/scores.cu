@@ -22,7 +22,7 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 // so the result does not depend on the order of accumulation).
 constexpr int kLrThreads = 256;
 constexpr int kLrUnroll = 8;
-constexpr int kLrChunk = 4096;
+constexpr int kLrChunk = 2048;
 
 template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
@@ -34,7 +34,7 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
     constexpr int kRowsPerPass = kLrThreads / 2;
     constexpr int kHb = HIST ? kHistBins : 1;
     __shared__ uint32_t h_cnt[kHb];
-    __shared__ unsigned long long h_mass[MASS ? kHb : 1];
+    __shared__ uint32_t h_mhi[MASS ? kHb : 1], h_mlo[MASS ? kHb : 1];
     __shared__ uint32_t h_max;
 
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
@@ -44,7 +44,7 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
         if (HIST) {
             for (int i = threadIdx.x; i < kHistBins; i += kLrThreads) {
                 h_cnt[i] = 0;
-                if (MASS) h_mass[i] = 0;
+                if (MASS) h_mhi[i] = h_mlo[i] = 0;
             }
             if (threadIdx.x == 0) h_max = 0;
             __syncthreads();
@@ -117,7 +117,14 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
                             const uint32_t bin = key >> 21;
                             my_max = max(my_max, key);
                             atomicAdd(&h_cnt[bin], 1u);
-                            if (MASS) atomicAdd(&h_mass[bin], fixed_mass(sc, bin_top_score(bin)));
+                            if (MASS) {
+                                // the 41-bit fixed-point mass as two 32-bit halves (20 low
+                                // bits, the rest high): with <= kLrChunk = 2048 rows per work
+                                // item neither half can overflow
+                                const unsigned long long e = fixed_mass(sc, bin_top_score(bin));
+                                atomicAdd(&h_mhi[bin], uint32_t(e >> 20));
+                                atomicAdd(&h_mlo[bin], uint32_t(e & 0xfffffu));
+                            }
                         }
                     }
                 }
@@ -134,7 +141,7 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
                 const uint32_t c = h_cnt[i];
                 if (c) {
                     atomicAdd(gc + i, c);
-                    if (MASS) atomicAdd(gm + i, h_mass[i]);
+                    if (MASS) atomicAdd(gm + i, (static_cast<unsigned long long>(h_mhi[i]) << 20) + h_mlo[i]);
                 }
             }
             if (threadIdx.x == 0) atomicMax(hist.max_key + kvu, h_max);

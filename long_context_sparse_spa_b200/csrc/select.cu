@@ -33,7 +33,8 @@ namespace cg = cooperative_groups;
 namespace spa {
 namespace {
 
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 512;
+constexpr int kPerMax = 2048 / kSelThreads;   // histogram bins per thread in a scan
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kMaxCluster = 8;
@@ -166,10 +167,12 @@ select_kernel(SelectParams p, int chunk, int resident) {
             const float4* s4 = reinterpret_cast<const float4*>(srow);
             float4* d4 = reinterpret_cast<float4*>(sv);
             int i = tid;
-            for (; i + 3 * kSelThreads < n4; i += 4 * kSelThreads) {
-                const float4 a = __ldg(s4 + i), b = __ldg(s4 + i + kSelThreads);
-                const float4 c = __ldg(s4 + i + 2 * kSelThreads), d = __ldg(s4 + i + 3 * kSelThreads);
-                d4[i] = a; d4[i + kSelThreads] = b; d4[i + 2 * kSelThreads] = c; d4[i + 3 * kSelThreads] = d;
+            for (; i + 7 * kSelThreads < n4; i += 8 * kSelThreads) {
+                float4 t[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) t[j] = __ldg(s4 + i + j * kSelThreads);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) d4[i + j * kSelThreads] = t[j];
             }
             for (; i < n4; i += kSelThreads) d4[i] = __ldg(s4 + i);
             for (int j = (n4 << 2) + tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
@@ -201,7 +204,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
             sh.found_above_cnt = 0;
             sh.found_above_f64 = 0.0;
         }
-        constexpr int per = kBins / kSelThreads;   // 8 bins per thread, descending
+        constexpr int per = kBins / kSelThreads;   // bins per thread, descending
         uint32_t vc[per];
         double vm[per];
         uint32_t sc = 0;
@@ -255,7 +258,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
         uint32_t target_cnt = 0;
         u64 target_mass = 0;
         if (TOPP) {
-            const double need = (T - cum_mass0) / scale0;
+            const double need = (T - cum_mass0) / (scale0 > 0.0 ? scale0 : 1.0);
             const u64 hb = __ldcg(hm + b0);
             u64 t = need <= 1.0 ? 1ull : (need >= double(hb) ? hb : u64(ceil(need)));
             target_mass = t < 1 ? 1 : t;
@@ -274,36 +277,51 @@ select_kernel(SelectParams p, int chunk, int resident) {
                 if (TOPP) sh.hist_mass[i] = 0;
             }
             __syncthreads();
-            for (int i = tid; i < n; i += kSelThreads) {
-                const float s = val_at(i);
+            auto add = [&](float s) {
                 const uint32_t k = score_key(s);
                 if ((k >> pshift) == prefix) {
                     const uint32_t bin = (k >> shift) & uint32_t(nb - 1);
                     atomicAdd(&sh.hist_cnt[bin], 1u);
                     if (TOPP) atomicAdd(&sh.hist_mass[bin], fixed_mass(s, r0));
                 }
+            };
+            if (resident) {
+                const int n4 = n >> 2;
+                const float4* v4 = reinterpret_cast<const float4*>(sv);
+                for (int i = tid; i < n4; i += kSelThreads) {
+                    const float4 v = v4[i];
+                    add(v.x); add(v.y); add(v.z); add(v.w);
+                }
+                for (int i = (n4 << 2) + tid; i < n; i += kSelThreads) add(sv[i]);
+            } else {
+                for (int i = tid; i < n; i += kSelThreads) add(__ldg(srow + i));
             }
             cluster.sync();   // local histograms complete
             const int per_owner = nb / C;
             for (int bin = rank * per_owner + tid; bin < (rank + 1) * per_owner; bin += kSelThreads) {
+                uint32_t cr[kMaxCluster];
+                u64 mr[kMaxCluster];
+#pragma unroll
+                for (int r = 0; r < kMaxCluster; ++r) {       // every peer load in flight at once
+                    cr[r] = r < C ? *cluster.map_shared_rank(&sh.hist_cnt[bin], r) : 0u;
+                    mr[r] = (TOPP && r < C) ? *cluster.map_shared_rank(&sh.hist_mass[bin], r) : 0ull;
+                }
                 uint32_t c = 0;
                 u64 ms = 0;
-                for (int r = 0; r < C; ++r) {
-                    c += *cluster.map_shared_rank(&sh.hist_cnt[bin], r);
-                    if (TOPP) ms += *cluster.map_shared_rank(&sh.hist_mass[bin], r);
-                }
+#pragma unroll
+                for (int r = 0; r < kMaxCluster; ++r) { c += cr[r]; ms += mr[r]; }   // fixed peer order
                 sh.mrg_cnt[bin] = c;
                 if (TOPP) sh.mrg_mass[bin] = ms;
             }
             cluster.sync();   // merged slices complete
 
-            const int per = nb / kSelThreads;    // 8 or 4 bins per thread, descending
-            uint32_t vc[8];
-            u64 vm[8];
+            const int per = nb / kSelThreads;    // bins per thread, descending
+            uint32_t vc[kPerMax];
+            u64 vm[kPerMax];
             uint32_t sc = 0;
             u64 sm = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < kPerMax; ++j) {
                 vc[j] = 0; vm[j] = 0;
                 if (j < per) {
                     const int bin = nb - 1 - (tid * per + j);
@@ -327,7 +345,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
             uint32_t ac = cum_c + ec;
             u64 am = cum_m + em;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < kPerMax; ++j) {
                 if (j < per) {
                     const bool hit = TOPP ? (am < target_mass && am + vm[j] >= target_mass)
                                           : (ac < target_cnt && ac + vc[j] >= target_cnt);
@@ -428,9 +446,62 @@ select_kernel(SelectParams p, int chunk, int resident) {
         for (int off = 16; off >= 1; off >>= 1) fmass += __shfl_xor_sync(0xffffffffu, fmass, off);
     };
 
+    // common case: resident chunk and no tie split.  Lane l of a step owns the four
+    // consecutive elements [4l, 4l + 4) of a 128-element run; a warp inclusive scan of the
+    // per-lane counts gives the packed offsets (ascending order is lane-major).
+    auto walk4 = [&](uint32_t& nsel_out, double& fmass_out) {
+        uint32_t ns = 0;
+        double fm = 0.0;
+        int* packed = reinterpret_cast<int*>(sv);
+        for (int i0 = w0; i0 < w1; i0 += 128) {
+            const int i = i0 + 4 * lane;
+            float v[4];
+            if (i + 3 < w1) {
+                const float4 t = *reinterpret_cast<const float4*>(sv + i);
+                v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[j] = i + j < w1 ? sv[i + j] : 0.f;
+            }
+            uint32_t flags = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const bool live = i + j < w1;
+                const int pos = lo + i + j;
+                const bool top = live && (select_all || (thresholded && score_key(v[j]) >= tau));
+                const bool f = live && (pos < p.sink || pos >= window_lo);
+                if (TOPP && f && !top) fm += exp(double(v[j]) - double(m));
+                flags |= uint32_t(top || f) << j;
+            }
+            const uint32_t cnt = __popc(flags);
+            uint32_t incl = cnt;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t x = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += x;
+            }
+            uint32_t at = ns + incl - cnt;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (flags >> j & 1u) packed[w0 + at++] = lo + i + j;   // never overtakes the reads
+            ns += __shfl_sync(0xffffffffu, incl, 31);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) fm += __shfl_xor_sync(0xffffffffu, fm, off);
+        nsel_out = ns;
+        fmass_out = fm;
+    };
+
     uint32_t nsel;
     double fmass;
-    walk(resident != 0, false, 0, nsel, fmass);
+    // the vector walk needs 16-byte aligned warp slices of the resident chunk
+    const bool fast = resident && !split_ties && (seg % 4 == 0);
+    if (fast) {
+        __syncwarp();
+        walk4(nsel, fmass);
+    } else {
+        walk(resident != 0, false, 0, nsel, fmass);
+    }
     if (lane == 0) { sh.warp_u32[warp] = nsel; sh.warp_f64[warp] = fmass; }
     __syncthreads();
     uint32_t sel_before_warp = 0;
