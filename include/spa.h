@@ -149,6 +149,29 @@ spa_status spa_select_topp(const float* scores, const int32_t* unit_len, int U, 
 size_t spa_select_workspace_bytes(int U, int M);
 
 /* ------------------------------------------------------------------------------------
+ * Top-p selection that needs no workspace from its caller.  The method pages have no
+ * counterpart: this is an interface addition for callers that cannot allocate device
+ * memory when they call -- for instance an inference server that reserves all device
+ * memory at start-up and forbids allocation on the request path, or a plug-in whose host
+ * framework owns every device buffer.
+ * Arguments and results are those of spa_select_topp without (ws, ws_bytes).  The
+ * scratch (a status word and the level-0 histograms of up to SPA_SELECT_STATIC_MAX_UNITS
+ * units, about 385 KiB) is a fixed array in the library's device memory, held by every GPU
+ * that loads the library until the process exits.  U > SPA_SELECT_STATIC_MAX_UNITS returns
+ * SPA_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks up the array's device
+ * address with cudaGetSymbolAddress (with that device current) and caches it; make that
+ * first call before any stream capture.  Each call clears the part of the array it uses
+ * (cudaMemsetAsync on `stream`) and allocates nothing.  All calls share the one array:
+ * calls that overlap on the GPU (other streams, other host threads on the same device)
+ * race, and the caller must serialise them.  A support larger than cap shows as
+ * count[u] > cap (there is no status word to read back).
+ */
+#define SPA_SELECT_STATIC_MAX_UNITS 16
+spa_status spa_select_topp_static(const float* scores, const int32_t* unit_len, int U, int M, float p,
+                                  int sink, int window, int32_t* idx, int32_t* count, int cap,
+                                  float* index_mass, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * a7/a8. Exact softmax attention on the gathered support ("Oracle-Guided Sparse
  * Prefill" 2.1: recompute with the original Q, K, V restricted to the support;
  * "RTPurbo" Methodology 5: bandwidth-optimised sparse decode).

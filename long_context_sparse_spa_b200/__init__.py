@@ -22,7 +22,7 @@ from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK
 
 __all__ = [
     "SpaError", "lib", "lib_path", "block_stats", "index_scores", "select_topk", "select_topp", "sparse_attend",
-    "decode", "DecodePlan", "workspace", "read_device_status", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
+    "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
     "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SELECT_TOPK", "SPA_SELECT_TOPP",
 ]
 
@@ -124,6 +124,25 @@ def select_topp(scores: torch.Tensor, p: float, sink: int, window: int, cap: Opt
     mass = torch.zeros(U, dtype=torch.float32, device=scores.device)
     check(lib().spa_select_topp(_ptr(scores), _ptr(unit_len), U, M, ctypes.c_float(p), sink, window, _ptr(idx),
                                 _ptr(count), cap, _ptr(mass), _ptr(ws), ws.numel(), _stream()))
+    return idx, count, mass
+
+
+def select_topp_static(scores: torch.Tensor, p: float, sink: int, window: int, cap: Optional[int] = None,
+                       unit_len: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """select_topp without a workspace: for callers that may not allocate device memory when
+    they call (outputs must then be preallocated by them; here they are allocated for
+    convenience).  The library keeps the scratch in a fixed device array shared by all calls,
+    so calls must not overlap on the GPU; at most SPA_SELECT_STATIC_MAX_UNITS units."""
+    _need(scores, torch.float32, "scores")
+    if unit_len is not None:
+        _need(unit_len, torch.int32, "unit_len")
+    U, M = scores.shape
+    cap = M if cap is None else cap
+    idx = torch.full((U, max(cap, 1)), -1, dtype=torch.int32, device=scores.device)
+    count = torch.zeros(U, dtype=torch.int32, device=scores.device)
+    mass = torch.zeros(U, dtype=torch.float32, device=scores.device)
+    check(lib().spa_select_topp_static(_ptr(scores), _ptr(unit_len), U, M, ctypes.c_float(p), sink, window,
+                                       _ptr(idx), _ptr(count), cap, _ptr(mass), _stream()))
     return idx, count, mass
 
 

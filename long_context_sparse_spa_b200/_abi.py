@@ -21,6 +21,7 @@ SPA_SCORE_LOWRANK = 0
 SPA_SCORE_TAYLOR_BLOCK = 1
 SPA_SELECT_TOPK = 0
 SPA_SELECT_TOPP = 1
+SPA_SELECT_STATIC_MAX_UNITS = 16
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -54,6 +55,7 @@ SIGNATURES = {
     "spa_select_topk": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _p, _sz, _p]),
     "spa_select_topp": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p, _sz, _p]),
     "spa_select_workspace_bytes": (_sz, [_i, _i]),
+    "spa_select_topp_static": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p]),
     "spa_sparse_attend": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "spa_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spa_decode": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p]),
