@@ -241,6 +241,43 @@ spa_status spa_decode_timed(const spa_decode_args* a, void* ws, size_t ws_bytes,
                             void* const* events);
 
 /* ------------------------------------------------------------------------------------
+ * a9. Selection-block-shared sparse prefill ("Oracle-Guided Sparse Prefill" 2.1 with
+ * b_sel = bq = 64: one support for 64 consecutive queries; 2.2: head-collapsed indexer).
+ * One chunk of T queries at positions q_start .. q_start + T - 1 of a single sequence,
+ * against the causal cache of N tokens (the chunk's own keys included).  For query block
+ * b (positions t0 = q_start + b*bq ...) and kv head g, unit u = b * Hkv + g:
+ *   index query = mean over the block's bq queries and the G heads of g of q_idx;
+ *   support     = exact top-k of score_scale * index_query . Kidx[g][n] over n < t0,
+ *                 united with the sink [0, sink) (written to idx[u], ascending);
+ *   out[t][h]   = softmax(sm_scale * q K^T) V over the support plus the block's own
+ *                 positions [t0, t] (causal), for every query t of the block and head h of g.
+ * Attention runs on tcgen05 tensor cores with TMEM accumulators.  Requires d = 128,
+ * bq = 64, G = Hq / Hkv even, T a multiple of bq with T / bq <= 128, q_start + T <= N,
+ * cap >= min(N, topk + sink).  ws >= spa_prefill_workspace_bytes.
+ */
+typedef struct spa_prefill_args {
+    int T, Hq, Hkv, N, d, r;
+    int q_start;
+    int bq;                   /* queries per shared support: 64 */
+    const uint16_t* Q;        /* [T, Hq, d] */
+    const uint16_t* q_idx;    /* [T, Hq, r] */
+    const uint16_t* K;        /* [Hkv, N, d] */
+    const uint16_t* V;        /* [Hkv, N, d] */
+    const uint16_t* Kidx;     /* [Hkv, N, r] */
+    float score_scale;
+    float sm_scale;
+    int topk, sink;
+    int32_t* idx;             /* [U, cap] out, U = (T / bq) * Hkv */
+    int32_t* count;           /* [U] out */
+    int cap;
+    uint16_t* out;            /* [T, Hq, d] out */
+    float* out_f32;           /* optional */
+} spa_prefill_args;
+
+spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream);
+size_t spa_prefill_workspace_bytes(const spa_prefill_args* a);
+
+/* ------------------------------------------------------------------------------------
  * Device status word of a workspace (sticky OR of SPA_ERR_* bits as (1 << code)).
  * Synchronises `stream`, copies the word to *bits and, if reset != 0, clears it.
  * Returns SPA_OK or SPA_ERR_CUDA.

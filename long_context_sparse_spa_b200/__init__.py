@@ -18,11 +18,11 @@ from typing import Optional, Tuple
 import torch
 
 from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK, SPA_SCORE_TAYLOR_BLOCK,
-                   SPA_SELECT_TOPK, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, check, lib, lib_path)
+                   SPA_SELECT_TOPK, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
 
 __all__ = [
     "SpaError", "lib", "lib_path", "block_stats", "index_scores", "select_topk", "select_topp", "sparse_attend",
-    "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
+    "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "prefill", "PrefillPlan", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
     "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SELECT_TOPK", "SPA_SELECT_TOPP",
 ]
 
@@ -233,6 +233,55 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
     a.out, a.out_f32, a.lse = _ptr(out), _ptr(out32), _ptr(lse)
     ws = workspace(lib().spa_decode_workspace_bytes(ctypes.byref(a)), dev)
     plan = DecodePlan(a, ws, idx, count, mass, out, out32, lse, (q, K, V, q_idx, Kidx, bmean, bvar))
+    if run:
+        plan.run()
+    return plan
+
+
+# ----------------------------------------------------------------------------- a9 shared-support prefill
+@dataclass
+class PrefillPlan:
+    """Arguments, outputs and workspace of one shared-support prefill call, reusable."""
+
+    args: SpaPrefillArgs
+    ws: torch.Tensor
+    idx: torch.Tensor
+    count: torch.Tensor
+    out: torch.Tensor
+    out_f32: Optional[torch.Tensor]
+    keep: tuple
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        check(lib().spa_prefill_shared(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()),
+                                       self.ws.numel(), _stream(stream)))
+
+
+def prefill(*, Q: torch.Tensor, q_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, Kidx: torch.Tensor,
+            q_start: int, score_scale: float, sm_scale: float, topk: int, sink: int, bq: int = 64,
+            want_f32: bool = True, run: bool = True) -> PrefillPlan:
+    """Selection-block-shared prefill of one query chunk; see spa_prefill_shared in include/spa.h.
+    Q [T, Hq, d], q_idx [T, Hq, r], K/V [Hkv, N, d], Kidx [Hkv, N, r], all bf16."""
+    for t, n in ((Q, "Q"), (q_idx, "q_idx"), (K, "K"), (V, "V"), (Kidx, "Kidx")):
+        _need(t, torch.bfloat16, n)
+    T, Hq, d = Q.shape
+    Hkv, N, _ = K.shape
+    U = (T // bq) * Hkv
+    cap = min(N, topk + sink)
+    dev = Q.device
+    idx = torch.full((U, max(cap, 1)), -1, dtype=torch.int32, device=dev)
+    count = torch.zeros(U, dtype=torch.int32, device=dev)
+    out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=dev)
+    out32 = torch.empty((T, Hq, d), dtype=torch.float32, device=dev) if want_f32 else None
+    a = SpaPrefillArgs()
+    a.T, a.Hq, a.Hkv, a.N, a.d, a.r = T, Hq, Hkv, N, d, q_idx.shape[-1]
+    a.q_start, a.bq = q_start, bq
+    a.Q, a.q_idx, a.K, a.V, a.Kidx = _ptr(Q), _ptr(q_idx), _ptr(K), _ptr(V), _ptr(Kidx)
+    a.score_scale, a.sm_scale = score_scale, sm_scale
+    a.topk, a.sink = topk, sink
+    a.idx, a.count, a.cap = _ptr(idx), _ptr(count), cap
+    a.out, a.out_f32 = _ptr(out), _ptr(out32)
+    ws = workspace(lib().spa_prefill_workspace_bytes(ctypes.byref(a)), dev)
+    plan = PrefillPlan(a, ws, idx, count, out, out32, (Q, q_idx, K, V, Kidx))
     if run:
         plan.run()
     return plan

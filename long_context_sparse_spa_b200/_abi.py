@@ -45,6 +45,18 @@ class SpaDecodeArgs(ctypes.Structure):
     ]
 
 
+class SpaPrefillArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", _i), ("Hq", _i), ("Hkv", _i), ("N", _i), ("d", _i), ("r", _i),
+        ("q_start", _i), ("bq", _i),
+        ("Q", _p), ("q_idx", _p), ("K", _p), ("V", _p), ("Kidx", _p),
+        ("score_scale", _f), ("sm_scale", _f),
+        ("topk", _i), ("sink", _i),
+        ("idx", _p), ("count", _p), ("cap", _i),
+        ("out", _p), ("out_f32", _p),
+    ]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "spa_status_string": (ctypes.c_char_p, [_i]),
@@ -62,6 +74,8 @@ SIGNATURES = {
     "spa_decode_workspace_bytes": (_sz, [ctypes.POINTER(SpaDecodeArgs)]),
     "spa_decode_timed": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p, ctypes.POINTER(_p)]),
     "spa_read_device_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32), _i]),
+    "spa_prefill_shared": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
+    "spa_prefill_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
 }
 
 _LIB = None

@@ -304,6 +304,32 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     return mark(3);
 }
 
+size_t spa_prefill_workspace_bytes(const spa_prefill_args* a) {
+    if (!a || a->bq <= 0 || a->Hkv <= 0 || a->T < 0 || a->N < 0) return 0;
+    const int U = (a->T / a->bq) * a->Hkv;
+    return kWsHeader + prefill_scratch_bytes(U, a->N);
+}
+
+spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {
+    if (!a || !ws) return SPA_ERR_INVALID_ARG;
+    if (a->T < 0 || a->N <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->bq <= 0 ||
+        a->q_start < 0 || a->topk < 0 || a->sink < 0 || a->cap < 0)
+        return SPA_ERR_INVALID_ARG;
+    if (a->T == 0) return SPA_OK;
+    if (!a->Q || !a->q_idx || !a->K || !a->V || !a->Kidx || !a->idx || !a->count || !a->out)
+        return SPA_ERR_INVALID_ARG;
+    const int G = a->Hq / a->Hkv;
+    if (a->d != 128 || a->r != 16 || a->bq != 64 || G % 2 != 0 || G > 16 || a->T % a->bq != 0 ||
+        a->T / a->bq > 128 || a->q_start + a->T > a->N)
+        return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (a->cap < (a->topk + a->sink < a->N ? a->topk + a->sink : a->N)) return SPA_ERR_INVALID_ARG;
+    if (!aligned16(a->Q) || !aligned16(a->q_idx) || !aligned16(a->K) || !aligned16(a->V) || !aligned16(a->Kidx) ||
+        !aligned16(a->out))
+        return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (ws_bytes < spa_prefill_workspace_bytes(a)) return SPA_ERR_WORKSPACE_TOO_SMALL;
+    return launch_prefill(a, ws, static_cast<cudaStream_t>(stream));
+}
+
 spa_status spa_read_device_status(void* ws, void* stream, uint32_t* bits, int reset) {
     if (!ws || !bits) return SPA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

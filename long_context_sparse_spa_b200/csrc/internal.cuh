@@ -122,6 +122,10 @@ spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st);
 spa_status launch_select(const SelectParams& p, bool topp, cudaStream_t st);
 size_t select_scratch_bytes(int U);
 
+// prefill.cu
+size_t prefill_scratch_bytes(int U, int N);
+spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st);
+
 // attend.cu
 struct AttendParams {
     const uint16_t* q;

@@ -48,7 +48,7 @@ def lib() -> ctypes.CDLL:
         L.orc_sparse_attention.argtypes = [_p, _int, _p, _p, _i64, _int, _p, _i64, _int, _dbl, _p, _p]
         L.orc_dense_probs.argtypes = [_p, _int, _p, _i64, _int, _dbl, _p]
         L.orc_prefill_unit.argtypes = [_p, _p, _int, _int, _int, _int, _p, _p, _p, _i64, _i64, _dbl,
-                                       _i64, _i64, _dbl, _int, _p, _p]
+                                       _i64, _i64, _dbl, _int, _p, _p, _p]
         L.orc_prefill_unit.restype = _i64
         _LIB = L
     return _LIB
@@ -143,19 +143,23 @@ def dense_probs(q: np.ndarray, K: np.ndarray, sm_scale: float) -> np.ndarray:
 
 
 def prefill_unit(qblk, qidx_blk, K, V, kidx, t0: int, idx_scale: float, k: int, sink: int,
-                 sm_scale: float, rank_f32: bool = True) -> Tuple[np.ndarray, np.ndarray]:
-    """One (query block, kv head) unit of the shared-support prefill -> (support, out [bq, G, d])."""
+                 sm_scale: float, rank_f32: bool = True, want_scores: bool = False):
+    """One (query block, kv head) unit of the shared-support prefill -> (support, out [bq, G, d])
+    (and the ranked scores [t0] when want_scores)."""
     qblk = _c(qblk, np.uint16); qidx_blk = _c(qidx_blk, np.uint16)
     K = _c(K, np.uint16); V = _c(V, np.uint16); kidx = _c(kidx, np.uint16)
     bq, G, d = qblk.shape
     r = qidx_blk.shape[2]
     support = np.empty(max(1, min(t0, k + sink)), np.int32)
     out = np.empty((bq, G, d))
+    scores = np.empty(max(1, t0)) if want_scores else None
     n = lib().orc_prefill_unit(_ptr(qblk), _ptr(qidx_blk), bq, G, d, r, _ptr(K), _ptr(V), _ptr(kidx),
                                K.shape[0], t0, float(idx_scale), k, sink, float(sm_scale), int(rank_f32),
-                               _ptr(support), _ptr(out))
+                               _ptr(support), _ptr(out), _ptr(scores))
     if n < 0:
         raise ValueError("query block outside the cache")
+    if want_scores:
+        return support[:n].copy(), out, scores[:t0].copy()
     return support[:n].copy(), out
 
 
@@ -236,11 +240,12 @@ def captured_mass(cfg, x: Dict[str, np.ndarray], u: int, idx: np.ndarray) -> flo
     return float(P[rows[rows < cfg.N]].sum())
 
 
-def prefill_block(cfg, x: Dict[str, np.ndarray], j: int, g: int) -> Tuple[np.ndarray, np.ndarray]:
-    """Unit (query block j, kv head g) of a shared-support prefill -> (support, out [bq, G, d])."""
+def prefill_block(cfg, x: Dict[str, np.ndarray], j: int, g: int, want_scores: bool = False):
+    """Unit (query block j, kv head g) of a shared-support prefill -> (support, out [bq, G, d])
+    (and the ranked scores of the candidates [0, t0) when want_scores)."""
     G, bq = cfg.G, cfg.bq
     rows = slice(j * bq, (j + 1) * bq)
     heads = slice(g * G, (g + 1) * G)
     t0 = cfg.q_start + j * bq
     return prefill_unit(x["Q"][rows, heads], x["q_idx"][rows, heads], x["K"][g], x["V"][g], x["Kidx"][g],
-                        t0, f32(cfg.score_scale), cfg.topk, cfg.sink, f32(cfg.sm_scale))
+                        t0, f32(cfg.score_scale), cfg.topk, cfg.sink, f32(cfg.sm_scale), want_scores=want_scores)

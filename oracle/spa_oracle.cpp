@@ -290,12 +290,13 @@ void orc_dense_probs(const uint16_t* q, int G, const uint16_t* K, int64_t N, int
 //    (rounded to binary32 when rank_f32 != 0, the precision a binary32 ranking sees);
 // 3. support = exact top-k of those scores united with the sink [0, sink)
 //    (written ascending to support, room for min(t0, k + sink)); returns its size;
+//    the ranked scores are copied to scores_out [t0] when it is not null;
 // 4. each query t0+i and head h attends, with the original q/K/V, to the support
 //    plus its own block's causal prefix [t0, t0+i]: out [bq, G, d].
 int64_t orc_prefill_unit(const uint16_t* qblk, const uint16_t* qidx_blk, int bq, int G, int d, int r,
                          const uint16_t* K, const uint16_t* V, const uint16_t* kidx, int64_t N,
                          int64_t t0, double idx_scale, int64_t k, int64_t sink, double sm_scale,
-                         int rank_f32, int32_t* support, double* out) {
+                         int rank_f32, int32_t* support, double* out, double* scores_out) {
     if (t0 < 0 || t0 + bq > N) return -1;
     std::vector<double> qhat(r, 0.0);
     for (int i = 0; i < bq; ++i)
@@ -309,6 +310,7 @@ int64_t orc_prefill_unit(const uint16_t* qblk, const uint16_t* qidx_blk, int bq,
         s[n] = idx_scale * dot;
         if (rank_f32) s[n] = static_cast<double>(static_cast<float>(s[n]));
     }
+    if (scores_out) std::copy(s.begin(), s.end(), scores_out);
     const int64_t cnt = t0 > 0 ? orc_select_topk(s.data(), t0, k, sink, 0, support) : 0;
 
     std::vector<int32_t> rows(support, support + cnt);
