@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from synth import DECODE_CONFIGS, decode_inputs  # noqa: E402
+from synth.shard import batch_range, global_config  # noqa: E402
 
 METRIC = "sparse-decode queries/s (query heads per second), 128K-token KV cache"
 UNIT = "queries/s"
@@ -204,9 +205,9 @@ def run_spa(a):
 
     base = DECODE_CONFIGS[a.config]
     # weak scaling: every rank holds its own B sequences (a shard of a global batch of world*B)
-    cfg_global = base.with_(B=base.B * world)
+    cfg_global = global_config(base, world)
     t = time.perf_counter()
-    x = decode_inputs(cfg_global, batch=(rank * base.B, (rank + 1) * base.B))
+    x = decode_inputs(cfg_global, batch=batch_range(base, rank, world))
     log(f"[rank {rank}] inputs generated in {time.perf_counter() - t:.1f} s")
 
     def up(arr):
