@@ -50,7 +50,7 @@ typedef enum spa_status {
     SPA_ERR_UNSUPPORTED_SHAPE = 2,   /* head dim, index dim, group size or alignment not supported */
     SPA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the spa_*_workspace_bytes() figure */
     SPA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed (spa_last_cuda_error) */
-    SPA_ERR_TIMEOUT = 5,             /* device: a bounded wait gave up (reserved; no kernel waits today) */
+    SPA_ERR_TIMEOUT = 5,             /* device: a bounded wait gave up (that call's results are undefined) */
     SPA_ERR_CAPACITY = 6             /* device: a support held more than cap entries (count[u] > cap) */
 } spa_status;
 
