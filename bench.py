@@ -248,10 +248,12 @@ def run_spa(a):
     M = cfg.N // cfg.block
     sparsity = 1.0 - counts.sum() / (cfg.U * M)
 
-    # ---- timed region: K steps, L2 flushed before each, per-kernel events inside each step
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
-    for e4 in ev:
-        for e in e4:
+    # ---- timed region: K steps, L2 flushed before each; a step is bracketed by two events and
+    # runs as one uninterrupted sequence of launches (events between its kernels would stop the
+    # next kernel from being scheduled while the previous one drains)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(a.steps)]
+    for e2 in ev:
+        for e in e2:
             e.record()
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
@@ -262,14 +264,28 @@ def run_spa(a):
     w0 = time.perf_counter()
     for i in range(a.steps):
         flush_l2()
-        plan.run_timed(ev[i])
+        ev[i][0].record()
+        plan.run()
+        ev[i][1].record()
     torch.cuda.synchronize()
     w1 = time.perf_counter()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    step_ms = np.array([ev[i][0].elapsed_time(ev[i][3]) for i in range(a.steps)])
-    k_ms = {name: np.array([ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(a.steps)])
+    step_ms = np.array([ev[i][0].elapsed_time(ev[i][1]) for i in range(a.steps)])
+
+    # ---- per-kernel split (for the roofline of the dominant kernel): a separate, untimed pass
+    # with events between the kernels
+    n_split = min(a.steps, 200)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_split)]
+    for e4 in kev:
+        for e in e4:
+            e.record()
+    for i in range(n_split):
+        flush_l2()
+        plan.run_timed(kev[i])
+    torch.cuda.synchronize()
+    k_ms = {name: np.array([kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(n_split)])
             for j, name in enumerate(("scores", "select", "attend"))}
     dev_s = float(step_ms.sum()) / 1e3
     t_max = dev_s
@@ -350,7 +366,9 @@ def run_spa(a):
             "kernels_ms": {k: round(v, 5) for k, v in mean_ms.items()},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": float(np.mean(e2e_ms))},
-            "gpu_launches": 3 * a.steps,
+            # per step: scores (with the level-0 histogram fused when one score row serves a
+            # kv head), [histogram], selection, attention, log-sum-exp combine
+            "gpu_launches": (4 if (lowrank and cfg.collapse == "group") else 5) * a.steps,
             "clocks": clocks,
             "wall_s_timed_region": w1 - w0,
         }

@@ -126,6 +126,7 @@ __device__ __forceinline__ int tile_owner(long long x, long long TT, int G) {
 template <int D, int NH8>
 __global__ void __launch_bounds__(kAtThreads, 2)
 attend_kernel(AttendParams p, int U, int nh) {
+    pdl_enter();
     using TL = Tile<D>;
     extern __shared__ __align__(128) uint8_t smem[];
     int* s_prefix = reinterpret_cast<int*>(smem);                            // [U + 1]
@@ -457,6 +458,7 @@ constexpr int kCombRecs = 48;    // records staged per chunk
 template <int D>
 __global__ void __launch_bounds__(256)
 combine_kernel(AttendParams p, int nh, int n_slots) {
+    pdl_enter();
     constexpr int REC = D + 2;
     constexpr int PAIRS = D / 2;                 // float2 columns
     constexpr int GROUPS = 256 / PAIRS;          // record groups
@@ -558,10 +560,8 @@ spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
         const size_t sm = attend_smem<DD>(U);                                                                 \
         SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<DD, H8>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                           int(sm)));                                                          \
-        attend_kernel<DD, H8><<<grid, kAtThreads, sm, st>>>(p, U, nh);                                        \
-        SPA_CUDA_TRY(cudaGetLastError());                                                                     \
-        combine_kernel<DD><<<dim3(U, nh), 256, 0, st>>>(p, nh, U + grid);                                     \
-        SPA_CUDA_TRY(cudaGetLastError());                                                                     \
+        SPA_CUDA_TRY(launch_pdl(attend_kernel<DD, H8>, dim3(grid), dim3(kAtThreads), sm, st, p, U, nh));      \
+        SPA_CUDA_TRY(launch_pdl(combine_kernel<DD>, dim3(U, nh), dim3(256), 0, st, p, nh, U + grid));          \
         return SPA_OK;                                                                                        \
     }
     SPA_AT_CASE(128, 1) SPA_AT_CASE(128, 2) SPA_AT_CASE(64, 1) SPA_AT_CASE(64, 2)

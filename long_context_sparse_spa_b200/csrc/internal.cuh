@@ -91,6 +91,34 @@ __device__ __forceinline__ void raise_status(uint32_t* status, int code) {
     if (status) atomicOr(status, 1u << code);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialization, so the
+// hardware may schedule it while the previous kernel of the stream is still draining.  Its
+// first statement waits until that kernel has completed and its memory is visible (a no-op
+// when there is none), and then lets the next kernel be scheduled likewise: dependents
+// become launchable only once every CTA of this grid has started, so CTAs waiting here never
+// hold back a CTA of the grid they wait for.
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ launchers
 // scores.cu
 // hist (optional, GROUP_MEAN only): also accumulate the level-0 histogram of the scores;

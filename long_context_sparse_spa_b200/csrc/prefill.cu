@@ -120,6 +120,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
 // (query, head) order; also unit_len[u] = t0, the number of candidate keys.
 __global__ void prefill_qhat_kernel(const uint16_t* __restrict__ qidx, int Hq, int Hkv, int bq, int q_start,
                                     float* __restrict__ qhat, int32_t* __restrict__ unit_len, int U) {
+    pdl_enter();
     const int u = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16;
     const int dim = threadIdx.x & 15;
     if (u >= U) return;
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(kPsThreads)
 prefill_scores_kernel(const float* __restrict__ qhat, const int32_t* __restrict__ unit_len,
                       const uint4* __restrict__ kidx, int Hkv, int N, int n_blocks, float scale,
                       float* __restrict__ scores) {
+    pdl_enter();
     __shared__ float qs[kPsMaxBlocks][16];
     __shared__ int t0s[kPsMaxBlocks];
     const int g = blockIdx.y;
@@ -201,6 +203,7 @@ struct __align__(1024) PfShared {
 // grid (U, G / 2): one CTA per (unit, pair of query heads); 128 threads.
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_attend_kernel(PrefillAttendParams p) {
+    pdl_enter();
     extern __shared__ __align__(1024) uint8_t dyn[];
     PfShared& sh = *reinterpret_cast<PfShared*>(dyn);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -445,11 +448,11 @@ spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) 
     w += align_up(size_t(U) * a->N * 4, 256);
     const Hist0 hist = hist0_carve(w, U);
 
-    prefill_qhat_kernel<<<(U + 15) / 16, 256, 0, st>>>(a->q_idx, a->Hq, a->Hkv, a->bq, a->q_start, qhat, unit_len, U);
-    SPA_CUDA_TRY(cudaGetLastError());
-    prefill_scores_kernel<<<dim3((a->N + kPsThreads - 1) / kPsThreads, a->Hkv), kPsThreads, 0, st>>>(
-        qhat, unit_len, reinterpret_cast<const uint4*>(a->Kidx), a->Hkv, a->N, n_blocks, a->score_scale, scores);
-    SPA_CUDA_TRY(cudaGetLastError());
+    SPA_CUDA_TRY(launch_pdl(prefill_qhat_kernel, dim3((U + 15) / 16), dim3(256), 0, st, a->q_idx, a->Hq, a->Hkv, a->bq,
+                            a->q_start, qhat, unit_len, U));
+    SPA_CUDA_TRY(launch_pdl(prefill_scores_kernel, dim3((a->N + kPsThreads - 1) / kPsThreads, a->Hkv), dim3(kPsThreads),
+                            0, st, qhat, unit_len, reinterpret_cast<const uint4*>(a->Kidx), a->Hkv, a->N, n_blocks,
+                            a->score_scale, scores));
     SelectParams sp{hist, scores, unit_len, U, a->N, a->topk, 0.f, a->sink, 0, a->idx, a->count, a->cap,
                     nullptr, status};
     spa_status s = launch_hist0(sp, false, st);
@@ -461,8 +464,7 @@ spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) 
                            a->sm_scale, a->out, a->out_f32, status};
     const size_t smem = sizeof(PfShared);
     SPA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    prefill_attend_kernel<<<dim3(U, G / 2), kPfThreads, smem, st>>>(pp);
-    SPA_CUDA_TRY(cudaGetLastError());
+    SPA_CUDA_TRY(launch_pdl(prefill_attend_kernel, dim3(U, G / 2), dim3(kPfThreads), smem, st, pp));
     return SPA_OK;
 }
 

@@ -28,6 +28,7 @@ template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
 lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict__ kidx, int Hq, int Hkv,
                       int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items, Hist0 hist) {
+    pdl_enter();
     const int G = Hq / Hkv;
     const int half = threadIdx.x & 1;          // which 8 of the 16 index dims this lane holds
     const int pair = threadIdx.x >> 1;         // row slot within a pass
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(kTyThreads)
 taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ mean, const float4* __restrict__ var,
                      int Hq, int Hkv, int M, int collapse, float scale, float* __restrict__ scores,
                      int chunks_per_unit, int n_items) {
+    pdl_enter();
     __shared__ float qs[G][D];
     constexpr int kPer = D / 8;          // dims per lane
     constexpr int kVec = kPer / 4;       // float4 loads per lane per tensor
@@ -251,6 +253,7 @@ template <int D, int BLOCK>
 __global__ void __launch_bounds__(128)
 block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, float* __restrict__ mean,
                    float* __restrict__ var) {
+    pdl_enter();
     constexpr int DV = D / 8;                 // 16-byte chunks per row
     constexpr int PH = 128 / DV;              // row phases
     constexpr int RPT = BLOCK / PH;           // rows per thread
@@ -335,29 +338,23 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
     const uint4* k4 = reinterpret_cast<const uint4*>(kidx);
     const Hist0 h = hist ? *hist : Hist0{nullptr, nullptr, nullptr};
     if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
-        if (hist && with_mass)
-            lowrank_scores_kernel<1, true, true><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores,
-                                                                              chunks, items, h);
-        else if (hist)
-            lowrank_scores_kernel<1, true, false><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores,
-                                                                               chunks, items, h);
-        else
-            lowrank_scores_kernel<1, false, false><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores,
-                                                                                chunks, items, h);
+        auto kern = hist && with_mass ? lowrank_scores_kernel<1, true, true>
+                                      : (hist ? lowrank_scores_kernel<1, true, false> : lowrank_scores_kernel<1, false, false>);
+        SPA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kLrThreads), 0, st, qidx, k4, Hq, Hkv, M, scale, scores, chunks,
+                                items, h));
     } else {
         if (hist) return SPA_ERR_INVALID_ARG;
         switch (G) {
 #define SPA_LR_CASE(n)                                                                                          \
     case n:                                                                                                     \
-        lowrank_scores_kernel<n, false, false><<<grid, kLrThreads, 0, st>>>(qidx, k4, Hq, Hkv, M, scale, scores, \
-                                                                            chunks, items, h);                  \
+        SPA_CUDA_TRY(launch_pdl(lowrank_scores_kernel<n, false, false>, dim3(grid), dim3(kLrThreads), 0, st, qidx, \
+                                k4, Hq, Hkv, M, scale, scores, chunks, items, h));                              \
         break;
             SPA_LR_CASE(1) SPA_LR_CASE(2) SPA_LR_CASE(4) SPA_LR_CASE(8) SPA_LR_CASE(16)
 #undef SPA_LR_CASE
             default: return SPA_ERR_UNSUPPORTED_SHAPE;
         }
     }
-    SPA_CUDA_TRY(cudaGetLastError());
     return SPA_OK;
 }
 
@@ -371,9 +368,8 @@ spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const floa
     const float4* v4 = reinterpret_cast<const float4*>(var);
 #define SPA_TY_CASE(D, GG)                                                                                  \
     if (d == D && G == GG) {                                                                               \
-        taylor_scores_kernel<D, GG><<<grid, kTyThreads, 0, st>>>(q, m4, v4, Hq, Hkv, M, collapse, scale, scores, \
-                                                                  chunks, items);                         \
-        SPA_CUDA_TRY(cudaGetLastError());                                                                  \
+        SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG>, dim3(grid), dim3(kTyThreads), 0, st, q, m4, v4, Hq,  \
+                                Hkv, M, collapse, scale, scores, chunks, items));                           \
         return SPA_OK;                                                                                     \
     }
     SPA_TY_CASE(64, 1) SPA_TY_CASE(64, 2) SPA_TY_CASE(64, 4) SPA_TY_CASE(64, 8) SPA_TY_CASE(64, 16)
@@ -391,8 +387,8 @@ spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, i
     const uint4* k4 = reinterpret_cast<const uint4*>(K);
 #define SPA_BS_CASE(D, BL)                                                                       \
     if (d == D && block == BL) {                                                                \
-        block_stats_kernel<D, BL><<<grid, 128, 0, st>>>(k4, n_blocks, nb, N, mean, var);        \
-        SPA_CUDA_TRY(cudaGetLastError());                                                       \
+        SPA_CUDA_TRY(launch_pdl(block_stats_kernel<D, BL>, dim3(grid), dim3(128), 0, st, k4,    \
+                                n_blocks, nb, N, mean, var));                                   \
         return SPA_OK;                                                                          \
     }
     SPA_BS_CASE(64, 32) SPA_BS_CASE(64, 64) SPA_BS_CASE(64, 128)

@@ -99,6 +99,7 @@ constexpr int kH0Chunk = 4096;
 template <bool MASS>
 __global__ void __launch_bounds__(kH0Threads)
 hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
+    pdl_enter();
     __shared__ uint32_t h_cnt[kBins];
     __shared__ u64 h_mass[MASS ? kBins : 1];
     __shared__ uint32_t h_max;
@@ -144,6 +145,7 @@ hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
 template <bool TOPP>
 __global__ void __launch_bounds__(kSelThreads, 2)
 select_kernel(SelectParams p, int chunk, int resident) {
+    pdl_enter();
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
     const int rank = int(cluster.block_rank());
@@ -629,13 +631,15 @@ spa_status launch_t(const SelectParams& p, cudaStream_t st) {
     cfg.blockDim = dim3(kSelThreads, 1, 1);
     cfg.dynamicSmemBytes = c.smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = c.C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_enter()
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     SPA_CUDA_TRY(cudaLaunchKernelEx(&cfg, select_kernel<TOPP>, p, c.chunk, c.resident));
     return SPA_OK;
 }
@@ -650,9 +654,8 @@ spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st) 
     if (items == 0) return SPA_OK;
     const int cap = device_info().num_sms * 8;
     const int grid = items < cap ? items : cap;
-    if (with_mass) hist0_kernel<true><<<grid, kH0Threads, 0, st>>>(p, chunks, items);
-    else hist0_kernel<false><<<grid, kH0Threads, 0, st>>>(p, chunks, items);
-    SPA_CUDA_TRY(cudaGetLastError());
+    if (with_mass) SPA_CUDA_TRY(launch_pdl(hist0_kernel<true>, dim3(grid), dim3(kH0Threads), 0, st, p, chunks, items));
+    else SPA_CUDA_TRY(launch_pdl(hist0_kernel<false>, dim3(grid), dim3(kH0Threads), 0, st, p, chunks, items));
     return SPA_OK;
 }
 
