@@ -56,7 +56,8 @@ __device__ __forceinline__ float key_score(uint32_t k) {
 // score a key of bin b can hold, so the sums need no knowledge of the unit's maximum and
 // are exact integers whatever the order of accumulation; plus the unit's largest key.
 // Producers (the fused scoring kernel, or the histogram kernel) add into it; the selection
-// kernel reads it and zeroes it again for the next call.
+// kernel reads it and zeroes it again for the next call, likewise the finer levels' merged
+// histograms it keeps beside it.
 constexpr int kHistBins = 2048;
 constexpr float kMassScale = 1099511627776.0f;   // 2^40
 
@@ -64,10 +65,15 @@ struct Hist0 {
     uint32_t* cnt;                 // [U][2048]
     unsigned long long* mass;      // [U][2048]
     uint32_t* max_key;             // [U]
+    // the selection kernel's merged level-1 (2048 bins) and level-2 (1024 bins) histograms
+    uint32_t* lvl_cnt;             // [U][3072]
+    unsigned long long* lvl_mass;  // [U][3072]
 };
+constexpr int kLvlBins = 3072;
 inline size_t hist0_bytes(int U) {
     return align_up(size_t(U) * kHistBins * 4, 256) + align_up(size_t(U) * kHistBins * 8, 256) +
-           align_up(size_t(U) * 4, 256);
+           align_up(size_t(U) * 4, 256) + align_up(size_t(U) * kLvlBins * 4, 256) +
+           align_up(size_t(U) * kLvlBins * 8, 256);
 }
 inline Hist0 hist0_carve(void* base, int U) {
     uint8_t* b = static_cast<uint8_t*>(base);
@@ -77,6 +83,10 @@ inline Hist0 hist0_carve(void* base, int U) {
     h.mass = reinterpret_cast<unsigned long long*>(b);
     b += align_up(size_t(U) * kHistBins * 8, 256);
     h.max_key = reinterpret_cast<uint32_t*>(b);
+    b += align_up(size_t(U) * 4, 256);
+    h.lvl_cnt = reinterpret_cast<uint32_t*>(b);
+    b += align_up(size_t(U) * kLvlBins * 4, 256);
+    h.lvl_mass = reinterpret_cast<unsigned long long*>(b);
     return h;
 }
 // largest score a key of level-0 bin b can hold (bin 2047 holds only +inf/NaN patterns)

@@ -22,7 +22,9 @@ constexpr int kStaticUnits = SPA_SELECT_STATIC_MAX_UNITS;
 constexpr size_t kStaticHistBytes =
     ((size_t(kStaticUnits) * kHistBins * 4 + 255) / 256) * 256 +
     ((size_t(kStaticUnits) * kHistBins * 8 + 255) / 256) * 256 +
-    ((size_t(kStaticUnits) * 4 + 255) / 256) * 256;
+    ((size_t(kStaticUnits) * 4 + 255) / 256) * 256 +
+    ((size_t(kStaticUnits) * kLvlBins * 4 + 255) / 256) * 256 +
+    ((size_t(kStaticUnits) * kLvlBins * 8 + 255) / 256) * 256;
 constexpr size_t kStaticScratchBytes = kWsHeader + kStaticHistBytes;
 
 // status word (first 256 bytes) + level-0 histogram of up to kStaticUnits units
@@ -67,7 +69,7 @@ extern "C" spa_status spa_select_topp_static(const float* scores, const int32_t*
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the array keeps the previous call's contents: start from a zero status word and
     // zero histograms (the part this call uses)
-    const size_t used = kWsHeader + hist0_bytes(U);
+    const size_t used = kWsHeader + hist0_bytes(U);   // never above kStaticScratchBytes (U <= kStaticUnits)
     SPA_CUDA_TRY(cudaMemsetAsync(scratch, 0, used, st));
     uint8_t* w = static_cast<uint8_t*>(scratch);
     SelectParams sp{hist0_carve(w + kWsHeader, U), scores, unit_len, U, M, 0, p, sink, window, idx, count, cap,

@@ -42,11 +42,14 @@ constexpr double kInvMassScale = 1.0 / 1099511627776.0;   // 2^-40
 
 using u64 = unsigned long long;
 
+// A CTA's local histogram sums fixed-point masses (< 2^41) in three 14-bit parts with 32-bit
+// shared atomics (a 64-bit shared atomic is several times slower); a part cannot overflow while
+// the chunk holds at most kPartSafe scores, longer chunks use 64-bit sums (aliased storage).
+constexpr int kPartSafe = 1 << 18;
+
 struct SelShared {
     uint32_t hist_cnt[kBins];     // local histogram of the current level (levels 1 and 2)
-    u64 hist_mass[kBins];
-    uint32_t mrg_cnt[kBins];      // merged histogram of the bins this CTA owns
-    u64 mrg_mass[kBins];
+    uint32_t hist_part[3][kBins];
     uint32_t warp_u32[kSelWarps];
     u64 warp_u64[kSelWarps];
     double warp_f64[kSelWarps];
@@ -274,9 +277,19 @@ select_kernel(SelectParams p, int chunk, int resident) {
             const int shift = level == 1 ? 10 : 0;
             const int nb = level == 1 ? 2048 : 1024;
             const int pshift = level == 1 ? 21 : 10;
+            const bool wide = n > kPartSafe;
+            u64* hist_wide = reinterpret_cast<u64*>(&sh.hist_part[0][0]);
             for (int i = tid; i < nb; i += kSelThreads) {
                 sh.hist_cnt[i] = 0;
-                if (TOPP) sh.hist_mass[i] = 0;
+                if (TOPP) {
+                    if (wide) {
+                        hist_wide[i] = 0;
+                    } else {
+                        sh.hist_part[0][i] = 0;
+                        sh.hist_part[1][i] = 0;
+                        sh.hist_part[2][i] = 0;
+                    }
+                }
             }
             __syncthreads();
             auto add = [&](float s) {
@@ -284,7 +297,16 @@ select_kernel(SelectParams p, int chunk, int resident) {
                 if ((k >> pshift) == prefix) {
                     const uint32_t bin = (k >> shift) & uint32_t(nb - 1);
                     atomicAdd(&sh.hist_cnt[bin], 1u);
-                    if (TOPP) atomicAdd(&sh.hist_mass[bin], fixed_mass(s, r0));
+                    if (TOPP) {
+                        const u64 m = fixed_mass(s, r0);
+                        if (wide) {
+                            atomicAdd(&hist_wide[bin], m);
+                        } else {
+                            atomicAdd(&sh.hist_part[0][bin], uint32_t(m) & 0x3fffu);
+                            atomicAdd(&sh.hist_part[1][bin], uint32_t(m >> 14) & 0x3fffu);
+                            atomicAdd(&sh.hist_part[2][bin], uint32_t(m >> 28));
+                        }
+                    }
                 }
             };
             if (resident) {
@@ -298,24 +320,25 @@ select_kernel(SelectParams p, int chunk, int resident) {
             } else {
                 for (int i = tid; i < n; i += kSelThreads) add(__ldg(srow + i));
             }
-            cluster.sync();   // local histograms complete
-            const int per_owner = nb / C;
-            for (int bin = rank * per_owner + tid; bin < (rank + 1) * per_owner; bin += kSelThreads) {
-                uint32_t cr[kMaxCluster];
-                u64 mr[kMaxCluster];
-#pragma unroll
-                for (int r = 0; r < kMaxCluster; ++r) {       // every peer load in flight at once
-                    cr[r] = r < C ? *cluster.map_shared_rank(&sh.hist_cnt[bin], r) : 0u;
-                    mr[r] = (TOPP && r < C) ? *cluster.map_shared_rank(&sh.hist_mass[bin], r) : 0ull;
+            __syncthreads();
+            // the unit's merged histogram: every CTA adds its nonzero bins with global
+            // reductions (integer sums: the result does not depend on their order)
+            const int goff = level == 1 ? 0 : kBins;
+            uint32_t* gcnt = p.hist.lvl_cnt + size_t(u) * kLvlBins + goff;
+            u64* gmass = p.hist.lvl_mass + size_t(u) * kLvlBins + goff;
+            for (int i = tid; i < nb; i += kSelThreads) {
+                const uint32_t c = sh.hist_cnt[i];
+                if (c) {
+                    atomicAdd(gcnt + i, c);
+                    if (TOPP) {
+                        const u64 m = wide ? hist_wide[i]
+                                           : u64(sh.hist_part[0][i]) + (u64(sh.hist_part[1][i]) << 14) +
+                                                 (u64(sh.hist_part[2][i]) << 28);
+                        atomicAdd(gmass + i, m);
+                    }
                 }
-                uint32_t c = 0;
-                u64 ms = 0;
-#pragma unroll
-                for (int r = 0; r < kMaxCluster; ++r) { c += cr[r]; ms += mr[r]; }   // fixed peer order
-                sh.mrg_cnt[bin] = c;
-                if (TOPP) sh.mrg_mass[bin] = ms;
             }
-            cluster.sync();   // merged slices complete
+            cluster.sync();   // every CTA's reductions are performed (release / acquire at cluster scope)
 
             const int per = nb / kSelThreads;    // bins per thread, descending
             uint32_t vc[kPerMax];
@@ -327,9 +350,8 @@ select_kernel(SelectParams p, int chunk, int resident) {
                 vc[j] = 0; vm[j] = 0;
                 if (j < per) {
                     const int bin = nb - 1 - (tid * per + j);
-                    const int owner = bin / per_owner;
-                    vc[j] = *cluster.map_shared_rank(&sh.mrg_cnt[bin], owner);
-                    if (TOPP) vm[j] = *cluster.map_shared_rank(&sh.mrg_mass[bin], owner);
+                    vc[j] = __ldcg(gcnt + bin);
+                    if (TOPP) vm[j] = __ldcg(gmass + bin);
                     sc += vc[j];
                     sm += vm[j];
                 }
@@ -538,6 +560,10 @@ select_kernel(SelectParams p, int chunk, int resident) {
         for (int i = tid; i < kBins; i += kSelThreads) {
             p.hist.cnt[size_t(u) * kBins + i] = 0;
             p.hist.mass[size_t(u) * kBins + i] = 0;
+        }
+        for (int i = tid; i < kLvlBins; i += kSelThreads) {
+            p.hist.lvl_cnt[size_t(u) * kLvlBins + i] = 0;
+            p.hist.lvl_mass[size_t(u) * kLvlBins + i] = 0;
         }
         if (tid == 0) {
             p.hist.max_key[u] = 0;
