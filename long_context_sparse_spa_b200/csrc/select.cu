@@ -46,6 +46,8 @@ using u64 = unsigned long long;
 // shared atomics (a 64-bit shared atomic is several times slower); a part cannot overflow while
 // the chunk holds at most kPartSafe scores, longer chunks use 64-bit sums (aliased storage).
 constexpr int kPartSafe = 1 << 18;
+constexpr uint32_t kLoadSpinLimit = 1u << 24;   // bounded polls of the chunk-load barrier
+constexpr int kBulkPiece = 32768;               // bytes per bulk copy of the chunk load
 
 struct SelShared {
     uint32_t hist_cnt[kBins];     // local histogram of the current level (levels 1 and 2)
@@ -53,8 +55,9 @@ struct SelShared {
     uint32_t warp_u32[kSelWarps];
     u64 warp_u64[kSelWarps];
     double warp_f64[kSelWarps];
-    uint32_t cta_sel;             // selected count of this CTA (published to peers)
-    double cta_fmass;             // mass of forced-only elements of this CTA (published)
+    uint32_t sel_of[kMaxCluster];   // selected count of every CTA of the cluster (pushed by each)
+    double fmass_of[kMaxCluster];   // mass of every CTA's forced-only elements (pushed by each)
+    u64 load_bar;                   // completion of the chunk's bulk copy
     uint32_t found_bin;
     uint32_t found_above_cnt;
     u64 found_above_mass;
@@ -165,27 +168,48 @@ select_kernel(SelectParams p, int chunk, int resident) {
     const int n = hi - lo;
     const float* srow = p.scores + size_t(u) * p.M + lo;
 
-    // ---- the chunk into shared memory (128-bit loads when the row slice is aligned)
-    if (resident) {
-        if ((reinterpret_cast<uintptr_t>(srow) & 15) == 0) {
-            const int n4 = n >> 2;
-            const float4* s4 = reinterpret_cast<const float4*>(srow);
-            float4* d4 = reinterpret_cast<float4*>(sv);
-            int i = tid;
-            for (; i + 7 * kSelThreads < n4; i += 8 * kSelThreads) {
-                float4 t[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) t[j] = __ldg(s4 + i + j * kSelThreads);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) d4[i + j * kSelThreads] = t[j];
+    // ---- the chunk into shared memory: bulk asynchronous copies when the row slice is
+    // 16-byte aligned (they run while the level-0 scan below executes), else plain loads
+    const int n16 = (reinterpret_cast<uintptr_t>(srow) & 15) == 0 ? (n & ~3) : 0;
+    const bool bulk = resident && n16 > 0;
+    const uint32_t bar = uint32_t(__cvta_generic_to_shared(&sh.load_bar));
+    if (bulk) {
+        if (tid == 0) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar));
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // the init precedes the copies
+            const uint32_t bytes = uint32_t(n16) * 4u;
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+            const uint32_t dst = uint32_t(__cvta_generic_to_shared(sv));
+            for (uint32_t off = 0; off < bytes; off += kBulkPiece) {
+                const uint32_t piece = min(uint32_t(kBulkPiece), bytes - off);
+                asm volatile(
+                    "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                        dst + off),
+                    "l"(reinterpret_cast<const uint8_t*>(srow) + off), "r"(piece), "r"(bar)
+                    : "memory");
             }
-            for (; i < n4; i += kSelThreads) d4[i] = __ldg(s4 + i);
-            for (int j = (n4 << 2) + tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
-        } else {
-            for (int j = tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
         }
+        for (int j = n16 + tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
+    } else if (resident) {
+        for (int j = tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
     }
-    __syncthreads();   // the resident chunk is read by every warp below
+    auto wait_chunk = [&]() {
+        if (bulk) {
+            uint32_t ok = 0;
+            for (uint32_t it = 0; !ok; ++it) {
+                asm volatile(
+                    "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n selp.u32 %0, 1, 0, q;\n}\n"
+                    : "=r"(ok)
+                    : "r"(bar)
+                    : "memory");
+                if (!ok && it >= kLoadSpinLimit) {
+                    raise_status(p.status, SPA_ERR_TIMEOUT);
+                    break;
+                }
+            }
+        }
+        __syncthreads();   // the resident chunk (bulk part and tail) is visible to every warp
+    };
     auto val_at = [&](int i) -> float { return resident ? sv[i] : __ldg(srow + i); };
 
     bool select_all = false, select_none = false;
@@ -214,15 +238,20 @@ select_kernel(SelectParams p, int chunk, int resident) {
         double vm[per];
         uint32_t sc = 0;
         double sm = 0.0;
+        u64 mb[per];
 #pragma unroll
         for (int j = 0; j < per; ++j) {
             const int bin = kBins - 1 - (tid * per + j);
             vc[j] = __ldcg(hc + bin);
+            mb[j] = TOPP ? __ldcg(hm + bin) : 0ull;
+        }
+#pragma unroll
+        for (int j = 0; j < per; ++j) {
+            const int bin = kBins - 1 - (tid * per + j);
             vm[j] = 0.0;
-            if (TOPP) {
-                const u64 mb = __ldcg(hm + bin);
-                if (mb) vm[j] = double(mb) * kInvMassScale * exp(double(bin_top_score(bin)) - double(m));
-            }
+            // fp64 exp only in warps that hold mass (most bins are empty)
+            if (TOPP && __any_sync(0xffffffffu, mb[j] != 0) && mb[j])
+                vm[j] = double(mb[j]) * kInvMassScale * exp(double(bin_top_score(bin)) - double(m));
             sc += vc[j];
             sm += vm[j];
         }
@@ -255,6 +284,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
     }
     const float r0 = bin_top_score(b0);                       // mass reference inside B0
     const double scale0 = TOPP ? kInvMassScale * exp(double(r0) - double(m)) : 0.0;
+    wait_chunk();
 
     // ---- levels 1 and 2 inside B0
     uint32_t tau = 0, q = 0, cnt_tau = 0, bin_last = 0;
@@ -414,6 +444,8 @@ select_kernel(SelectParams p, int chunk, int resident) {
     const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
     const int window_lo = L - p.window;
     const unsigned lt_mask = (1u << lane) - 1u;
+    // whether this warp's slice holds a forced position (sink or window)
+    const bool fx_slice = w0 < w1 && (lo + w0 < p.sink || lo + w1 > window_lo);
 
     // ties before each warp are needed only when the quota splits the run of equal keys
     int64_t q_warp = int64_t(q);
@@ -487,15 +519,20 @@ select_kernel(SelectParams p, int chunk, int resident) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) v[j] = i + j < w1 ? sv[i + j] : 0.f;
             }
-            uint32_t flags = 0;
+            uint32_t flags = 0, fx = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const bool live = i + j < w1;
                 const int pos = lo + i + j;
                 const bool top = live && (select_all || (thresholded && score_key(v[j]) >= tau));
-                const bool f = live && (pos < p.sink || pos >= window_lo);
-                if (TOPP && f && !top) fm += exp(double(v[j]) - double(m));
+                const bool f = fx_slice && live && (pos < p.sink || pos >= window_lo);
+                fx |= uint32_t(f && !top) << j;
                 flags |= uint32_t(top || f) << j;
+            }
+            if (TOPP && __any_sync(0xffffffffu, fx != 0)) {   // forced-only elements are few
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (fx >> j & 1u) fm += exp(double(v[j]) - double(m));
             }
             const uint32_t cnt = __popc(flags);
             uint32_t incl = cnt;
@@ -530,21 +567,24 @@ select_kernel(SelectParams p, int chunk, int resident) {
     __syncthreads();
     uint32_t sel_before_warp = 0;
     for (int w = 0; w < warp; ++w) sel_before_warp += sh.warp_u32[w];
-    if (tid == 0) {
+    if (tid < C) {   // this CTA's totals, pushed into every CTA of the cluster
         uint32_t t = 0;
         double fm = 0.0;
         for (int w = 0; w < kSelWarps; ++w) { t += sh.warp_u32[w]; fm += sh.warp_f64[w]; }
-        sh.cta_sel = t;
-        sh.cta_fmass = fm;
+        SelShared& peer = *cluster.map_shared_rank(&sh, tid);
+        peer.sel_of[rank] = t;
+        peer.fmass_of[rank] = fm;
     }
-    cluster.sync();   // CTA counts visible to peers; every CTA is past its level-0 reads
+    // the counts are in place; every CTA is past its reads of the histograms and of its peers'
+    // shared memory, so after this barrier no CTA touches another's
+    cluster.sync();
     uint32_t sel_before_cta = 0, total = 0;
     double fmass_total = 0.0;
     for (int r = 0; r < C; ++r) {
-        const uint32_t c = *cluster.map_shared_rank(&sh.cta_sel, r);
+        const uint32_t c = sh.sel_of[r];
         if (r < rank) sel_before_cta += c;
         total += c;
-        if (TOPP) fmass_total += *cluster.map_shared_rank(&sh.cta_fmass, r);
+        if (TOPP) fmass_total += sh.fmass_of[r];
     }
     const uint32_t base = sel_before_cta + sel_before_warp;
     if (resident) {
@@ -576,7 +616,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
             }
         }
     }
-    cluster.sync();   // no CTA leaves while a peer may still read its shared memory
+    // no barrier here: after the count barrier no CTA reads or writes another's shared memory
 }
 
 struct SelectConfig {
