@@ -31,7 +31,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import DECODE_CONFIGS, decode_inputs  # noqa: E402
+from synth import DECODE_CONFIGS, decode_inputs, prefill_inputs  # noqa: E402
+from synth.configs import C5  # noqa: E402
 from synth.shard import batch_range, global_config  # noqa: E402
 
 METRIC = "sparse-decode queries/s (query heads per second), 128K-token KV cache"
@@ -50,7 +51,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
-    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS))
+    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS) + ["c5"],
+                    help="decode workload (default), or c5: the selection-block-shared prefill")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
@@ -384,8 +386,136 @@ def run_spa(a):
     return 0
 
 
+def bf16_dev(x):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def prefill_flops(cfg, counts):
+    """Algorithmic flops of one prefill chunk: query row i of a block attends to the block's
+    support and to the block's own rows up to i (QK^T and PV: 4 d flops per (query head, key))."""
+    diag = cfg.bq * (cfg.bq + 1) // 2                 # sum over the block's rows of (i + 1)
+    keys = cfg.bq * counts.astype(np.int64) + diag    # per unit and query head
+    return float(4 * cfg.d * cfg.G * keys.sum())
+
+
+def run_prefill(a):
+    """--config c5: the selection-block-shared prefill (one chunk of T queries), in TFLOP/s of
+    its algorithmic flops; the L2 is flushed before every step."""
+    import oracle
+
+    cfg = C5
+    if a.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    x = prefill_inputs(cfg)
+    if a.impl == "reference":       # the fp64 oracle on host cores, one (query block, kv head) unit per step
+        units = [(j, g) for j in range(cfg.n_blocks) for g in range(cfg.Hkv)]
+        flops, t_tot = 0.0, 0.0
+        for i in range(a.warmup + a.steps):
+            j, g = units[i % len(units)]
+            t0 = time.perf_counter()
+            sup, _ = oracle.prefill_block(cfg, x, j, g)
+            dt = time.perf_counter() - t0
+            if i >= a.warmup:
+                flops += prefill_flops(cfg.with_(T=cfg.bq), np.array([sup.size]))
+                t_tot += dt
+        v = flops / t_tot / 1e12
+        print(json.dumps({"impl": "reference", "metric": "sparse-prefill TFLOP/s (algorithmic)", "value": v,
+                          "unit": "TFLOP/s", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+                          "ms_per_step": t_tot / a.steps * 1e3, "higher_is_better": True, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": f"{cfg.name} prefill, one unit per step"},
+                          "cpu_baseline": {"kind": "oracle", "cores": 1, "value": v,
+                                           "sample": f"{a.steps} (query block, kv head) units, fp64 oracle"},
+                          "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return 0
+    import torch
+
+    import long_context_sparse_spa_b200 as spa
+
+    plan = spa.prefill(Q=bf16_dev(x["Q"]), q_idx=bf16_dev(x["q_idx"]), K=bf16_dev(x["K"]), V=bf16_dev(x["V"]),
+                       Kidx=bf16_dev(x["Kidx"]), q_start=cfg.q_start, score_scale=float(np.float32(cfg.score_scale)),
+                       sm_scale=float(np.float32(cfg.sm_scale)), topk=cfg.topk, sink=cfg.sink, want_f32=False,
+                       run=False)
+    wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    for _ in range(a.warmup):
+        wbuf.zero_(); rbuf.sum(); plan.run()
+    torch.cuda.synchronize()
+    assert spa.read_device_status(plan.ws) == 0, "device status raised during warm-up"
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(a.steps)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(a.steps):
+        wbuf.zero_(); rbuf.sum()
+        ev[i][0].record(); plan.run(); ev[i][1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    counts = plan.count.cpu().numpy()
+    flops = prefill_flops(cfg, counts)
+    tflops = flops / (ms * 1e-3) / 1e12
+    # end to end: the chunk's queries (Q, q_idx) from pinned host memory, output read back
+    hq = [torch.from_numpy(np.ascontiguousarray(x[k]).view(np.int16)).pin_memory() for k in ("Q", "q_idx")]
+    dq = [plan.keep[0], plan.keep[1]]
+    hout = torch.empty(plan.out.shape, dtype=plan.out.dtype).pin_memory()
+    n_e2e = min(a.steps, 50)
+    e2e = []
+    for i in range(n_e2e + 2):
+        wbuf.zero_(); rbuf.sum(); torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for h, d in zip(hq, dq):
+            d.view(torch.int16).copy_(h, non_blocking=True)
+        plan.run()
+        hout.copy_(plan.out, non_blocking=True)
+        s1.record(); s1.synchronize()
+        if i >= 2:
+            e2e.append(s0.elapsed_time(s1))
+    e2e_ms = float(np.mean(e2e))
+    peak = None
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    peak_kind = "measured" if peak else "fallback"
+    peak = peak or 1590.0
+    # the oracle on a bounded sample of units (one host core per unit, all cores)
+    cpu = None
+    if not a.no_cpu_baseline:
+        units = [(j, g) for j in range(cfg.n_blocks) for g in range(cfg.Hkv)]
+        t0, done, cf = time.perf_counter(), 0, 0.0
+        while time.perf_counter() - t0 < a.cpu_seconds and done < len(units):
+            j, g = units[done]
+            sup, _ = oracle.prefill_block(cfg, x, j, g)
+            cf += prefill_flops(cfg.with_(T=cfg.bq), np.array([sup.size]))
+            done += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": cf / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": f"{done} (query block, kv head) units of {cfg.name}, fp64 oracle, {dt:.1f} s"}
+    out = {"metric": "sparse-prefill TFLOP/s (algorithmic), selection-block-shared", "value": tflops,
+           "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"{cfg.name}: prefill chunk T={cfg.T} at q_start={cfg.q_start}, N={cfg.N}, "
+                                  f"Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} bq={cfg.bq} top-k={cfg.topk} sink={cfg.sink}",
+                      "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
+                      "support_mean": float(counts.mean()), "algorithmic_gflop_per_step": flops / 1e9},
+           "roofline": {"bound": "tensor", "kernel": "prefill (all kernels of the step)", "achieved": tflops,
+                        "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
+                        "traffic": None},
+           "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": int(sum(h.numel() * 2 for h in hq)),
+                   "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms},
+           "gpu_launches": 6 * a.steps, "clocks": clocks, "cpu_baseline": cpu}
+    print(json.dumps(out))
+    return 0
+
+
 def main():
     a = parse()
+    if a.config == "c5":
+        return run_prefill(a)
     if a.impl == "reference":
         return run_reference(a)
     return run_spa(a)

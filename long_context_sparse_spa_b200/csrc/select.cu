@@ -347,6 +347,23 @@ select_kernel(SelectParams p, int chunk, int resident) {
                     add(v.x); add(v.y); add(v.z); add(v.w);
                 }
                 for (int i = (n4 << 2) + tid; i < n; i += kSelThreads) add(sv[i]);
+            } else if ((reinterpret_cast<uintptr_t>(srow) & 15) == 0) {
+                // streaming chunk (too long for shared memory): four float4 loads in flight
+                const int n4 = n >> 2;
+                const float4* s4 = reinterpret_cast<const float4*>(srow);
+                int i = tid;
+                for (; i + 3 * kSelThreads < n4; i += 4 * kSelThreads) {
+                    float4 v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) v[j] = __ldg(s4 + i + j * kSelThreads);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) { add(v[j].x); add(v[j].y); add(v[j].z); add(v[j].w); }
+                }
+                for (; i < n4; i += kSelThreads) {
+                    const float4 v = __ldg(s4 + i);
+                    add(v.x); add(v.y); add(v.z); add(v.w);
+                }
+                for (int j = (n4 << 2) + tid; j < n; j += kSelThreads) add(__ldg(srow + j));
             } else {
                 for (int i = tid; i < n; i += kSelThreads) add(__ldg(srow + i));
             }
@@ -454,9 +471,18 @@ select_kernel(SelectParams p, int chunk, int resident) {
         uint32_t before = 0;
         for (int r = 0; r < rank; ++r) before += *cluster.map_shared_rank(&sh.hist_cnt[bin_last], r);
         uint32_t wt = 0;
-        for (int i0 = w0; i0 < w1; i0 += 32) {
-            const int i = i0 + lane;
-            wt += __popc(__ballot_sync(0xffffffffu, i < w1 && score_key(val_at(i)) == tau));
+        for (int g0 = w0; g0 < w1; g0 += 256) {
+            float vals[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = g0 + 32 * j + lane;
+                vals[j] = i < w1 ? val_at(i) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = g0 + 32 * j + lane;
+                wt += __popc(__ballot_sync(0xffffffffu, i < w1 && score_key(vals[j]) == tau));
+            }
         }
         if (lane == 0) sh.warp_u32[warp] = wt;
         __syncthreads();
@@ -472,31 +498,43 @@ select_kernel(SelectParams p, int chunk, int resident) {
         nsel = 0;
         fmass = 0.0;
         int* packed = reinterpret_cast<int*>(sv);
-        for (int i0 = w0; i0 < w1; i0 += 32) {
-            const int i = i0 + lane;
-            const bool live = i < w1;
-            const float s = live ? val_at(i) : 0.f;
-            const uint32_t k = score_key(s);
-            const int pos = lo + i;
-            bool top = false, tie = false;
-            if (select_all) top = live;
-            else if (thresholded) {
-                top = live && k > tau;
-                tie = live && k == tau;
+        constexpr int kAhead = 8;     // groups of 32 scores loaded ahead (streaming chunk)
+        for (int g0 = w0; g0 < w1; g0 += 32 * kAhead) {
+            float vals[kAhead];
+#pragma unroll
+            for (int j = 0; j < kAhead; ++j) {
+                const int i = g0 + 32 * j + lane;
+                vals[j] = i < w1 ? val_at(i) : 0.f;
             }
-            const unsigned tb = __ballot_sync(0xffffffffu, tie);
-            if (tie) top = !split_ties || int64_t(run_tie + __popc(tb & lt_mask)) < q_warp;
-            run_tie += __popc(tb);
-            const bool f = live && (pos < p.sink || pos >= window_lo);
-            const bool sel = top || f;
-            if (TOPP && f && !top) fmass += exp(double(s) - double(m));
-            const unsigned sb = __ballot_sync(0xffffffffu, sel);
-            if (sel) {
-                const uint32_t at = nsel + __popc(sb & lt_mask);
-                if (pack) packed[w0 + at] = pos;     // at <= i: never overtakes the reads
-                if (write && base + at < uint32_t(p.cap)) p.idx[size_t(u) * p.cap + base + at] = pos;
+#pragma unroll
+            for (int j = 0; j < kAhead; ++j) {
+                const int i0 = g0 + 32 * j;
+                if (i0 >= w1) break;                      // warp-uniform
+                const int i = i0 + lane;
+                const bool live = i < w1;
+                const float s = vals[j];
+                const uint32_t k = score_key(s);
+                const int pos = lo + i;
+                bool top = false, tie = false;
+                if (select_all) top = live;
+                else if (thresholded) {
+                    top = live && k > tau;
+                    tie = live && k == tau;
+                }
+                const unsigned tb = __ballot_sync(0xffffffffu, tie);
+                if (tie) top = !split_ties || int64_t(run_tie + __popc(tb & lt_mask)) < q_warp;
+                run_tie += __popc(tb);
+                const bool f = fx_slice && live && (pos < p.sink || pos >= window_lo);
+                const bool sel = top || f;
+                if (TOPP && __any_sync(0xffffffffu, f && !top) && f && !top) fmass += exp(double(s) - double(m));
+                const unsigned sb = __ballot_sync(0xffffffffu, sel);
+                if (sel) {
+                    const uint32_t at = nsel + __popc(sb & lt_mask);
+                    if (pack) packed[w0 + at] = pos;     // at <= i: never overtakes the reads
+                    if (write && base + at < uint32_t(p.cap)) p.idx[size_t(u) * p.cap + base + at] = pos;
+                }
+                nsel += __popc(sb);
             }
-            nsel += __popc(sb);
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) fmass += __shfl_xor_sync(0xffffffffu, fmass, off);
