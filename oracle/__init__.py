@@ -175,13 +175,22 @@ def decode_units(cfg) -> List[Tuple[int, int]]:
     return [(b, h) for b in range(cfg.B) for h in range(heads)]
 
 
+def local_support(M: int, sink: int, window: int) -> np.ndarray:
+    """Support of a local head ("Full Attention Strikes Back" (RTPurbo), Methodology 1: local
+    heads attend through a sliding window with an attention sink): the selection units
+    [0, sink) and [M - window, M), ascending, without duplicates."""
+    return np.union1d(np.arange(min(sink, M)), np.arange(max(0, M - window), M)).astype(np.int32)
+
+
 def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.ndarray, np.ndarray]] = None,
-                with_output: bool = True) -> Dict[str, object]:
+                with_output: bool = True, local: bool = False) -> Dict[str, object]:
     """The sparse decode path of one unit: scores -> support -> attention.
 
     Returns scores (float64, as computed), the ranked scores (binary32-rounded; for
     Taylor scores their natural log), the support, the index mass (top-p), the output
-    [heads, d] and lse [heads] of the query heads sharing the support.
+    [heads, d] and lse [heads] of the query heads sharing the support.  A local unit
+    (head-wise routing, RTPurbo Methodology 1) is not scored: its support is the sink and
+    the window, and it has no index mass.
     """
     b, h = decode_units(cfg)[u]
     G = cfg.G
@@ -190,6 +199,15 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
     else:
         g, heads = h, slice(h * G, (h + 1) * G)
     res: Dict[str, object] = {"b": b, "g": g}
+    if local:
+        idx = local_support(cfg.M, cfg.sink, cfg.window)
+        res.update(scores=None, ranked=None, index_mass=None, idx=idx)
+        if with_output:
+            out, lse = sparse_attention(x["q"][b, heads], x["K"][b, g], x["V"][b, g], idx, f32(cfg.sm_scale),
+                                        cfg.block)
+            res["out"] = out
+            res["lse"] = lse
+        return res
     if cfg.score == "lowrank":
         s = lowrank_scores(x["q_idx"][b, heads], x["Kidx"][b, g], cfg.collapse == "group", f32(cfg.score_scale))
         s = s.reshape(-1)                 # one row: the group's shared scores, or the one head's
@@ -218,13 +236,15 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
 
 
 def decode(cfg, x: Dict[str, np.ndarray], units: Optional[Sequence[int]] = None, threads: int = 1,
-           with_output: bool = True) -> List[Dict[str, object]]:
-    """decode_unit over several units, optionally on a thread pool (the C calls release the GIL)."""
+           with_output: bool = True, local: Optional[Sequence[bool]] = None) -> List[Dict[str, object]]:
+    """decode_unit over several units, optionally on a thread pool (the C calls release the GIL);
+    local[u] marks the local units of a head-wise routing."""
     todo = list(range(cfg.U)) if units is None else list(units)
+    loc = (lambda u: bool(local[u])) if local is not None else (lambda u: False)
     if threads <= 1:
-        return [decode_unit(cfg, x, u, with_output=with_output) for u in todo]
+        return [decode_unit(cfg, x, u, with_output=with_output, local=loc(u)) for u in todo]
     with ThreadPoolExecutor(threads) as ex:
-        return list(ex.map(lambda u: decode_unit(cfg, x, u, with_output=with_output), todo))
+        return list(ex.map(lambda u: decode_unit(cfg, x, u, with_output=with_output, local=loc(u)), todo))
 
 
 def captured_mass(cfg, x: Dict[str, np.ndarray], u: int, idx: np.ndarray) -> float:

@@ -291,3 +291,35 @@ def test_decode_driver_c1():
         needles = x["needles"][(b, h // C1.G)]
         mine = [n for i, n in enumerate(sorted(needles)) if True]
         assert len(set(mine) & set(idx.tolist())) >= 1
+
+
+# ------------------------------------------------------------------ head-wise routing (local units)
+@pytest.mark.parametrize("M,sink,window", [(100, 4, 16), (10, 4, 8), (5, 0, 0), (7, 9, 2), (1, 1, 1)])
+def test_local_support_is_sink_and_window(M, sink, window):
+    """Brute force over the positions: a local unit keeps n < sink or n >= M - window."""
+    want = [n for n in range(M) if n < sink or n >= M - window]
+    assert oracle.local_support(M, sink, window).tolist() == want
+
+
+def test_routed_decode_local_units_attend_over_sink_and_window():
+    """A local unit of a routed decode attends over exactly its sink and window (torch fp64
+    attention over those rows); the retrieval units are the unrouted path."""
+    cfg = SMALL["c2s"]
+    x = decode_inputs(cfg)
+    local = [u % 2 == 1 for u in range(cfg.U)]
+    routed = oracle.decode(cfg, x, local=local)
+    plain = oracle.decode(cfg, x)
+    for u, (r, q) in enumerate(zip(routed, plain)):
+        if not local[u]:
+            np.testing.assert_array_equal(r["idx"], q["idx"])
+            np.testing.assert_array_equal(r["out"], q["out"])
+            continue
+        assert r["index_mass"] is None and r["scores"] is None
+        rows = [n for n in range(cfg.N) if n < cfg.sink or n >= cfg.N - cfg.window]
+        assert r["idx"].tolist() == rows
+        b, g = r["b"], r["g"]
+        heads = slice(g * cfg.G, (g + 1) * cfg.G)
+        qf = bf16_value(x["q"][b, heads]).astype(np.float64)
+        Kf = bf16_value(x["K"][b, g][rows]).astype(np.float64)
+        Vf = bf16_value(x["V"][b, g][rows]).astype(np.float64)
+        np.testing.assert_allclose(r["out"], _sdpa(qf, Kf, Vf, oracle.f32(cfg.sm_scale)), rtol=1e-10, atol=1e-12)
