@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS) + ["c5"],
                     help="decode workload (default), or c5: the selection-block-shared prefill")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--local-fraction", type=float, default=0.0,
+                    help="head-wise routing: this fraction of every sequence's units is local (sink + window)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
     if a.steps is None:
@@ -139,7 +141,7 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline(cfg, x, seconds: float):
+def cpu_baseline(cfg, x, seconds: float, local=None):
     """The fp64 oracle's sparse path (scores -> selection -> attention), as it stands, on the
     host cores: units of the same workload cycled until the time budget is spent."""
     import oracle
@@ -149,7 +151,7 @@ def cpu_baseline(cfg, x, seconds: float):
     done = 0
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < seconds:      # whole rounds over all units
-        oracle.decode(cfg, x, units=units, threads=cores)
+        oracle.decode(cfg, x, units=units, threads=cores, local=local)
         done += len(units)
     dt = time.perf_counter() - t0
     return {"value": done * cfg.heads_per_unit / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -230,6 +232,12 @@ def run_spa(a):
     else:
         bm, bv = spa.block_stats(dK, cfg.block)      # once per filled block, off the per-step path
         kw.update(bmean=bm, bvar=bv)
+    # head-wise routing: the first round(f * units per sequence) units of every sequence are local
+    units_per_seq = cfg.U // cfg.B
+    n_local = int(round(a.local_fraction * units_per_seq))
+    local_np = np.array([int(u % units_per_seq < n_local) for u in range(cfg.U)], np.uint8)
+    if n_local:
+        kw["local_units"] = torch.from_numpy(local_np).cuda()
     plan = spa.decode(**kw)
     wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
@@ -302,8 +310,12 @@ def run_spa(a):
     d = cfg.d
     if lowrank:
         score_bytes = cfg.B * cfg.Hkv * cfg.N * cfg.r * 2 + cfg.B * cfg.Hq * cfg.r * 2
+        if cfg.collapse == "group":      # a local unit's index keys are not read
+            score_bytes -= int(local_np.sum()) * cfg.N * cfg.r * 2
     else:
         score_bytes = 2 * cfg.B * cfg.Hkv * M * d * 4 + cfg.B * cfg.Hq * d * 2
+        if cfg.collapse == "group":      # a local unit's block statistics are not read
+            score_bytes -= int(local_np.sum()) * 2 * M * d * 4
     attend_bytes = rows * KV_ROW_BYTES(d) + 2 * cfg.B * cfg.Hq * d * 2
     step_bytes = score_bytes + attend_bytes
     peak, peak_kind = peaks()
@@ -363,6 +375,7 @@ def run_spa(a):
                        "parallelism": f"dp{world} (independent sequence shards, no collective on the data path)",
                        "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
                        "support_rows_per_step": rows, "sparsity": round(float(sparsity), 4),
+                       "local_units": int(local_np.sum()),
                        "algorithmic_bytes_per_step": step_bytes},
             "roofline": roofline,
             "kernels_ms": {k: round(v, 5) for k, v in mean_ms.items()},
@@ -375,7 +388,7 @@ def run_spa(a):
             "wall_s_timed_region": w1 - w0,
         }
         if not a.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(cfg, x, a.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(cfg, x, a.cpu_seconds, local=local_np if n_local else None)
         elif world > 1:
             line["cpu_baseline"] = None
     if world > 1:

@@ -229,6 +229,13 @@ typedef struct spa_decode_args {
     uint16_t* out;           /* [B, Hq, d] out */
     float* out_f32;          /* optional */
     float* lse;              /* optional */
+    /* Head-wise routing ("Full Attention Strikes Back" (RTPurbo), Methodology 1: local heads
+     * attend through a sliding window with an attention sink, retrieval heads through the
+     * dynamic sparse selection).  local_units[u] != 0 makes unit u local: it is not scored
+     * (GROUP_MEAN: its index keys are not read) and its support is [0, sink) and
+     * [M - window, M) only; its index_mass is 0.  NULL: every unit is a retrieval unit.
+     * [U] bytes, device memory, read-only. */
+    const uint8_t* local_units;
 } spa_decode_args;
 
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream);

@@ -201,8 +201,10 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
            bmean: Optional[torch.Tensor] = None, bvar: Optional[torch.Tensor] = None, block: int = 1,
            score_scale: float, sm_scale: float, topk: int = 0, topp: float = 0.0, sink: int = 0,
            window: int = 0, cap: Optional[int] = None, want_f32: bool = True, want_lse: bool = True,
-           run: bool = True) -> DecodePlan:
-    """Build (and by default run) a fused decode step; see spa_decode in include/spa.h."""
+           local_units: Optional[torch.Tensor] = None, run: bool = True) -> DecodePlan:
+    """Build (and by default run) a fused decode step; see spa_decode in include/spa.h.
+    local_units: optional uint8 [U] on the device, nonzero for the units that head-wise routing
+    makes local (support = sink + window, not scored)."""
     for t, n in ((q, "q"), (K, "K"), (V, "V")):
         _need(t, torch.bfloat16, n)
     B, Hq, d = q.shape
@@ -231,8 +233,13 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
     a.idx, a.count, a.cap = _ptr(idx), _ptr(count), cap
     a.index_mass = _ptr(mass)
     a.out, a.out_f32, a.lse = _ptr(out), _ptr(out32), _ptr(lse)
+    if local_units is not None:
+        _need(local_units, torch.uint8, "local_units")
+        if local_units.numel() != U:
+            raise ValueError(f"local_units must hold one flag per unit ({U})")
+    a.local_units = _ptr(local_units)
     ws = workspace(lib().spa_decode_workspace_bytes(ctypes.byref(a)), dev)
-    plan = DecodePlan(a, ws, idx, count, mass, out, out32, lse, (q, K, V, q_idx, Kidx, bmean, bvar))
+    plan = DecodePlan(a, ws, idx, count, mass, out, out32, lse, (q, K, V, q_idx, Kidx, bmean, bvar, local_units))
     if run:
         plan.run()
     return plan

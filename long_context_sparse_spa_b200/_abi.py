@@ -42,6 +42,7 @@ class SpaDecodeArgs(ctypes.Structure):
         ("idx", _p), ("count", _p), ("cap", _i),
         ("index_mass", _p),
         ("out", _p), ("out_f32", _p), ("lse", _p),
+        ("local_units", _p),
     ]
 
 

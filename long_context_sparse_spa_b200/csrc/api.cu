@@ -73,7 +73,7 @@ const char* spa_status_string(int s) {
 
 const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
-int spa_abi_version(void) { return 1; }
+int spa_abi_version(void) { return 2; }
 
 spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean, float* var,
                            void* stream) {
@@ -282,16 +282,16 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     if ((s = mark(0)) != SPA_OK) return s;
     if (taylor) {
         s = launch_taylor_scores(a->q, a->bmean, a->bvar, a->B, a->Hq, a->Hkv, M, a->d, a->collapse,
-                                 a->score_scale, scores, st);
+                                 a->score_scale, scores, st, a->local_units);
     } else {
         s = launch_lowrank_scores(a->q_idx, a->Kidx, a->B, a->Hq, a->Hkv, M, a->collapse, a->score_scale, scores,
-                                  fused_hist ? &hist : nullptr, topp, st);
+                                  fused_hist ? &hist : nullptr, topp, st, a->local_units);
     }
     if (s != SPA_OK) return s;
 
     // 2. selection
     SelectParams sp{hist, scores, nullptr, U, M, a->topk, a->topp, a->sink, a->window, a->idx, a->count, a->cap,
-                    a->index_mass, status};
+                    a->index_mass, status, a->local_units};
     if (!fused_hist && (s = launch_hist0(sp, topp, st)) != SPA_OK) return s;
     if ((s = mark(1)) != SPA_OK) return s;
     s = launch_select(sp, topp, st);

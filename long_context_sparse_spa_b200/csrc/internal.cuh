@@ -133,11 +133,13 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // scores.cu
 // hist (optional, GROUP_MEAN only): also accumulate the level-0 histogram of the scores;
 // with_mass adds the fixed-point masses (top-p), else counts only.
+// local (optional, GROUP_MEAN): [B * Hkv] flags of units that are not scored (head-wise routing)
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
                                  int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
-                                 cudaStream_t st);
+                                 cudaStream_t st, const uint8_t* local = nullptr);
 spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
-                                int M, int d, int collapse, float scale, float* scores, cudaStream_t st);
+                                int M, int d, int collapse, float scale, float* scores, cudaStream_t st,
+                                const uint8_t* local = nullptr);
 spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean,
                               float* var, cudaStream_t st);
 
@@ -155,6 +157,7 @@ struct SelectParams {
     int cap;
     float* index_mass;
     uint32_t* status;
+    const uint8_t* local;   // [U] or null: local units (head-wise routing) select only sink + window
 };
 spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st);
 spa_status launch_select(const SelectParams& p, bool topp, cudaStream_t st);

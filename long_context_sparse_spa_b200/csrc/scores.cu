@@ -27,7 +27,8 @@ constexpr int kLrChunk = 2048;
 template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
 lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict__ kidx, int Hq, int Hkv,
-                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items, Hist0 hist) {
+                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items, Hist0 hist,
+                      const uint8_t* __restrict__ local) {
     pdl_enter();
     const int G = Hq / Hkv;
     const int half = threadIdx.x & 1;          // which 8 of the 16 index dims this lane holds
@@ -42,6 +43,7 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
         const int kvu = item / chunks_per_unit;        // b * Hkv + g
         const int chunk = item - kvu * chunks_per_unit;
         const int b = kvu / Hkv, g = kvu - b * Hkv;
+        if (NQ == 1 && local && local[kvu]) continue;  // a local unit is not scored (uniform per CTA)
         if (HIST) {
             for (int i = threadIdx.x; i < kHistBins; i += kLrThreads) {
                 h_cnt[i] = 0;
@@ -163,7 +165,7 @@ template <int D, int G>
 __global__ void __launch_bounds__(kTyThreads)
 taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ mean, const float4* __restrict__ var,
                      int Hq, int Hkv, int M, int collapse, float scale, float* __restrict__ scores,
-                     int chunks_per_unit, int n_items) {
+                     int chunks_per_unit, int n_items, const uint8_t* __restrict__ local) {
     pdl_enter();
     __shared__ float qs[G][D];
     constexpr int kPer = D / 8;          // dims per lane
@@ -177,6 +179,8 @@ taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ 
         const int kvu = item / chunks_per_unit;
         const int chunk = item - kvu * chunks_per_unit;
         const int b = kvu / Hkv, g = kvu - b * Hkv;
+        // a local unit (GROUP_MEAN: one unit per kv head) is not scored (uniform per CTA)
+        if (collapse == SPA_COLLAPSE_GROUP_MEAN && local && local[kvu]) continue;
         if (kvu != cur_kvu) {
             __syncthreads();
             for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
@@ -330,7 +334,7 @@ int grid_for(int items, int per_sm) {
 
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
                                  int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, const uint8_t* local) {
     const int G = Hq / Hkv;
     const int chunks = (M + kLrChunk - 1) / kLrChunk;
     const int items = B * Hkv * chunks;
@@ -341,14 +345,14 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
         auto kern = hist && with_mass ? lowrank_scores_kernel<1, true, true>
                                       : (hist ? lowrank_scores_kernel<1, true, false> : lowrank_scores_kernel<1, false, false>);
         SPA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kLrThreads), 0, st, qidx, k4, Hq, Hkv, M, scale, scores, chunks,
-                                items, h));
+                                items, h, local));
     } else {
         if (hist) return SPA_ERR_INVALID_ARG;
         switch (G) {
 #define SPA_LR_CASE(n)                                                                                          \
     case n:                                                                                                     \
         SPA_CUDA_TRY(launch_pdl(lowrank_scores_kernel<n, false, false>, dim3(grid), dim3(kLrThreads), 0, st, qidx, \
-                                k4, Hq, Hkv, M, scale, scores, chunks, items, h));                              \
+                                k4, Hq, Hkv, M, scale, scores, chunks, items, h, nullptr));                     \
         break;
             SPA_LR_CASE(1) SPA_LR_CASE(2) SPA_LR_CASE(4) SPA_LR_CASE(8) SPA_LR_CASE(16)
 #undef SPA_LR_CASE
@@ -359,7 +363,8 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
 }
 
 spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
-                                int M, int d, int collapse, float scale, float* scores, cudaStream_t st) {
+                                int M, int d, int collapse, float scale, float* scores, cudaStream_t st,
+                                const uint8_t* local) {
     const int G = Hq / Hkv;
     const int chunks = (M + kTyChunk - 1) / kTyChunk;
     const int items = B * Hkv * chunks;
@@ -369,7 +374,7 @@ spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const floa
 #define SPA_TY_CASE(D, GG)                                                                                  \
     if (d == D && G == GG) {                                                                               \
         SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG>, dim3(grid), dim3(kTyThreads), 0, st, q, m4, v4, Hq,  \
-                                Hkv, M, collapse, scale, scores, chunks, items));                           \
+                                Hkv, M, collapse, scale, scores, chunks, items, local));                    \
         return SPA_OK;                                                                                     \
     }
     SPA_TY_CASE(64, 1) SPA_TY_CASE(64, 2) SPA_TY_CASE(64, 4) SPA_TY_CASE(64, 8) SPA_TY_CASE(64, 16)

@@ -114,7 +114,7 @@ hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
         const int chunk = item - u * chunks_per_unit;
         const int L = p.unit_len ? min(max(p.unit_len[u], 0), p.M) : p.M;
         const int n0 = chunk * kH0Chunk, n1 = min(L, n0 + kH0Chunk);
-        if (n0 >= n1) continue;
+        if (n0 >= n1 || (p.local && p.local[u])) continue;   // local units are not selected from
         for (int i = threadIdx.x; i < kBins; i += kH0Threads) {
             h_cnt[i] = 0;
             if (MASS) h_mass[i] = 0;
@@ -212,10 +212,12 @@ select_kernel(SelectParams p, int chunk, int resident) {
     };
     auto val_at = [&](int i) -> float { return resident ? sv[i] : __ldg(srow + i); };
 
-    bool select_all = false, select_none = false;
+    // a local unit (head-wise routing) keeps its sink and window only
+    const bool local = p.local && p.local[u];
+    bool select_all = false, select_none = local;
     if (!TOPP) {
-        select_all = p.topk >= L;
-        select_none = p.topk <= 0;
+        select_all = !local && p.topk >= L;
+        select_none = local || p.topk <= 0;
     }
     const bool thresholded = L > 0 && !select_all && !select_none;
 

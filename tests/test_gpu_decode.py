@@ -20,7 +20,7 @@ if not torch.cuda.is_available():
 import long_context_sparse_spa_b200 as spa  # noqa: E402
 
 
-def run_gpu(cfg, x):
+def run_gpu(cfg, x, local=None):
     lowrank = cfg.score == "lowrank"
     kw = dict(
         score_kind=spa.SPA_SCORE_LOWRANK if lowrank else spa.SPA_SCORE_TAYLOR_BLOCK,
@@ -34,6 +34,8 @@ def run_gpu(cfg, x):
     else:
         mean, var = spa.block_stats(kw["K"], cfg.block)   # off the per-step path: once per filled block
         kw.update(bmean=mean, bvar=var)
+    if local is not None:
+        kw["local_units"] = torch.from_numpy(np.asarray(local, np.uint8)).cuda()
     plan = spa.decode(**kw)
     torch.cuda.synchronize()
     assert spa.read_device_status(plan.ws) == 0
@@ -93,3 +95,30 @@ def test_decode_c1():
 @pytest.mark.parametrize("cfg", [C2, C2_128K, C3, C4], ids=lambda c: c.name)
 def test_decode_full_size(cfg):
     check_decode(cfg, report_mass=True)
+
+
+@pytest.mark.parametrize("name", ["c1s", "c2s", "c3s"])
+def test_decode_routed(name):
+    """Head-wise routing: every other unit is local (support = sink + window, exactly), the
+    others run the sparse selection; every unit is compared with the oracle's routed path."""
+    cfg = SMALL[name]
+    x = decode_inputs(cfg)
+    local = np.array([u % 2 for u in range(cfg.U)], np.uint8)
+    g = run_gpu(cfg, x, local=local)
+    G = cfg.G
+    for u, (b, h) in enumerate(oracle.decode_units(cfg)):
+        r = oracle.decode_unit(cfg, x, u, local=bool(local[u]))
+        got = g["idx"][u, :g["count"][u]]
+        if local[u]:
+            np.testing.assert_array_equal(got, r["idx"])
+            d = 0
+        else:
+            s = r["ranked"]
+            band = topk_band(s, cfg.topk) if cfg.select == "topk" else topp_band(s, oracle.f32(cfg.topp))
+            d = compare_support(got, r["idx"], band, f"{cfg.name} unit {u}")
+        if d == 0:
+            heads = slice(h, h + 1) if cfg.collapse == "head" else slice(h * G, (h + 1) * G)
+            check_outputs(g["out"][b, heads], g["out32"][b, heads], r["out"], f"{cfg.name} routed unit {u}")
+            np.testing.assert_allclose(g["lse"][b, heads], r["lse"], rtol=2e-6, atol=2e-6)
+            if g["mass"] is not None and not local[u]:
+                assert abs(g["mass"][u] - r["index_mass"]) <= 4 * MASS_TIE_REL + 1e-6
