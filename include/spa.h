@@ -75,7 +75,7 @@ const char* spa_status_string(int status);
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
 const char* spa_last_cuda_error(void);
 
-/* ABI version of this header: 1. */
+/* ABI version of this header: 2 (spa_decode_args gained local_units). */
 int spa_abi_version(void);
 
 /* ------------------------------------------------------------------------------------
