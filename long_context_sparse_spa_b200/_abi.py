@@ -7,6 +7,8 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(HERE, "libspa.so")
 
+ABI_VERSION = 2   # spa_abi_version() of the library these declarations describe
+
 SPA_OK = 0
 SPA_ERR_INVALID_ARG = 1
 SPA_ERR_UNSUPPORTED_SHAPE = 2
@@ -102,6 +104,9 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        if L.spa_abi_version() != ABI_VERSION:
+            raise ImportError(f"{lib_path} has ABI version {L.spa_abi_version()}, these bindings expect "
+                              f"{ABI_VERSION}; rebuild it")
         _LIB = L
     return _LIB
 
