@@ -50,6 +50,11 @@ def lib() -> ctypes.CDLL:
         L.orc_prefill_unit.argtypes = [_p, _p, _int, _int, _int, _int, _p, _p, _p, _i64, _i64, _dbl,
                                        _i64, _i64, _dbl, _int, _p, _p, _p]
         L.orc_prefill_unit.restype = _i64
+        L.orc_rla_state.argtypes = [_p, _p, _int, _i64, _i64, _p, _p]
+        L.orc_rla_direct.argtypes = [_p, _int, _p, _p, _i64, _int, _p, _i64, _int, _p]
+        L.orc_rla_subtract.argtypes = [_p, _int, _p, _p, _i64, _int, _p, _i64, _int, _p, _p, _p]
+        L.orc_rms_norm.argtypes = [_p, _int, _p, _dbl, _p]
+        assert L.orc_abi_version() == 2, "stale oracle library; rebuild it"
         _LIB = L
     return _LIB
 
@@ -135,6 +140,48 @@ def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarra
     return out, lse
 
 
+def rla_state(K: np.ndarray, V: np.ndarray, n0: int = 0, n1: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """RLA state of rows [n0, n1) of one (batch, kv head) ("SPLA", section 2.2):
+    S [d, d] = sum_n exp(k_n) v_n^T and z [d] = sum_n exp(k_n), float64."""
+    K = _c(K, np.uint16); V = _c(V, np.uint16)
+    d = K.shape[1]
+    n1 = K.shape[0] if n1 is None else n1
+    S = np.empty((d, d)); z = np.empty(d)
+    lib().orc_rla_state(_ptr(K), _ptr(V), d, n0, n1, _ptr(S), _ptr(z))
+    return S, z
+
+
+def rla_direct(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, unit_tokens: int = 1) -> np.ndarray:
+    """RLA output by definition ("SPLA", section 2.2): normalised linear attention with
+    phi = exp over the rows the support leaves out.  q [G, d] -> [G, d] float64."""
+    q = _c(q, np.uint16); K = _c(K, np.uint16); V = _c(V, np.uint16); idx = _c(idx, np.int32)
+    G, d = q.shape
+    o = np.empty((G, d))
+    lib().orc_rla_direct(_ptr(q), G, _ptr(K), _ptr(V), K.shape[0], d, _ptr(idx), idx.size, unit_tokens, _ptr(o))
+    return o
+
+
+def rla_subtract(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, S: np.ndarray, z: np.ndarray,
+                 unit_tokens: int = 1) -> np.ndarray:
+    """RLA output in the IO form ("SPLA", section 2.2): global linear attention from the
+    state (S, z) minus linear attention over the gathered support rows."""
+    q = _c(q, np.uint16); K = _c(K, np.uint16); V = _c(V, np.uint16); idx = _c(idx, np.int32)
+    S = _c(S, np.float64); z = _c(z, np.float64)
+    G, d = q.shape
+    o = np.empty((G, d))
+    lib().orc_rla_subtract(_ptr(q), G, _ptr(K), _ptr(V), K.shape[0], d, _ptr(idx), idx.size, unit_tokens,
+                           _ptr(S), _ptr(z), _ptr(o))
+    return o
+
+
+def rms_norm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm with scale gamma ("SPLA", section 2.3) of x [d] -> [d] float64."""
+    x = _c(x, np.float64); gamma = _c(gamma, np.float64)
+    y = np.empty_like(x)
+    lib().orc_rms_norm(_ptr(x), x.size, _ptr(gamma), float(eps), _ptr(y))
+    return y
+
+
 def dense_probs(q: np.ndarray, K: np.ndarray, sm_scale: float) -> np.ndarray:
     q = _c(q, np.uint16); K = _c(K, np.uint16)
     P = np.empty(K.shape[0])
@@ -183,7 +230,8 @@ def local_support(M: int, sink: int, window: int) -> np.ndarray:
 
 
 def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.ndarray, np.ndarray]] = None,
-                with_output: bool = True, local: bool = False) -> Dict[str, object]:
+                with_output: bool = True, local: bool = False, rla: Optional[Dict[str, object]] = None
+                ) -> Dict[str, object]:
     """The sparse decode path of one unit: scores -> support -> attention.
 
     Returns scores (float64, as computed), the ranked scores (binary32-rounded; for
@@ -191,6 +239,11 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
     [heads, d] and lse [heads] of the query heads sharing the support.  A local unit
     (head-wise routing, RTPurbo Methodology 1) is not scored: its support is the sink and
     the window, and it has no index mass.
+
+    rla = {"gamma": [Hq, d], "eps": float} adds the residual linear attention ("SPLA",
+    sections 2.2-2.3): out = exact sparse attention + RMSNorm_gamma(RLA over the rows the
+    support leaves out); "out_exact" and "o_rla" keep the two parts.  gamma and eps are
+    taken as the CUDA path receives them (binary32).
     """
     b, h = decode_units(cfg)[u]
     G = cfg.G
@@ -207,6 +260,7 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
                                         cfg.block)
             res["out"] = out
             res["lse"] = lse
+            _add_rla(cfg, x, res, heads, rla)
         return res
     if cfg.score == "lowrank":
         s = lowrank_scores(x["q_idx"][b, heads], x["Kidx"][b, g], cfg.collapse == "group", f32(cfg.score_scale))
@@ -232,19 +286,37 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
                                     cfg.block)
         res["out"] = out
         res["lse"] = lse
+        _add_rla(cfg, x, res, heads, rla)
     return res
 
 
+def _add_rla(cfg, x: Dict[str, np.ndarray], res: Dict[str, object], heads: slice,
+             rla: Optional[Dict[str, object]]) -> None:
+    """out += RMSNorm_gamma(RLA over the rows outside the support), per query head."""
+    if rla is None:
+        return
+    b, g = res["b"], res["g"]
+    o = rla_direct(x["q"][b, heads], x["K"][b, g], x["V"][b, g], res["idx"], cfg.block)
+    gamma = np.asarray(rla["gamma"], np.float32).astype(np.float64)[heads]
+    y = np.stack([rms_norm(o[i], gamma[i], f32(rla["eps"])) for i in range(o.shape[0])])
+    res["out_exact"] = res["out"]
+    res["o_rla"] = o
+    res["out"] = res["out"] + y
+
+
 def decode(cfg, x: Dict[str, np.ndarray], units: Optional[Sequence[int]] = None, threads: int = 1,
-           with_output: bool = True, local: Optional[Sequence[bool]] = None) -> List[Dict[str, object]]:
+           with_output: bool = True, local: Optional[Sequence[bool]] = None,
+           rla: Optional[Dict[str, object]] = None) -> List[Dict[str, object]]:
     """decode_unit over several units, optionally on a thread pool (the C calls release the GIL);
-    local[u] marks the local units of a head-wise routing."""
+    local[u] marks the local units of a head-wise routing; rla adds the residual linear
+    attention (see decode_unit)."""
     todo = list(range(cfg.U)) if units is None else list(units)
     loc = (lambda u: bool(local[u])) if local is not None else (lambda u: False)
+    one = lambda u: decode_unit(cfg, x, u, with_output=with_output, local=loc(u), rla=rla)
     if threads <= 1:
-        return [decode_unit(cfg, x, u, with_output=with_output, local=loc(u)) for u in todo]
+        return [one(u) for u in todo]
     with ThreadPoolExecutor(threads) as ex:
-        return list(ex.map(lambda u: decode_unit(cfg, x, u, with_output=with_output, local=loc(u)), todo))
+        return list(ex.map(one, todo))
 
 
 def captured_mass(cfg, x: Dict[str, np.ndarray], u: int, idx: np.ndarray) -> float:

@@ -23,12 +23,20 @@
 //            channel per GQA group.
 //   [SPLA-2.1] "SPLA", section 2.1: block score exp(q^T kbar)(1 + 1/2 q^T Cov(k) q)
 //            with Cov(k) replaced by its diagonal.
+//   [SPLA-2.2] "SPLA", section 2.2: residual linear attention (RLA) over the blocks the
+//            selection left out, with the parameter-free feature map phi(x) = exp(x); its
+//            IO form subtracts linear attention over the selected rows from linear
+//            attention over all rows, so the left-out rows are never read.
+//   [SPLA-2.3] same page, section 2.3: the output is the exact sparse attention plus the
+//            RLA output passed through an RMSNorm whose scale is the only new parameter.
 //
 // Parity pins (tests/test_oracle.py): dense attention and masked attention against
 // torch's fp64 scaled_dot_product_attention, top-k against numpy's lexsort, top-p
 // against brute force over all subsets, block statistics against numpy mean/var,
 // the Taylor score's zero-variance identity and fourth-order agreement on
-// axis-symmetric blocks, and the prefill path against dense causal attention.
+// axis-symmetric blocks, the prefill path against dense causal attention, and the
+// residual linear attention's subtraction form against its direct definition, its
+// closed forms (zero query, one left-out row) and brute-force Python loops.
 
 #include <algorithm>
 #include <cmath>
@@ -76,7 +84,7 @@ int64_t emit_ascending(const std::vector<char>& keep, int32_t* idx) {
 
 extern "C" {
 
-int orc_abi_version() { return 1; }
+int orc_abi_version() { return 2; }
 
 // a1 -- per-block mean and diagonal (population) variance of K [SPLA-2.1].
 // K: [N, d] bf16 of one (batch, kv head); only the nb = N / block full blocks count.
@@ -323,6 +331,100 @@ int64_t orc_prefill_unit(const uint16_t* qblk, const uint16_t* qidx_blk, int bq,
                                  out + (static_cast<int64_t>(i) * G + h) * d, nullptr);
     }
     return cnt;
+}
+
+// ---------------------------------------------------------------- residual linear attention
+// Rows of a support (selection units idx[0..cnt) of unit_tokens rows each), kept in
+// [0, N), in the order they are gathered.
+static std::vector<int64_t> support_rows(const int32_t* idx, int64_t cnt, int unit_tokens, int64_t N) {
+    std::vector<int64_t> rows;
+    for (int64_t i = 0; i < cnt; ++i)
+        for (int t = 0; t < unit_tokens; ++t) {
+            const int64_t row = static_cast<int64_t>(idx[i]) * unit_tokens + t;
+            if (row >= 0 && row < N) rows.push_back(row);
+        }
+    return rows;
+}
+
+// Linear-attention weight of row n for query q [SPLA-2.2]: phi(q) . phi(k_n) with phi = exp
+// applied to every component.
+static double rla_weight(const uint16_t* q, const uint16_t* K, int64_t n, int d) {
+    double w = 0.0;
+    for (int i = 0; i < d; ++i) w += std::exp(widen_bf16(q[i])) * std::exp(widen_bf16(K[n * d + i]));
+    return w;
+}
+
+// RLA state of rows [n0, n1) [SPLA-2.2]: S[i][j] = sum_n exp(k_n[i]) v_n[j], z[i] = sum_n exp(k_n[i]).
+void orc_rla_state(const uint16_t* K, const uint16_t* V, int d, int64_t n0, int64_t n1, double* S, double* z) {
+    std::fill(S, S + static_cast<int64_t>(d) * d, 0.0);
+    std::fill(z, z + d, 0.0);
+    for (int64_t n = n0; n < n1; ++n)
+        for (int i = 0; i < d; ++i) {
+            const double f = std::exp(widen_bf16(K[n * d + i]));
+            z[i] += f;
+            for (int j = 0; j < d; ++j) S[static_cast<int64_t>(i) * d + j] += f * widen_bf16(V[n * d + j]);
+        }
+}
+
+// RLA output by its definition [SPLA-2.2]: normalised linear attention of every query head
+// over the rows of [0, N) that the support leaves out,
+//   o = sum_{n not in S} w_n v_n / sum_{n not in S} w_n,   w_n = phi(q) . phi(k_n);
+// o = 0 when the support covers every row.  q [G, d]; o [G, d].
+void orc_rla_direct(const uint16_t* q, int G, const uint16_t* K, const uint16_t* V, int64_t N, int d,
+                    const int32_t* idx, int64_t cnt, int unit_tokens, double* o) {
+    std::vector<char> in_support(static_cast<size_t>(N), 0);
+    for (int64_t row : support_rows(idx, cnt, unit_tokens, N)) in_support[static_cast<size_t>(row)] = 1;
+    for (int h = 0; h < G; ++h) {
+        double* oh = o + static_cast<int64_t>(h) * d;
+        std::fill(oh, oh + d, 0.0);
+        double den = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            if (in_support[static_cast<size_t>(n)]) continue;
+            const double w = rla_weight(q + static_cast<int64_t>(h) * d, K, n, d);
+            den += w;
+            for (int j = 0; j < d; ++j) oh[j] += w * widen_bf16(V[n * d + j]);
+        }
+        if (den > 0.0)
+            for (int j = 0; j < d; ++j) oh[j] /= den;
+    }
+}
+
+// RLA output in the pages' IO form [SPLA-2.2]: the global linear attention of the state
+// (S, z) over all rows minus the linear attention over the gathered support rows, taken for
+// numerator and normaliser alike: o = (phi(q)^T S - sum_sel w v) / (phi(q) . z - sum_sel w).
+// o = 0 when the support covers every row.  Equal to orc_rla_direct for a support without
+// repeated rows.
+void orc_rla_subtract(const uint16_t* q, int G, const uint16_t* K, const uint16_t* V, int64_t N, int d,
+                      const int32_t* idx, int64_t cnt, int unit_tokens, const double* S, const double* z,
+                      double* o) {
+    const std::vector<int64_t> rows = support_rows(idx, cnt, unit_tokens, N);
+    for (int h = 0; h < G; ++h) {
+        const uint16_t* qh = q + static_cast<int64_t>(h) * d;
+        double* oh = o + static_cast<int64_t>(h) * d;
+        std::vector<double> num(d, 0.0);
+        double den = 0.0;
+        for (int i = 0; i < d; ++i) {
+            const double f = std::exp(widen_bf16(qh[i]));
+            den += f * z[i];
+            for (int j = 0; j < d; ++j) num[j] += f * S[static_cast<int64_t>(i) * d + j];
+        }
+        for (int64_t n : rows) {
+            const double w = rla_weight(qh, K, n, d);
+            den -= w;
+            for (int j = 0; j < d; ++j) num[j] -= w * widen_bf16(V[n * d + j]);
+        }
+        const bool covered = static_cast<int64_t>(rows.size()) >= N;
+        for (int j = 0; j < d; ++j) oh[j] = covered ? 0.0 : num[j] / den;
+    }
+}
+
+// RMSNorm with scale [SPLA-2.3]: y = gamma * x / sqrt(mean(x^2) + eps), x [d].
+void orc_rms_norm(const double* x, int d, const double* gamma, double eps, double* y) {
+    double ms = 0.0;
+    for (int j = 0; j < d; ++j) ms += x[j] * x[j];
+    ms /= d;
+    const double inv = 1.0 / std::sqrt(ms + eps);
+    for (int j = 0; j < d; ++j) y[j] = gamma[j] * x[j] * inv;
 }
 
 }  // extern "C"
