@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--local-fraction", type=float, default=0.0,
                     help="head-wise routing: this fraction of every sequence's units is local (sink + window)")
+    ap.add_argument("--rla", action="store_true",
+                    help="add the residual linear attention over the rows outside each support (SPLA)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
     if a.steps is None:
@@ -141,7 +143,14 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline(cfg, x, seconds: float, local=None):
+def rla_params(cfg):
+    """RMSNorm scale and epsilon of the residual linear attention (a trained parameter in the
+    method; fixed seeded values here)."""
+    gamma = np.random.default_rng(11).uniform(0.5, 1.5, (cfg.Hq, cfg.d)).astype(np.float32)
+    return {"gamma": gamma, "eps": 1e-6}
+
+
+def cpu_baseline(cfg, x, seconds: float, local=None, rla=None):
     """The fp64 oracle's sparse path (scores -> selection -> attention), as it stands, on the
     host cores: units of the same workload cycled until the time budget is spent."""
     import oracle
@@ -151,7 +160,7 @@ def cpu_baseline(cfg, x, seconds: float, local=None):
     done = 0
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < seconds:      # whole rounds over all units
-        oracle.decode(cfg, x, units=units, threads=cores, local=local)
+        oracle.decode(cfg, x, units=units, threads=cores, local=local, rla=rla)
         done += len(units)
     dt = time.perf_counter() - t0
     return {"value": done * cfg.heads_per_unit / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -169,19 +178,22 @@ def run_reference(a):
 
     x = decode_inputs(cfg)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    rla = rla_params(cfg) if a.rla else None
     # one step = one unit (a kv head of one sequence: its index scores over all N keys,
     # the top-p cut and exact attention for its query heads), cycling over the units
     for i in range(a.warmup):
-        oracle.decode_unit(cfg, x, i % cfg.U)
+        oracle.decode_unit(cfg, x, i % cfg.U, rla=rla)
     t0 = time.perf_counter()
     for i in range(a.steps):
-        oracle.decode_unit(cfg, x, i % cfg.U)
+        oracle.decode_unit(cfg, x, i % cfg.U, rla=rla)
     dt = time.perf_counter() - t0
     value = a.steps * cfg.heads_per_unit / dt
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": workload_desc(cfg), "sample": "one unit per step, cycling over the units"},
+            "config": {"workload": workload_desc(cfg) + (" + SPLA residual linear attention over the rows "
+                                                         "outside each support" if rla is not None else ""),
+                       "sample": "one unit per step, cycling over the units"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{a.steps} units of {cfg.name}, one per step, single thread "
                                        f"({cores} cores available)"},
@@ -238,6 +250,12 @@ def run_spa(a):
     local_np = np.array([int(u % units_per_seq < n_local) for u in range(cfg.U)], np.uint8)
     if n_local:
         kw["local_units"] = torch.from_numpy(local_np).cuda()
+    # residual linear attention: the state of all N rows is built once, like a prefill would
+    # (a decoder then appends one row per token); gamma and eps are fixed seeded values
+    rla = rla_params(cfg) if a.rla else None
+    if rla is not None:
+        S, z = spa.rla_state(dK, dV)
+        kw.update(rla_state=S, rla_z=z, rla_gamma=torch.from_numpy(rla["gamma"]).cuda(), rla_eps=rla["eps"])
     plan = spa.decode(**kw)
     wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
@@ -317,6 +335,8 @@ def run_spa(a):
         if cfg.collapse == "group":      # a local unit's block statistics are not read
             score_bytes -= int(local_np.sum()) * 2 * M * d * 4
     attend_bytes = rows * KV_ROW_BYTES(d) + 2 * cfg.B * cfg.Hq * d * 2
+    if rla is not None:      # the state (S, z) of every kv head and gamma, read once
+        attend_bytes += cfg.B * cfg.Hkv * (d * d + d) * 4 + cfg.Hq * d * 4
     step_bytes = score_bytes + attend_bytes
     peak, peak_kind = peaks()
     mean_ms = {k: float(v.mean()) for k, v in k_ms.items()}
@@ -325,7 +345,7 @@ def run_spa(a):
     achieved = kbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": peak_kind,
-                "traffic": recorded_traffic(dom, cfg.name),
+                "traffic": recorded_traffic(dom, cfg.name + ("+rla" if rla is not None else "")),
                 "step_achieved": step_bytes / (float(step_ms.mean()) * 1e-3) / 1e9,
                 "step_frac": step_bytes / (float(step_ms.mean()) * 1e-3) / 1e9 / peak}
     roofline["algorithmic_bytes_per_launch"] = kbytes[dom]
@@ -371,11 +391,13 @@ def run_spa(a):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": float(step_ms.mean()), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "seq_len": cfg.N,
+            "config": {"workload": workload_desc(cfg) + (" + SPLA residual linear attention over the rows outside "
+                                                         "each support" if rla is not None else ""),
+                       "global_batch": cfg.B * world, "seq_len": cfg.N,
                        "parallelism": f"dp{world} (independent sequence shards, no collective on the data path)",
                        "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
                        "support_rows_per_step": rows, "sparsity": round(float(sparsity), 4),
-                       "local_units": int(local_np.sum()),
+                       "local_units": int(local_np.sum()), "rla": rla is not None,
                        "algorithmic_bytes_per_step": step_bytes},
             "roofline": roofline,
             "kernels_ms": {k: round(v, 5) for k, v in mean_ms.items()},
@@ -388,7 +410,8 @@ def run_spa(a):
             "wall_s_timed_region": w1 - w0,
         }
         if not a.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(cfg, x, a.cpu_seconds, local=local_np if n_local else None)
+            line["cpu_baseline"] = cpu_baseline(cfg, x, a.cpu_seconds, local=local_np if n_local else None,
+                                                rla=rla)
         elif world > 1:
             line["cpu_baseline"] = None
     if world > 1:

@@ -75,7 +75,7 @@ const char* spa_status_string(int status);
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
 const char* spa_last_cuda_error(void);
 
-/* ABI version of this header: 2 (spa_decode_args gained local_units). */
+/* ABI version of this header: 3 (spa_decode_args gained local_units in 2, the RLA fields in 3). */
 int spa_abi_version(void);
 
 /* ------------------------------------------------------------------------------------
@@ -236,6 +236,25 @@ typedef struct spa_decode_args {
      * [M - window, M) only; its index_mass is 0.  NULL: every unit is a retrieval unit.
      * [U] bytes, device memory, read-only. */
     const uint8_t* local_units;
+    /* Residual linear attention ("SPLA", sections 2.2-2.3): the rows a support leaves out
+     * are condensed by linear attention with the feature map phi(x) = exp(x) (every
+     * component), and the output becomes
+     *   out = exact sparse attention + gamma * o_rla / sqrt(mean_j o_rla[j]^2 + eps),
+     *   o_rla = (phi(q)^T S - sum_sel w v) / (phi(q) . z - sum_sel w),  w = phi(q) . phi(k),
+     * where sum_sel runs over the gathered rows (the same tiles the exact attention reads;
+     * the left-out rows are never read) and (S, z) is the state of all N rows
+     * (spa_rla_state).  o_rla = 0 when the support covers every row.  lse stays the exact
+     * attention's.  The subtraction assumes supports without repeated rows and loses
+     * precision when the left-out rows carry a tiny share of sum w; binary32 overflows once
+     * q[i] + k[i] exceeds about 88 for some component i.
+     * rla_state NULL: off (the fields below are not read).  Device memory, fp32, read-only:
+     *   rla_state [B, Hkv, d, d]: S[i][j] = sum_n exp(k_n[i]) v_n[j] over rows [0, N);
+     *   rla_z     [B, Hkv, d]:    z[i]    = sum_n exp(k_n[i]);
+     *   rla_gamma [Hq, d]:        RMSNorm scale of the RLA output, per query head. */
+    const float* rla_state;
+    const float* rla_z;
+    const float* rla_gamma;
+    float rla_eps;           /* RMSNorm epsilon, >= 0 */
 } spa_decode_args;
 
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream);
@@ -246,6 +265,21 @@ size_t spa_decode_workspace_bytes(const spa_decode_args* a);
  * events[3] after the attention kernel, so a caller can time each kernel inside a real step. */
 spa_status spa_decode_timed(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
                             void* const* events);
+
+/* ------------------------------------------------------------------------------------
+ * RLA state ("SPLA", section 2.2): adds rows [n0, n1) of every (batch, kv head) of the
+ * cache into the linear-attention state with the feature map phi(x) = exp(x):
+ *   S[bg][i][j] += sum_{n0 <= n < n1} exp(K[bg][n][i]) * V[bg][n][j],
+ *   z[bg][i]    += sum_{n0 <= n < n1} exp(K[bg][n][i]).
+ * Zero S and z and call it with [0, N) after a prefill, then with [N, N + 1) for each
+ * appended token.  K, V [B, Hkv, N, d] bf16 (16-byte aligned); S [B, Hkv, d, d] and
+ * z [B, Hkv, d] fp32, device memory, read and written.  Runs on tensor cores with phi(k)
+ * carried as two bf16 terms (about 16 significant bits) and fp32 accumulation; the
+ * order of summation is fixed, so equal calls give equal bits.  d in {64, 128};
+ * 0 <= n0 <= n1 <= N; B * Hkv <= 65535.  n0 == n1 or B == 0 does nothing.
+ */
+spa_status spa_rla_state(const uint16_t* K, const uint16_t* V, int B, int Hkv, int N, int d, int n0, int n1,
+                         float* S, float* z, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * a9. Selection-block-shared sparse prefill ("Oracle-Guided Sparse Prefill" 2.1 with

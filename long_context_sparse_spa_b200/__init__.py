@@ -201,10 +201,15 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
            bmean: Optional[torch.Tensor] = None, bvar: Optional[torch.Tensor] = None, block: int = 1,
            score_scale: float, sm_scale: float, topk: int = 0, topp: float = 0.0, sink: int = 0,
            window: int = 0, cap: Optional[int] = None, want_f32: bool = True, want_lse: bool = True,
-           local_units: Optional[torch.Tensor] = None, run: bool = True) -> DecodePlan:
+           local_units: Optional[torch.Tensor] = None, rla_state: Optional[torch.Tensor] = None,
+           rla_z: Optional[torch.Tensor] = None, rla_gamma: Optional[torch.Tensor] = None,
+           rla_eps: float = 1e-6, run: bool = True) -> DecodePlan:
     """Build (and by default run) a fused decode step; see spa_decode in include/spa.h.
     local_units: optional uint8 [U] on the device, nonzero for the units that head-wise routing
-    makes local (support = sink + window, not scored)."""
+    makes local (support = sink + window, not scored).
+    rla_state / rla_z / rla_gamma: optional fp32 [B, Hkv, d, d] / [B, Hkv, d] / [Hq, d] that
+    add the residual linear attention over the rows outside each support (state from
+    rla_state())."""
     for t, n in ((q, "q"), (K, "K"), (V, "V")):
         _need(t, torch.bfloat16, n)
     B, Hq, d = q.shape
@@ -238,11 +243,44 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
         if local_units.numel() != U:
             raise ValueError(f"local_units must hold one flag per unit ({U})")
     a.local_units = _ptr(local_units)
+    if rla_state is not None:
+        for t, n, shape in ((rla_state, "rla_state", (B, Hkv, d, d)), (rla_z, "rla_z", (B, Hkv, d)),
+                            (rla_gamma, "rla_gamma", (Hq, d))):
+            if t is None:
+                raise ValueError(f"{n} is required with rla_state")
+            _need(t, torch.float32, n)
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{n} must have shape {shape}, got {tuple(t.shape)}")
+        a.rla_state, a.rla_z, a.rla_gamma, a.rla_eps = _ptr(rla_state), _ptr(rla_z), _ptr(rla_gamma), rla_eps
     ws = workspace(lib().spa_decode_workspace_bytes(ctypes.byref(a)), dev)
-    plan = DecodePlan(a, ws, idx, count, mass, out, out32, lse, (q, K, V, q_idx, Kidx, bmean, bvar, local_units))
+    plan = DecodePlan(a, ws, idx, count, mass, out, out32, lse,
+                      (q, K, V, q_idx, Kidx, bmean, bvar, local_units, rla_state, rla_z, rla_gamma))
     if run:
         plan.run()
     return plan
+
+
+# ----------------------------------------------------------------------------- RLA state
+def rla_state(K: torch.Tensor, V: torch.Tensor, S: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+              n0: int = 0, n1: Optional[int] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Add rows [n0, n1) of K, V [B, Hkv, N, d] bf16 into the residual-linear-attention state
+    S [B, Hkv, d, d], z [B, Hkv, d] (fp32, zero-filled when not given); see spa_rla_state
+    in include/spa.h.  Returns (S, z)."""
+    _need(K, torch.bfloat16, "K")
+    _need(V, torch.bfloat16, "V")
+    B, Hkv, N, d = K.shape
+    if tuple(V.shape) != (B, Hkv, N, d):
+        raise ValueError("K and V must have the same shape")
+    S = torch.zeros((B, Hkv, d, d), dtype=torch.float32, device=K.device) if S is None else S
+    z = torch.zeros((B, Hkv, d), dtype=torch.float32, device=K.device) if z is None else z
+    _need(S, torch.float32, "S")
+    _need(z, torch.float32, "z")
+    if tuple(S.shape) != (B, Hkv, d, d) or tuple(z.shape) != (B, Hkv, d):
+        raise ValueError("S must be [B, Hkv, d, d] and z [B, Hkv, d]")
+    n1 = N if n1 is None else n1
+    check(lib().spa_rla_state(_ptr(K), _ptr(V), B, Hkv, N, d, n0, n1, _ptr(S), _ptr(z), _stream(stream)),
+          "spa_rla_state")
+    return S, z
 
 
 # ----------------------------------------------------------------------------- a9 shared-support prefill

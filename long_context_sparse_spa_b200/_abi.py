@@ -7,7 +7,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(HERE, "libspa.so")
 
-ABI_VERSION = 2   # spa_abi_version() of the library these declarations describe
+ABI_VERSION = 3   # spa_abi_version() of the library these declarations describe
 
 SPA_OK = 0
 SPA_ERR_INVALID_ARG = 1
@@ -45,6 +45,7 @@ class SpaDecodeArgs(ctypes.Structure):
         ("index_mass", _p),
         ("out", _p), ("out_f32", _p), ("lse", _p),
         ("local_units", _p),
+        ("rla_state", _p), ("rla_z", _p), ("rla_gamma", _p), ("rla_eps", _f),
     ]
 
 
@@ -71,6 +72,7 @@ SIGNATURES = {
     "spa_select_topp": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p, _sz, _p]),
     "spa_select_workspace_bytes": (_sz, [_i, _i]),
     "spa_select_topp_static": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p]),
+    "spa_rla_state": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_sparse_attend": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "spa_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spa_decode": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p]),

@@ -73,7 +73,7 @@ const char* spa_status_string(int s) {
 
 const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
-int spa_abi_version(void) { return 2; }
+int spa_abi_version(void) { return 3; }
 
 spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean, float* var,
                            void* stream) {
@@ -272,6 +272,13 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     if (s != SPA_OK) return s;
     ap.unit_ctas = reinterpret_cast<int*>(attend_ws);
     ap.partials = reinterpret_cast<float*>(attend_ws + align_up(size_t(U) * 8, 256));
+    if (a->rla_state) {
+        if (!a->rla_z || !a->rla_gamma || !(a->rla_eps >= 0.f)) return SPA_ERR_INVALID_ARG;
+        ap.rla_S = a->rla_state;
+        ap.rla_z = a->rla_z;
+        ap.rla_gamma = a->rla_gamma;
+        ap.rla_eps = a->rla_eps;
+    }
 
     auto mark = [&](int i) -> spa_status {
         if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st));
@@ -308,6 +315,17 @@ size_t spa_prefill_workspace_bytes(const spa_prefill_args* a) {
     if (!a || a->bq <= 0 || a->Hkv <= 0 || a->T < 0 || a->N < 0) return 0;
     const int U = (a->T / a->bq) * a->Hkv;
     return kWsHeader + prefill_scratch_bytes(U, a->N);
+}
+
+spa_status spa_rla_state(const uint16_t* K, const uint16_t* V, int B, int Hkv, int N, int d, int n0, int n1,
+                         float* S, float* z, void* stream) {
+    if (B < 0 || Hkv <= 0 || N < 0 || n0 < 0 || n1 < n0 || n1 > N) return SPA_ERR_INVALID_ARG;
+    if (B == 0 || n0 == n1) return SPA_OK;
+    if (!K || !V || !S || !z) return SPA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(S) || !aligned16(z)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (size_t(B) * Hkv > 65535) return SPA_ERR_UNSUPPORTED_SHAPE;
+    return launch_rla_state(K, V, B * Hkv, N, d, n0, n1, S, z, static_cast<cudaStream_t>(stream));
 }
 
 spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {

@@ -29,6 +29,7 @@
 // and a second kernel, one CTA per (unit, head) with eight warps splitting the unit's
 // partials, merges them in a fixed order (log-sum-exp combine) and writes the output.
 #include "internal.cuh"
+#include "warp_mma.cuh"
 
 namespace spa {
 namespace {
@@ -42,48 +43,9 @@ constexpr int kWinTiles = 128;      // tiles whose row indices are staged in sha
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0));
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// transpose of an 8x8 b16 matrix held in mma fragment layout (one b16x2 per thread)
-__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-    return y;
-}
-// p ~= hi + lo with hi = bf16(p), lo = bf16(p - hi)
-__device__ __forceinline__ void split_bf16(float p0, float p1, uint32_t& hi, uint32_t& lo) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-    const float2 hf = __bfloat1622float2(h);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-    hi = *reinterpret_cast<const uint32_t*>(&h);
-    lo = *reinterpret_cast<const uint32_t*>(&l);
-}
-
 struct UnitGeom {
     int b, h0, nh;        // batch, first query head, query heads served
+    int bh;               // batch * Hkv + kv head
     size_t kv;            // row offset of the unit's kv head in K/V
     int rows;             // gathered rows R_u
 };
@@ -95,11 +57,13 @@ __device__ __forceinline__ UnitGeom unit_geom(const AttendParams& p, int u, int 
         g.b = u / p.Hkv;
         const int kvh = u - g.b * p.Hkv;
         g.h0 = kvh * G;
-        g.kv = (size_t(g.b) * p.Hkv + kvh) * size_t(p.N);
+        g.bh = g.b * p.Hkv + kvh;
+        g.kv = size_t(g.bh) * size_t(p.N);
     } else {
         g.b = u / p.Hq;
         g.h0 = u - g.b * p.Hq;
-        g.kv = (size_t(g.b) * p.Hkv + g.h0 / G) * size_t(p.N);
+        g.bh = g.b * p.Hkv + g.h0 / G;
+        g.kv = size_t(g.bh) * size_t(p.N);
     }
     g.nh = nh;
     int c = p.count[u];
@@ -123,7 +87,11 @@ __device__ __forceinline__ int tile_owner(long long x, long long TT, int G) {
     return int(((x + 1) * G - 1) / TT);
 }
 
-template <int D, int NH8>
+// RLA: also accumulate, per head, the linear attention of the gathered rows with phi = exp
+// ("SPLA", section 2.2): W^T = phi(K) phi(Q)^T on the same K fragments as S^T, and
+// Olin^T += V^T W^T on the same V fragments as O^T; every unit then leaves partials for the
+// combine kernel, which forms the residual term.
+template <int D, int NH8, bool RLA>
 __global__ void __launch_bounds__(kAtThreads, 2)
 attend_kernel(AttendParams p, int U, int nh) {
     pdl_enter();
@@ -174,7 +142,7 @@ attend_kernel(AttendParams p, int U, int nh) {
     const int G = int(TT < (long long)gridDim.x ? TT : (long long)gridDim.x);
 
     // ---- empty supports: out = 0, lse = -inf
-    for (int u = cta; u < U; u += gridDim.x) {
+    for (int u = cta; !RLA && u < U; u += gridDim.x) {   // (with RLA the combine kernel writes them)
         if (s_prefix[u + 1] != s_prefix[u]) continue;
         const UnitGeom ug = unit_geom(p, u, nh);
         for (int i = tid; i < nh * D; i += kAtThreads) {
@@ -193,7 +161,7 @@ attend_kernel(AttendParams p, int U, int nh) {
             if (s_prefix[v + 1] > s_prefix[v]) {
                 lo = tile_owner(s_prefix[v], TT, G);
                 hi = tile_owner(s_prefix[v + 1] - 1, TT, G);
-                if (lo == hi) lo = hi = -1;
+                if (lo == hi && !RLA) lo = hi = -1;
             }
             p.unit_ctas[2 * v] = lo;
             p.unit_ctas[2 * v + 1] = hi;
@@ -241,6 +209,22 @@ attend_kernel(AttendParams p, int U, int nh) {
             }
         }
 
+        // RLA: phi(Q)^T as B operand, exp of the same elements as qb, hi + lo bf16; zero for
+        // absent heads
+        uint32_t qfh[RLA ? TL::KSTEPS : 1][NH8][2], qfl[RLA ? TL::KSTEPS : 1][NH8][2];
+        if constexpr (RLA) {
+#pragma unroll
+            for (int nt = 0; nt < NH8; ++nt)
+#pragma unroll
+                for (int kk = 0; kk < TL::KSTEPS; ++kk)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool v = nt * 8 + gq < nh;
+                        const float2 f = bf16x2_to_float2(qb[kk][nt][e]);
+                        split_bf16(v ? expf(f.x) : 0.f, v ? expf(f.y) : 0.f, qfh[kk][nt][e], qfl[kk][nt][e]);
+                    }
+        }
+
         const int32_t* idx_u = p.idx + size_t(u) * p.cap;
         const int T = p.unit_tokens;
         auto issue = [&](long long row, int stage) {
@@ -265,10 +249,16 @@ attend_kernel(AttendParams p, int U, int nh) {
         // online-softmax state of heads 8nt + 2cq + e (e = 0, 1); l is this thread's partial sum
         float m_r[NH8][2], l_r[NH8][2];
         float acc[TL::KSTEPS][NH8][4];      // O^T: d-tile x head tile, rows d = 16dt + gq (+8)
+        float lin[RLA ? TL::KSTEPS : 1][NH8][4], den_r[NH8][2];   // RLA: Olin^T and sum of weights
+        int nval = 0;                                             // RLA: rows gathered in [0, N)
 #pragma unroll
         for (int nt = 0; nt < NH8; ++nt) {
             m_r[nt][0] = m_r[nt][1] = -INFINITY;
             l_r[nt][0] = l_r[nt][1] = 0.f;
+            den_r[nt][0] = den_r[nt][1] = 0.f;
+#pragma unroll
+            for (int dt = 0; dt < (RLA ? TL::KSTEPS : 1); ++dt)
+                lin[dt][nt][0] = lin[dt][nt][1] = lin[dt][nt][2] = lin[dt][nt][3] = 0.f;
 #pragma unroll
             for (int dt = 0; dt < TL::KSTEPS; ++dt) acc[dt][nt][0] = acc[dt][nt][1] = acc[dt][nt][2] = acc[dt][nt][3] = 0.f;
         }
@@ -311,9 +301,11 @@ attend_kernel(AttendParams p, int U, int nh) {
             const uint32_t vm = s_vmask[warp][stage];
 
             // S^T = K Q^T: 16 keys x 8 heads per head tile
-            float s[NH8][4];
+            float s[NH8][4], w[RLA ? NH8 : 1][4];
 #pragma unroll
             for (int nt = 0; nt < NH8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < (RLA ? NH8 : 1); ++nt) w[nt][0] = w[nt][1] = w[nt][2] = w[nt][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < TL::KSTEPS; ++kk) {
                 const int mat = lane >> 3;
@@ -323,9 +315,42 @@ attend_kernel(AttendParams p, int U, int nh) {
                 ldsm_x4(kbase + (rr * TL::CPR + (c ^ (rr & 7))) * 16, a[0], a[1], a[2], a[3]);
 #pragma unroll
                 for (int nt = 0; nt < NH8; ++nt) mma16816(s[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+                if constexpr (RLA) {
+                    // W^T += phi(K) phi(Q)^T, both factors as hi + lo (the lo * lo term dropped)
+                    uint32_t fh[4], fl[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 kf = bf16x2_to_float2(a[i]);
+                        split_bf16(expf(kf.x), expf(kf.y), fh[i], fl[i]);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NH8; ++nt) {
+                        mma16816(w[nt], fh, qfh[kk][nt][0], qfh[kk][nt][1]);
+                        mma16816(w[nt], fl, qfh[kk][nt][0], qfh[kk][nt][1]);
+                        mma16816(w[nt], fh, qfl[kk][nt][0], qfl[kk][nt][1]);
+                    }
+                }
             }
             // mask, scale; per-head max over the 16 keys (keys gq, gq + 8 here; xor over gq)
             const bool kv0 = (vm >> gq) & 1u, kv1 = (vm >> (gq + 8)) & 1u;
+            // RLA: masked weights (zero-filled rows would weigh phi(q) . 1), their sums, and
+            // W^T moved into the B-operand layout like P^T
+            uint32_t wh[RLA ? NH8 : 1][2], wl[RLA ? NH8 : 1][2];
+            if constexpr (RLA) {
+                nval += __popc(vm);
+#pragma unroll
+                for (int nt = 0; nt < NH8; ++nt) {
+                    const float w00 = kv0 ? w[nt][0] : 0.f, w01 = kv0 ? w[nt][1] : 0.f;
+                    const float w10 = kv1 ? w[nt][2] : 0.f, w11 = kv1 ? w[nt][3] : 0.f;
+                    den_r[nt][0] += w00 + w10;
+                    den_r[nt][1] += w01 + w11;
+                    uint32_t h0, l0, h1, l1;
+                    split_bf16(w00, w01, h0, l0);
+                    split_bf16(w10, w11, h1, l1);
+                    wh[nt][0] = movm_t(h0); wh[nt][1] = movm_t(h1);
+                    wl[nt][0] = movm_t(l0); wl[nt][1] = movm_t(l1);
+                }
+            }
             uint32_t bh[NH8][2], bl[NH8][2];
 #pragma unroll
             for (int nt = 0; nt < NH8; ++nt) {
@@ -370,6 +395,10 @@ attend_kernel(AttendParams p, int U, int nh) {
                 for (int nt = 0; nt < NH8; ++nt) {
                     mma16816(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
                     mma16816(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                    if constexpr (RLA) {
+                        mma16816(lin[dt][nt], a, wh[nt][0], wh[nt][1]);
+                        mma16816(lin[dt][nt], a, wl[nt][0], wl[nt][1]);
+                    }
                 }
             }
             __syncwarp();   // this stage may be refilled after the next wait
@@ -383,6 +412,11 @@ attend_kernel(AttendParams p, int U, int nh) {
                 l_r[nt][e] += __shfl_xor_sync(0xffffffffu, l_r[nt][e], 4);
                 l_r[nt][e] += __shfl_xor_sync(0xffffffffu, l_r[nt][e], 8);
                 l_r[nt][e] += __shfl_xor_sync(0xffffffffu, l_r[nt][e], 16);
+                if constexpr (RLA) {
+                    den_r[nt][e] += __shfl_xor_sync(0xffffffffu, den_r[nt][e], 4);
+                    den_r[nt][e] += __shfl_xor_sync(0xffffffffu, den_r[nt][e], 8);
+                    den_r[nt][e] += __shfl_xor_sync(0xffffffffu, den_r[nt][e], 16);
+                }
             }
 
         // ---- merge the warps: each warp parks (m, l, o) in its own ring
@@ -407,8 +441,25 @@ attend_kernel(AttendParams p, int U, int nh) {
             wbuf[8 + lane] = -INFINITY;
             wbuf[24 + lane] = 0.f;
         }
+        // RLA: den[16] at kDen, the warp's row count at kNval, Olin[16][D] at kLin
+        constexpr int kDen = 32 + 16 * D, kNval = kDen + 16, kLin = kDen + 32;
+        if constexpr (RLA) {
+#pragma unroll
+            for (int nt = 0; nt < NH8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int hd = nt * 8 + 2 * cq + e;
+                    if (gq == 0) wbuf[kDen + hd] = den_r[nt][e];
+#pragma unroll
+                    for (int dt = 0; dt < TL::KSTEPS; ++dt) {
+                        wbuf[kLin + hd * D + dt * 16 + gq] = lin[dt][nt][e];
+                        wbuf[kLin + hd * D + dt * 16 + gq + 8] = lin[dt][nt][2 + e];
+                    }
+                }
+            if (lane == 0) wbuf[kNval] = float(nval);
+        }
         __syncthreads();
-        const bool whole = a == 0 && bnd == tiles_u;
+        const bool whole = !RLA && a == 0 && bnd == tiles_u;
         const int slot = u + cta;
         const size_t n_slots = size_t(U) + gridDim.x;
         for (int i = tid; i < nh * D; i += kAtThreads) {
@@ -441,6 +492,22 @@ attend_kernel(AttendParams p, int U, int nh) {
                     part[D] = M;
                     part[D + 1] = L;
                 }
+                if constexpr (RLA) {     // (Olin, sum of weights, rows) of this CTA's share
+                    float* rp = p.partials + (size_t(nh) * n_slots + size_t(row) * n_slots + slot) * (D + 2);
+                    float Lin = 0.f, Den = 0.f, Nv = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kAtWarps; ++w) {
+                        const float* wb = reinterpret_cast<const float*>(ring + size_t(w) * kStages * TL::BYTES);
+                        Lin += wb[kLin + row * D + col];
+                        Den += wb[kDen + row];
+                        Nv += wb[kNval];
+                    }
+                    rp[col] = Lin;
+                    if (col == 0) {
+                        rp[D] = Den;
+                        rp[D + 1] = Nv;
+                    }
+                }
             }
         }
         __syncthreads();   // rings are reused by the next segment
@@ -455,7 +522,13 @@ attend_kernel(AttendParams p, int U, int nh) {
 // maximum M with a fixed assignment of records to thread groups and a fixed-order sum.
 constexpr int kCombRecs = 48;    // records staged per chunk
 
-template <int D>
+//
+// RLA: every unit, empty ones included, is finished here.  With the unit's sums of Olin,
+// weights and rows over its CTAs, the residual linear attention of head h is
+//   o_rla = (phi(q)^T S - Olin) / (phi(q) . z - sum w),   0 when the rows cover the cache,
+// and the output is the exact attention plus gamma * o_rla / sqrt(mean(o_rla^2) + eps)
+// ("SPLA", sections 2.2-2.3).
+template <int D, bool RLA>
 __global__ void __launch_bounds__(256)
 combine_kernel(AttendParams p, int nh, int n_slots) {
     pdl_enter();
@@ -465,10 +538,11 @@ combine_kernel(AttendParams p, int nh, int n_slots) {
     constexpr int LOADS = (kCombRecs * REC / 2 + 255) / 256;
     const int u = blockIdx.x, row = blockIdx.y;
     const int c_lo = p.unit_ctas[2 * u], c_hi = p.unit_ctas[2 * u + 1];
-    if (c_lo < 0 || row >= nh) return;
+    if ((!RLA && c_lo < 0) || row >= nh) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n_c = c_hi - c_lo + 1;
-    const float* base = p.partials + (size_t(row) * n_slots + u + c_lo) * REC;
+    const int n_c = c_lo < 0 ? 0 : c_hi - c_lo + 1;
+    const size_t first = size_t(row) * n_slots + u + (c_lo < 0 ? 0 : c_lo);
+    const float* base = p.partials + first * REC;
 
     __shared__ __align__(16) float st[kCombRecs * REC];
     __shared__ float s_red[8];
@@ -516,16 +590,55 @@ combine_kernel(AttendParams p, int nh, int n_slots) {
     sO[grp][2 * pair] = O0;
     sO[grp][2 * pair + 1] = O1;
     __syncthreads();
-    if (tid >= D) return;
+    if (!RLA && tid >= D) return;
+    const bool act = tid < D;
     float Lt = 0.f, Ot = 0.f;
+    if (act) {
 #pragma unroll
-    for (int g = 0; g < GROUPS; ++g) {
-        Lt += sL[g];
-        Ot += sO[g][tid];
+        for (int g = 0; g < GROUPS; ++g) {
+            Lt += sL[g];
+            Ot += sO[g][tid];
+        }
     }
     const UnitGeom ug = unit_geom(p, u, nh);
     const size_t o = (size_t(ug.b) * p.Hq + ug.h0 + row) * D + tid;
-    const float val = Lt > 0.f ? Ot / Lt : 0.f;
+    float val = Lt > 0.f ? Ot / Lt : 0.f;
+    if constexpr (RLA) {
+        __shared__ float s_phq[D], s_sq[8];
+        const float* rbase = p.partials + (size_t(nh) * n_slots + first) * REC;
+        float lin = 0.f, den = 0.f, nval = 0.f;
+        if (act) {
+            for (int c = 0; c < n_c; ++c) {           // fixed order over the unit's CTAs
+                const float* rec = rbase + size_t(c) * REC;
+                lin += __ldcg(rec + tid);
+                den += __ldcg(rec + D);
+                nval += __ldcg(rec + D + 1);
+            }
+            s_phq[tid] = expf(__uint_as_float(uint32_t(p.q[o]) << 16));
+        }
+        __syncthreads();
+        float num_all = 0.f, den_all = 0.f;
+        if (act) {
+            const float* Sb = p.rla_S + size_t(ug.bh) * D * D;
+            const float* zb = p.rla_z + size_t(ug.bh) * D;
+#pragma unroll 8
+            for (int i = 0; i < D; ++i) {
+                num_all += s_phq[i] * __ldg(Sb + size_t(i) * D + tid);
+                den_all += s_phq[i] * __ldg(zb + i);
+            }
+        }
+        const float orla = act && nval < float(p.N) ? (num_all - lin) / (den_all - den) : 0.f;
+        float sq = orla * orla;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        if (lane == 0) s_sq[warp] = sq;
+        __syncthreads();
+        if (!act) return;
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) tot += s_sq[w];
+        val += __ldg(p.rla_gamma + size_t(ug.h0 + row) * D + tid) * orla / sqrtf(tot / D + p.rla_eps);
+    }
     const __nv_bfloat16 bv = __float2bfloat16_rn(val);
     p.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
     if (p.out_f32) p.out_f32[o] = val;
@@ -545,7 +658,8 @@ int attend_grid() { return device_info().num_sms * 2; }
 
 size_t attend_scratch_bytes(int U, int heads_per_unit, int d) {
     const size_t meta = align_up(size_t(U) * 8, 256);
-    const size_t partials = size_t(U + attend_grid()) * heads_per_unit * (d + 2) * 4;
+    // exact partials (o, m, l), then the RLA partials (Olin, sum of weights, rows)
+    const size_t partials = 2 * size_t(U + attend_grid()) * heads_per_unit * (d + 2) * 4;
     return meta + align_up(partials, 256);
 }
 
@@ -555,16 +669,18 @@ spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
     const int nh = p.collapse == SPA_COLLAPSE_GROUP_MEAN ? G : 1;
     if (U > kMaxUnits || nh > 16) return SPA_ERR_UNSUPPORTED_SHAPE;
     const int grid = attend_grid();
-#define SPA_AT_CASE(DD, H8)                                                                                    \
-    if (p.d == DD && (nh + 7) / 8 == H8) {                                                                    \
-        const size_t sm = attend_smem<DD>(U);                                                                 \
-        SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<DD, H8>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                          int(sm)));                                                          \
-        SPA_CUDA_TRY(launch_pdl(attend_kernel<DD, H8>, dim3(grid), dim3(kAtThreads), sm, st, p, U, nh));      \
-        SPA_CUDA_TRY(launch_pdl(combine_kernel<DD>, dim3(U, nh), dim3(256), 0, st, p, nh, U + grid));          \
-        return SPA_OK;                                                                                        \
+    const bool rla = p.rla_S != nullptr;
+#define SPA_AT_CASE(DD, H8, R)                                                                                   \
+    if (p.d == DD && (nh + 7) / 8 == H8 && rla == R) {                                                          \
+        const size_t sm = attend_smem<DD>(U);                                                                   \
+        SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<DD, H8, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                          int(sm)));                                                            \
+        SPA_CUDA_TRY(launch_pdl(attend_kernel<DD, H8, R>, dim3(grid), dim3(kAtThreads), sm, st, p, U, nh));      \
+        SPA_CUDA_TRY(launch_pdl(combine_kernel<DD, R>, dim3(U, nh), dim3(256), 0, st, p, nh, U + grid));          \
+        return SPA_OK;                                                                                          \
     }
-    SPA_AT_CASE(128, 1) SPA_AT_CASE(128, 2) SPA_AT_CASE(64, 1) SPA_AT_CASE(64, 2)
+    SPA_AT_CASE(128, 1, false) SPA_AT_CASE(128, 2, false) SPA_AT_CASE(64, 1, false) SPA_AT_CASE(64, 2, false)
+    SPA_AT_CASE(128, 1, true) SPA_AT_CASE(128, 2, true) SPA_AT_CASE(64, 1, true) SPA_AT_CASE(64, 2, true)
 #undef SPA_AT_CASE
     return SPA_ERR_UNSUPPORTED_SHAPE;
 }

@@ -163,6 +163,10 @@ spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st);
 spa_status launch_select(const SelectParams& p, bool topp, cudaStream_t st);
 size_t select_scratch_bytes(int U);
 
+// rla.cu: adds rows [n0, n1) of every (batch, kv head) into S [B*Hkv][d][d] and z [B*Hkv][d]
+spa_status launch_rla_state(const uint16_t* K, const uint16_t* V, int BH, int N, int d, int n0, int n1, float* S,
+                            float* z, cudaStream_t st);
+
 // prefill.cu
 size_t prefill_scratch_bytes(int U, int N);
 spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st);
@@ -184,8 +188,14 @@ struct AttendParams {
     float* lse;
     // workspace pieces
     int* unit_ctas;    // [U][2]: first and last CTA of a unit split over several CTAs, else -1
-    float* partials;   // [(U + grid) * heads_per_unit * (d + 2)]
+    float* partials;   // [(U + grid) * heads_per_unit * (d + 2)]; the RLA partials follow
     uint32_t* status;
+    // residual linear attention (null rla_S: off): state S [B*Hkv][d][d], z [B*Hkv][d],
+    // RMSNorm scale gamma [Hq][d] and epsilon
+    const float* rla_S;
+    const float* rla_z;
+    const float* rla_gamma;
+    float rla_eps;
 };
 size_t attend_scratch_bytes(int U, int heads_per_unit, int d);   // unit CTA ranges + partials
 int attend_grid();

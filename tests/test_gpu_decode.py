@@ -20,7 +20,7 @@ if not torch.cuda.is_available():
 import long_context_sparse_spa_b200 as spa  # noqa: E402
 
 
-def run_gpu(cfg, x, local=None):
+def run_gpu(cfg, x, local=None, rla=None):
     lowrank = cfg.score == "lowrank"
     kw = dict(
         score_kind=spa.SPA_SCORE_LOWRANK if lowrank else spa.SPA_SCORE_TAYLOR_BLOCK,
@@ -36,6 +36,10 @@ def run_gpu(cfg, x, local=None):
         kw.update(bmean=mean, bvar=var)
     if local is not None:
         kw["local_units"] = torch.from_numpy(np.asarray(local, np.uint8)).cuda()
+    if rla is not None:
+        S, z = spa.rla_state(kw["K"], kw["V"])            # the state of all N rows, once
+        kw.update(rla_state=S, rla_z=z, rla_gamma=torch.from_numpy(np.asarray(rla["gamma"], np.float32)).cuda(),
+                  rla_eps=float(np.float32(rla["eps"])))
     plan = spa.decode(**kw)
     torch.cuda.synchronize()
     assert spa.read_device_status(plan.ws) == 0
@@ -122,3 +126,61 @@ def test_decode_routed(name):
             np.testing.assert_allclose(g["lse"][b, heads], r["lse"], rtol=2e-6, atol=2e-6)
             if g["mass"] is not None and not local[u]:
                 assert abs(g["mass"][u] - r["index_mass"]) <= 4 * MASS_TIE_REL + 1e-6
+
+
+def _rla_params(cfg, seed=7):
+    rng = np.random.default_rng(seed)
+    return {"gamma": rng.uniform(0.5, 1.5, (cfg.Hq, cfg.d)).astype(np.float32), "eps": 1e-6}
+
+
+def check_decode_rla(cfg, local=None, units=None):
+    """Residual linear attention ("SPLA", sections 2.2-2.3): supports as without it, outputs
+    = exact + RMSNorm(RLA over the left-out rows), compared with the oracle's direct form."""
+    x = decode_inputs(cfg)
+    rla = _rla_params(cfg)
+    g = run_gpu(cfg, x, local=local, rla=rla)
+    G = cfg.G
+    worst, ties = 0.0, 0
+    all_units = oracle.decode_units(cfg)
+    for u in (range(cfg.U) if units is None else units):
+        b, h = all_units[u]
+        loc = bool(local[u]) if local is not None else False
+        r = oracle.decode_unit(cfg, x, u, local=loc, rla=rla)
+        got = g["idx"][u, :g["count"][u]]
+        if loc:
+            np.testing.assert_array_equal(got, r["idx"])
+            d = 0
+        else:
+            s = r["ranked"]
+            band = topk_band(s, cfg.topk) if cfg.select == "topk" else topp_band(s, oracle.f32(cfg.topp))
+            d = compare_support(got, r["idx"], band, f"{cfg.name} unit {u}")
+        ties += d
+        if d == 0:
+            heads = slice(h, h + 1) if cfg.collapse == "head" else slice(h * G, (h + 1) * G)
+            worst = max(worst, check_outputs(g["out"][b, heads], g["out32"][b, heads], r["out"],
+                                             f"{cfg.name} RLA unit {u}"))
+            np.testing.assert_allclose(g["lse"][b, heads], r["lse"], rtol=2e-6, atol=2e-6)
+    print(f"{cfg.name} RLA: max|err| {worst:.2e}, tie differences {ties}")
+
+
+@pytest.mark.parametrize("name", ["c1s", "c2s", "c3s"])
+def test_decode_rla(name):
+    check_decode_rla(SMALL[name])
+
+
+def test_decode_rla_routed():
+    cfg = SMALL["c2s"]
+    check_decode_rla(cfg, local=np.array([u % 2 for u in range(cfg.U)], np.uint8))
+
+
+def test_decode_rla_empty_and_full_supports():
+    # k = 0 with no sink or window: every support is empty, the output is the RLA of all rows;
+    # k >= M: the support is every row, RLA contributes nothing
+    check_decode_rla(SMALL["c1s"].with_(topk=0, sink=0, window=0))
+    check_decode_rla(SMALL["c1s"].with_(N=700, topk=800))
+
+
+def test_decode_rla_full_size_c3():
+    # the bench's launch configuration at full size; the oracle's direct RLA reads all 131072
+    # rows per head, so three units (first, middle, last) are compared
+    check_decode_rla(C3, units=[0, C3.U // 2 + 3, C3.U - 1])
