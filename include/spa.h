@@ -156,7 +156,7 @@ size_t spa_select_workspace_bytes(int U, int M);
  * framework owns every device buffer.
  * Arguments and results are those of spa_select_topp without (ws, ws_bytes).  The
  * scratch (a status word and the level-0 histograms of up to SPA_SELECT_STATIC_MAX_UNITS
- * units, about 385 KiB) is a fixed array in the library's device memory, held by every GPU
+ * units, about 960 KiB) is a fixed array in the library's device memory, held by every GPU
  * that loads the library until the process exits.  U > SPA_SELECT_STATIC_MAX_UNITS returns
  * SPA_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks up the array's device
  * address with cudaGetSymbolAddress (with that device current) and caches it; make that
@@ -185,9 +185,11 @@ spa_status spa_select_topp_static(const float* scores, const int32_t* unit_len, 
  *   lse    [B, Hq] fp32 out (optional): log sum_rows exp(sm_scale * q . k_row).
  *   An empty support gives out = 0 and lse = -inf.
  * Split-KV over all SMs: every CTA takes an equal share of all units' rows, gathers
- * them with cp.async, runs an fp32 online softmax on tensor-core tiles and emits a
- * partial (o, m, l); the last CTA of each unit merges the partials (log-sum-exp
- * combine).  d in {64, 128}; G <= 16 for GROUP_MEAN.  ws >= spa_attend_workspace_bytes.
+ * them with cp.async and runs an fp32 online softmax on tensor-core tiles.  A CTA that
+ * holds a whole unit writes its output; a unit split over several CTAs leaves one
+ * partial (o, m, l) per CTA, and a second kernel, one CTA per (unit, head), merges them
+ * in a fixed order (log-sum-exp combine).  d in {64, 128}; G <= 16 for GROUP_MEAN.
+ * ws >= spa_attend_workspace_bytes.
  */
 spa_status spa_sparse_attend(const uint16_t* q, const uint16_t* K, const uint16_t* V,
                              int B, int Hq, int Hkv, int N, int d,
