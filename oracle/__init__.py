@@ -54,7 +54,11 @@ def lib() -> ctypes.CDLL:
         L.orc_rla_direct.argtypes = [_p, _int, _p, _p, _i64, _int, _p, _i64, _int, _p]
         L.orc_rla_subtract.argtypes = [_p, _int, _p, _p, _i64, _int, _p, _i64, _int, _p, _p, _p]
         L.orc_rms_norm.argtypes = [_p, _int, _p, _dbl, _p]
-        assert L.orc_abi_version() == 2, "stale oracle library; rebuild it"
+        L.orc_pbs_importance.argtypes = [_p, _int, _int, _i64, _p, _i64, _int, _dbl, _p]
+        L.orc_pbs_permutation.argtypes = [_p, _i64, _i64, _p]
+        L.orc_pbs_prefill_unit.argtypes = [_p, _int, _int, _int, _i64, _p, _p, _i64, _p, _i64, _i64, _dbl, _p, _p]
+        L.orc_pbs_prefill_unit.restype = _i64
+        assert L.orc_abi_version() == 3, "stale oracle library; rebuild it"
         _LIB = L
     return _LIB
 
@@ -180,6 +184,42 @@ def rms_norm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
     y = np.empty_like(x)
     lib().orc_rms_norm(_ptr(x), x.size, _ptr(gamma), float(eps), _ptr(y))
     return y
+
+
+def pbs_importance(Qlast: np.ndarray, t_last0: int, K: np.ndarray, sm_scale: float) -> np.ndarray:
+    """Global key importance of PBS-Attn ("Sparser Block-Sparse Attention via Token
+    Permutation", section 3): the mean causal softmax probability each key receives from
+    the last query block.  Qlast [bl, G, d] bf16 at positions t_last0 ...; K [T, d]."""
+    Qlast = _c(Qlast, np.uint16); K = _c(K, np.uint16)
+    bl, G, d = Qlast.shape
+    imp = np.empty(K.shape[0])
+    lib().orc_pbs_importance(_ptr(Qlast), bl, G, t_last0, _ptr(K), K.shape[0], d, float(sm_scale), _ptr(imp))
+    return imp
+
+
+def pbs_permutation(imp: np.ndarray, S: int) -> np.ndarray:
+    """Intra-segment key order of PBS-Attn (sections 2-3): perm[p] = original position of
+    the key at permuted position p, sorted by descending importance inside each segment."""
+    imp = _c(imp, np.float64)
+    perm = np.empty(imp.size, np.int32)
+    lib().orc_pbs_permutation(_ptr(imp), imp.size, S, _ptr(perm))
+    return perm
+
+
+def pbs_prefill_unit(Qblk: np.ndarray, t0: int, K: np.ndarray, V: np.ndarray, perm: np.ndarray, S: int, k: int,
+                     sm_scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """One (query block, kv head) of the permuted block-sparse prefill (PBS-Attn, sections
+    1-4) -> (support: original positions of the k selected permuted blocks, ascending;
+    out [b, G, d] float64 over the support and the causal own segment)."""
+    Qblk = _c(Qblk, np.uint16); K = _c(K, np.uint16); V = _c(V, np.uint16); perm = _c(perm, np.int32)
+    b, G, d = Qblk.shape
+    support = np.empty(max(1, min(max(k, 0), K.shape[0] // b) * b), np.int32)
+    out = np.empty((b, G, d))
+    n = lib().orc_pbs_prefill_unit(_ptr(Qblk), b, G, d, t0, _ptr(K), _ptr(V), K.shape[0], _ptr(perm), S, k,
+                                   float(sm_scale), _ptr(support), _ptr(out))
+    if n < 0:
+        raise ValueError("need S % b == 0, t0 % b == 0 and t0 + b <= T")
+    return support[:n].copy(), out
 
 
 def dense_probs(q: np.ndarray, K: np.ndarray, sm_scale: float) -> np.ndarray:

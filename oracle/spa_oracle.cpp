@@ -29,6 +29,15 @@
 //            attention over all rows, so the left-out rows are never read.
 //   [SPLA-2.3] same page, section 2.3: the output is the exact sparse attention plus the
 //            RLA output passed through an RMSNorm whose scale is the only new parameter.
+//   [PBS-1]  "Sparser Block-Sparse Attention via Token Permutation" (PBS-Attn), section 1:
+//            attention is invariant to a joint permutation of the key-value pairs.
+//   [PBS-2]  same page, section 2: keys are permuted only inside contiguous segments of
+//            S tokens, so causality between segments is kept.
+//   [PBS-3]  same page, section 3: the global importance of a key is the mean-pooled
+//            attention it receives from the last query block; inside each segment keys are
+//            sorted by descending importance; queries keep their order.
+//   [PBS-4]  same page, section 4: blocks of the permuted keys are selected by a
+//            mean-pooled block score, then attention runs over the selected blocks.
 //
 // Parity pins (tests/test_oracle.py): dense attention and masked attention against
 // torch's fp64 scaled_dot_product_attention, top-k against numpy's lexsort, top-p
@@ -36,7 +45,10 @@
 // the Taylor score's zero-variance identity and fourth-order agreement on
 // axis-symmetric blocks, the prefill path against dense causal attention, and the
 // residual linear attention's subtraction form against its direct definition, its
-// closed forms (zero query, one left-out row) and brute-force Python loops.
+// closed forms (zero query, one left-out row) and brute-force Python loops, and the
+// permuted block-sparse prefill against dense causal attention (full budget), the
+// segment-local causal attention (empty budget), its invariance to a shuffle of the
+// key-value pairs inside segments, and a planted cluster of scattered heavy hitters.
 
 #include <algorithm>
 #include <cmath>
@@ -84,7 +96,7 @@ int64_t emit_ascending(const std::vector<char>& keep, int32_t* idx) {
 
 extern "C" {
 
-int orc_abi_version() { return 2; }
+int orc_abi_version() { return 3; }
 
 // a1 -- per-block mean and diagonal (population) variance of K [SPLA-2.1].
 // K: [N, d] bf16 of one (batch, kv head); only the nb = N / block full blocks count.
@@ -425,6 +437,98 @@ void orc_rms_norm(const double* x, int d, const double* gamma, double eps, doubl
     ms /= d;
     const double inv = 1.0 / std::sqrt(ms + eps);
     for (int j = 0; j < d; ++j) y[j] = gamma[j] * x[j] * inv;
+}
+
+// ---------------------------------------------------------------- PBS-Attn prefill
+// Global importance of every key [PBS-3]: the mean, over the bl queries of the last query
+// block (positions t_last0 ...) and the G query heads sharing the kv head, of their causal
+// softmax probabilities softmax_n(sm_scale * q . k_n), n <= t (0 for keys after t).
+// Qlast [bl, G, d] bf16; K [T, d] bf16; imp [T] out.
+void orc_pbs_importance(const uint16_t* Qlast, int bl, int G, int64_t t_last0, const uint16_t* K, int64_t T,
+                        int d, double sm_scale, double* imp) {
+    std::fill(imp, imp + T, 0.0);
+    std::vector<double> logit(static_cast<size_t>(T));
+    for (int i = 0; i < bl; ++i)
+        for (int h = 0; h < G; ++h) {
+            const uint16_t* q = Qlast + (static_cast<int64_t>(i) * G + h) * d;
+            const int64_t t = std::min(t_last0 + i, T - 1);
+            double mx = -std::numeric_limits<double>::infinity();
+            for (int64_t n = 0; n <= t; ++n) {
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += widen_bf16(q[c]) * widen_bf16(K[n * d + c]);
+                logit[static_cast<size_t>(n)] = sm_scale * dot;
+                mx = std::max(mx, logit[static_cast<size_t>(n)]);
+            }
+            double Z = 0.0;
+            for (int64_t n = 0; n <= t; ++n) Z += std::exp(logit[static_cast<size_t>(n)] - mx);
+            for (int64_t n = 0; n <= t; ++n)
+                imp[n] += std::exp(logit[static_cast<size_t>(n)] - mx) / Z / (static_cast<double>(bl) * G);
+        }
+}
+
+// Intra-segment key order [PBS-2, PBS-3]: inside each segment [j S, min((j + 1) S, T)) the
+// keys sorted by descending importance, equal importance by ascending position.
+// perm[p] = original position of the key at permuted position p.
+void orc_pbs_permutation(const double* imp, int64_t T, int64_t S, int32_t* perm) {
+    for (int64_t s0 = 0; s0 < T; s0 += S) {
+        const int64_t len = std::min(S, T - s0);
+        const std::vector<int64_t> order = rank_order(imp + s0, len);
+        for (int64_t p = 0; p < len; ++p) perm[s0 + p] = static_cast<int32_t>(s0 + order[static_cast<size_t>(p)]);
+    }
+}
+
+// One (query block, kv head) of the permuted block-sparse prefill [PBS-1..4].
+// Qblk [b, G, d] bf16: the block's queries at positions t0 .. t0 + b - 1 (t0 a multiple of
+// b, S a multiple of b) for the G heads of the kv head; K, V [T, d] bf16; perm from
+// orc_pbs_permutation.  The query block lies in segment j = t0 / S.  Candidates are the
+// blocks of b consecutive permuted keys in segments 0 .. j - 1; block c scores
+// sm_scale * qbar . kbar_c, qbar the mean of the block's b x G queries and kbar_c the mean
+// of the block's keys (mean pooling); the k best (score desc, block asc) are selected.
+// support [min(k, candidates) * b] out: the original positions of the selected keys,
+// ascending; returns their number.  out [b, G, d]: for query t and head h, softmax
+// attention over the support and the keys [j S, t] of its own segment (causal by original
+// position; the diagonal segment is never skipped).
+int64_t orc_pbs_prefill_unit(const uint16_t* Qblk, int b, int G, int d, int64_t t0, const uint16_t* K,
+                             const uint16_t* V, int64_t T, const int32_t* perm, int64_t S, int64_t k,
+                             double sm_scale, int32_t* support, double* out) {
+    if (b <= 0 || S % b != 0 || t0 % b != 0 || t0 + b > T) return -1;
+    const int64_t seg0 = t0 / S * S;
+    const int64_t nc = seg0 / b;                       // candidate blocks
+    std::vector<double> qbar(d, 0.0);
+    for (int i = 0; i < b; ++i)
+        for (int h = 0; h < G; ++h)
+            for (int c = 0; c < d; ++c) qbar[c] += widen_bf16(Qblk[(static_cast<int64_t>(i) * G + h) * d + c]);
+    for (int c = 0; c < d; ++c) qbar[c] /= static_cast<double>(b) * G;
+    std::vector<double> score(static_cast<size_t>(nc));
+    for (int64_t blk = 0; blk < nc; ++blk) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) {
+            double kbar = 0.0;
+            for (int64_t p = blk * b; p < (blk + 1) * b; ++p) kbar += widen_bf16(K[static_cast<int64_t>(perm[p]) * d + c]);
+            dot += qbar[c] * (kbar / b);
+        }
+        score[static_cast<size_t>(blk)] = sm_scale * dot;
+    }
+    const std::vector<int64_t> order = rank_order(score.data(), nc);
+    const int64_t nsel = std::min<int64_t>(std::max<int64_t>(k, 0), nc);
+    std::vector<int32_t> rows;
+    for (int64_t r = 0; r < nsel; ++r)
+        for (int64_t p = order[static_cast<size_t>(r)] * b; p < (order[static_cast<size_t>(r)] + 1) * b; ++p)
+            rows.push_back(perm[p]);
+    std::sort(rows.begin(), rows.end());
+    std::copy(rows.begin(), rows.end(), support);
+    const int64_t n_sup = static_cast<int64_t>(rows.size());
+    for (int i = 0; i < b; ++i) {
+        const int64_t t = t0 + i;
+        std::vector<int32_t> all(rows);
+        for (int64_t n = seg0; n <= t; ++n) all.push_back(static_cast<int32_t>(n));
+        for (int h = 0; h < G; ++h) {
+            const int64_t qi = static_cast<int64_t>(i) * G + h;
+            orc_sparse_attention(Qblk + qi * d, 1, K, V, T, d, all.data(), static_cast<int64_t>(all.size()), 1,
+                                 sm_scale, out + qi * d, nullptr);
+        }
+    }
+    return n_sup;
 }
 
 }  // extern "C"
