@@ -58,7 +58,10 @@ def lib() -> ctypes.CDLL:
         L.orc_pbs_permutation.argtypes = [_p, _i64, _i64, _p]
         L.orc_pbs_prefill_unit.argtypes = [_p, _int, _int, _int, _i64, _p, _p, _i64, _p, _i64, _i64, _dbl, _p, _p]
         L.orc_pbs_prefill_unit.restype = _i64
-        assert L.orc_abi_version() == 3, "stale oracle library; rebuild it"
+        L.orc_block_minmax.argtypes = [_p, _i64, _int, _int, _p, _p]
+        L.orc_minmax_scores.argtypes = [_p, _int, _p, _p, _i64, _int, _dbl, _int, _p]
+        L.orc_mean_scores.argtypes = [_p, _int, _p, _i64, _int, _dbl, _int, _p]
+        assert L.orc_abi_version() == 4, "stale oracle library; rebuild it"
         _LIB = L
     return _LIB
 
@@ -104,6 +107,40 @@ def taylor_scores(q: np.ndarray, mean: np.ndarray, var: np.ndarray, scale: float
     nb = mean.shape[0]
     out = np.empty(nb if collapse else (G, nb))
     lib().orc_taylor_scores(_ptr(q), G, _ptr(mean), _ptr(var), nb, d, float(scale), int(collapse), _ptr(out))
+    return out
+
+
+def block_minmax(K: np.ndarray, block: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-block channel min and max of K [N, d] bf16 bits (full blocks) -> [nb, d] float64
+    ("SPLA", section 1: min/max pooling)."""
+    K = _c(K, np.uint16)
+    N, d = K.shape
+    nb = N // block
+    mn = np.empty((nb, d)); mx = np.empty((nb, d))
+    lib().orc_block_minmax(_ptr(K), N, d, block, _ptr(mn), _ptr(mx))
+    return mn, mx
+
+
+def minmax_scores(q: np.ndarray, mn: np.ndarray, mx: np.ndarray, scale: float, collapse: bool) -> np.ndarray:
+    """Min-max page score: scale * sum_i max(q_i mn_i, q_i mx_i), the upper bound of every
+    key logit in the block ("SPLA" section 1; "The Sparse Frontier", token-to-page decode
+    selection).  q [G, d] bf16 bits -> [nb] (mean over heads) or [G, nb]."""
+    q = _c(q, np.uint16); mn = _c(mn, np.float64); mx = _c(mx, np.float64)
+    G, d = q.shape
+    nb = mn.shape[0]
+    out = np.empty(nb if collapse else (G, nb))
+    lib().orc_minmax_scores(_ptr(q), G, _ptr(mn), _ptr(mx), nb, d, float(scale), int(collapse), _ptr(out))
+    return out
+
+
+def mean_scores(q: np.ndarray, mean: np.ndarray, scale: float, collapse: bool) -> np.ndarray:
+    """Mean-pooling block score scale * q . kbar ("SPLA" section 1; PBS-Attn section 4).
+    q [G, d] bf16 bits, mean [nb, d] -> [nb] (mean over heads) or [G, nb]."""
+    q = _c(q, np.uint16); mean = _c(mean, np.float64)
+    G, d = q.shape
+    nb = mean.shape[0]
+    out = np.empty(nb if collapse else (G, nb))
+    lib().orc_mean_scores(_ptr(q), G, _ptr(mean), nb, d, float(scale), int(collapse), _ptr(out))
     return out
 
 

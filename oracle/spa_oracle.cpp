@@ -29,6 +29,10 @@
 //            attention over all rows, so the left-out rows are never read.
 //   [SPLA-2.3] same page, section 2.3: the output is the exact sparse attention plus the
 //            RLA output passed through an RMSNorm whose scale is the only new parameter.
+//   [SPLA-1] "SPLA", section 1: the block proxies it improves on -- min/max pooling and
+//            plain mean pooling of a block's keys.
+//   [SF-4]   "The Sparse Frontier", decoding findings: token-to-page selection over a full
+//            KV cache (Quest) for decode.
 //   [PBS-1]  "Sparser Block-Sparse Attention via Token Permutation" (PBS-Attn), section 1:
 //            attention is invariant to a joint permutation of the key-value pairs.
 //   [PBS-2]  same page, section 2: keys are permuted only inside contiguous segments of
@@ -96,7 +100,7 @@ int64_t emit_ascending(const std::vector<char>& keep, int32_t* idx) {
 
 extern "C" {
 
-int orc_abi_version() { return 3; }
+int orc_abi_version() { return 4; }
 
 // a1 -- per-block mean and diagonal (population) variance of K [SPLA-2.1].
 // K: [N, d] bf16 of one (batch, kv head); only the nb = N / block full blocks count.
@@ -529,6 +533,60 @@ int64_t orc_pbs_prefill_unit(const uint16_t* Qblk, int b, int G, int d, int64_t 
         }
     }
     return n_sup;
+}
+
+// ---------------------------------------------------------------- first-order block proxies
+// Per-block channel minimum and maximum of K [SPLA-1] (full blocks only, like a1).
+// K [N, d] bf16; mn, mx [N / block, d] out.
+void orc_block_minmax(const uint16_t* K, int64_t N, int d, int block, double* mn, double* mx) {
+    const int64_t nb = N / block;
+    for (int64_t b = 0; b < nb; ++b)
+        for (int c = 0; c < d; ++c) {
+            double lo = std::numeric_limits<double>::infinity(), hi = -lo;
+            for (int64_t n = b * block; n < (b + 1) * block; ++n) {
+                lo = std::min(lo, widen_bf16(K[n * d + c]));
+                hi = std::max(hi, widen_bf16(K[n * d + c]));
+            }
+            mn[b * d + c] = lo;
+            mx[b * d + c] = hi;
+        }
+}
+
+// Min-max page score [SPLA-1, SF-4]: the largest scale * q . k over every k inside the
+// block's channel box [mn, mx], s_{h,b} = scale * sum_i max(q_i mn_{b,i}, q_i mx_{b,i}); an
+// upper bound of every key's logit in the block.  q [G, d] bf16; collapse = 0: out [G, nb];
+// collapse = 1: out [nb] = mean over the G heads.
+void orc_minmax_scores(const uint16_t* q, int G, const double* mn, const double* mx, int64_t nb, int d,
+                       double scale, int collapse, double* out) {
+    for (int64_t b = 0; b < nb; ++b) {
+        double acc = 0.0;
+        for (int h = 0; h < G; ++h) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const double qc = widen_bf16(q[h * d + c]);
+                s += std::max(qc * mn[b * d + c], qc * mx[b * d + c]);
+            }
+            s *= scale;
+            if (collapse) acc += s; else out[h * nb + b] = s;
+        }
+        if (collapse) out[b] = acc / G;
+    }
+}
+
+// Mean-pooling block score [SPLA-1, PBS-4]: s_{h,b} = scale * q_h . kbar_b (the first-order
+// term of the Taylor score).  mean [nb, d]; collapse as orc_minmax_scores.
+void orc_mean_scores(const uint16_t* q, int G, const double* mean, int64_t nb, int d, double scale, int collapse,
+                     double* out) {
+    for (int64_t b = 0; b < nb; ++b) {
+        double acc = 0.0;
+        for (int h = 0; h < G; ++h) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s += widen_bf16(q[h * d + c]) * mean[b * d + c];
+            s *= scale;
+            if (collapse) acc += s; else out[h * nb + b] = s;
+        }
+        if (collapse) out[b] = acc / G;
+    }
 }
 
 }  // extern "C"
