@@ -61,7 +61,9 @@ typedef enum spa_collapse {
 
 typedef enum spa_score_kind {
     SPA_SCORE_LOWRANK = 0,      /* s_n = scale * qhat . Kidx_n (r = 16) */
-    SPA_SCORE_TAYLOR_BLOCK = 1  /* s_b = log t_b, t_b = mean_h exp(q'_h . mean_b)(1 + 1/2 sum_i q'_hi^2 var_bi), q' = scale * q */
+    SPA_SCORE_TAYLOR_BLOCK = 1, /* s_b = log t_b, t_b = mean_h exp(q'_h . mean_b)(1 + 1/2 sum_i q'_hi^2 var_bi), q' = scale * q */
+    SPA_SCORE_MINMAX_BLOCK = 2, /* s_b = mean_h sum_i max(q'_hi min_bi, q'_hi max_bi): the largest logit in the block's channel box */
+    SPA_SCORE_MEAN_BLOCK = 3    /* s_b = mean_h q'_h . mean_b (first-order, mean pooling) */
 } spa_score_kind;
 
 typedef enum spa_select_kind {
@@ -75,7 +77,8 @@ const char* spa_status_string(int status);
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
 const char* spa_last_cuda_error(void);
 
-/* ABI version of this header: 3 (spa_decode_args gained local_units in 2, the RLA fields in 3). */
+/* ABI version of this header: 4 (spa_decode_args gained local_units in 2, the RLA fields in 3;
+ * the min-max and mean block scores and spa_block_minmax came in 4). */
 int spa_abi_version(void);
 
 /* ------------------------------------------------------------------------------------
@@ -89,6 +92,13 @@ int spa_abi_version(void);
  */
 spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block,
                            float* mean, float* var, void* stream);
+
+/* Per-block channel minimum and maximum of K (min/max pooling, the block proxy "SPLA" 1
+ * compares against; the statistics of token-to-page selection, "The Sparse Frontier"):
+ *   mn, mx [B, Hkv, N / block, d] fp32 out, exact.  Full blocks only; shapes as
+ *   spa_block_stats. */
+spa_status spa_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block,
+                            float* mn, float* mx, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * a2/a3. Index scores, one row of M scores per selection unit.
@@ -106,6 +116,11 @@ spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int 
  *   s[u, b] = log t, t = exp(q'.mean_b) * (1 + 1/2 sum_i q'_i^2 var_bi), q' = scale * q,
  *   with t averaged over the G heads of kv head g (GROUP_MEAN) or per head (NONE).  The
  *   log keeps the score finite for any input; it ranks blocks exactly as t does.
+ * kind = SPA_SCORE_MINMAX_BLOCK: keys = block minima, var = block maxima (spa_block_minmax);
+ *   s[u, b] = sum_i max(q'_i min_bi, q'_i max_bi), q' = scale * q, scale > 0; averaged
+ *   over the G heads under GROUP_MEAN.
+ * kind = SPA_SCORE_MEAN_BLOCK: keys = block means, var NULL (not read);
+ *   s[u, b] = q' . mean_b; averaged over the G heads under GROUP_MEAN.
  * scores [U, M] fp32 out.  G = Hq / Hkv must be an integer, G <= 16.
  */
 spa_status spa_index_scores(int kind, const void* q, const void* keys, const float* var,
@@ -211,15 +226,15 @@ typedef struct spa_decode_args {
     int collapse;            /* spa_collapse */
     int B, Hq, Hkv, N, d;
     int r;                   /* index dim (LOWRANK), 16 */
-    int block;               /* tokens per scored unit: 1 (LOWRANK) or the block size (TAYLOR) */
+    int block;               /* tokens per scored unit: 1 (LOWRANK) or the block size (block kinds) */
     const uint16_t* q;       /* [B, Hq, d] */
     const uint16_t* q_idx;   /* [B, Hq, r] (LOWRANK) */
     const uint16_t* K;       /* [B, Hkv, N, d] */
     const uint16_t* V;       /* [B, Hkv, N, d] */
     const uint16_t* Kidx;    /* [B, Hkv, N, r] (LOWRANK) */
-    const float* bmean;      /* [B, Hkv, N / block, d] (TAYLOR) */
-    const float* bvar;       /* [B, Hkv, N / block, d] (TAYLOR) */
-    float score_scale;       /* LOWRANK: index-score scale; TAYLOR: q' = score_scale * q */
+    const float* bmean;      /* [B, Hkv, N / block, d]: TAYLOR and MEAN block means; MINMAX block minima */
+    const float* bvar;       /* [B, Hkv, N / block, d]: TAYLOR block variances; MINMAX block maxima; MEAN unused */
+    float score_scale;       /* LOWRANK: index-score scale; block kinds: q' = score_scale * q */
     float sm_scale;          /* softmax scale of the exact attention */
     int topk;                /* SPA_SELECT_TOPK */
     float topp;              /* SPA_SELECT_TOPP */

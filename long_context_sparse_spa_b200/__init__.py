@@ -17,13 +17,14 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK, SPA_SCORE_TAYLOR_BLOCK,
-                   SPA_SELECT_TOPK, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
+from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK, SPA_SCORE_MEAN_BLOCK,
+                   SPA_SCORE_MINMAX_BLOCK, SPA_SCORE_TAYLOR_BLOCK, SPA_SELECT_TOPK, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
 
 __all__ = [
     "SpaError", "lib", "lib_path", "block_stats", "index_scores", "select_topk", "select_topp", "sparse_attend",
     "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "prefill", "PrefillPlan", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
-    "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SELECT_TOPK", "SPA_SELECT_TOPP",
+    "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SCORE_MINMAX_BLOCK", "SPA_SCORE_MEAN_BLOCK",
+    "SPA_SELECT_TOPK", "SPA_SELECT_TOPP", "block_minmax", "rla_state",
 ]
 
 
@@ -69,11 +70,23 @@ def block_stats(K: torch.Tensor, block: int = 64) -> Tuple[torch.Tensor, torch.T
     return mean, var
 
 
+def block_minmax(K: torch.Tensor, block: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K [B, Hkv, N, d] bf16 -> per-block channel (min, max) [B, Hkv, N // block, d] fp32."""
+    _need(K, torch.bfloat16, "K")
+    B, Hkv, N, d = K.shape
+    nb = N // block
+    mn = torch.empty((B, Hkv, nb, d), dtype=torch.float32, device=K.device)
+    mx = torch.empty_like(mn)
+    check(lib().spa_block_minmax(_ptr(K), B, Hkv, N, d, block, _ptr(mn), _ptr(mx), _stream()))
+    return mn, mx
+
+
 # ----------------------------------------------------------------------------- a2/a3
 def index_scores(kind: int, q: torch.Tensor, keys: torch.Tensor, var: Optional[torch.Tensor], Hkv: int,
                  collapse: int, scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Scores [U, M] fp32.  LOWRANK: q = q_idx [B, Hq, 16] bf16, keys = Kidx [B, Hkv, M, 16] bf16.
-    TAYLOR: q [B, Hq, d] bf16, keys = block means [B, Hkv, M, d] fp32, var likewise."""
+    TAYLOR: q [B, Hq, d] bf16, keys = block means [B, Hkv, M, d] fp32, var likewise.
+    MINMAX: keys = block minima, var = block maxima.  MEAN: keys = block means, var None."""
     _need(q, torch.bfloat16, "q")
     B, Hq, dim = q.shape
     M = keys.shape[2]
@@ -81,7 +94,8 @@ def index_scores(kind: int, q: torch.Tensor, keys: torch.Tensor, var: Optional[t
         _need(keys, torch.bfloat16, "keys")
     else:
         _need(keys, torch.float32, "keys")
-        _need(var, torch.float32, "var")
+        if kind != SPA_SCORE_MEAN_BLOCK:
+            _need(var, torch.float32, "var")
     U = B * (Hkv if collapse == SPA_COLLAPSE_GROUP_MEAN else Hq)
     if out is None:
         out = torch.empty((U, M), dtype=torch.float32, device=q.device)

@@ -7,7 +7,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(HERE, "libspa.so")
 
-ABI_VERSION = 3   # spa_abi_version() of the library these declarations describe
+ABI_VERSION = 4   # spa_abi_version() of the library these declarations describe
 
 SPA_OK = 0
 SPA_ERR_INVALID_ARG = 1
@@ -21,6 +21,8 @@ SPA_COLLAPSE_NONE = 0
 SPA_COLLAPSE_GROUP_MEAN = 1
 SPA_SCORE_LOWRANK = 0
 SPA_SCORE_TAYLOR_BLOCK = 1
+SPA_SCORE_MINMAX_BLOCK = 2
+SPA_SCORE_MEAN_BLOCK = 3
 SPA_SELECT_TOPK = 0
 SPA_SELECT_TOPP = 1
 SPA_SELECT_STATIC_MAX_UNITS = 16
@@ -72,6 +74,7 @@ SIGNATURES = {
     "spa_select_topp": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p, _sz, _p]),
     "spa_select_workspace_bytes": (_sz, [_i, _i]),
     "spa_select_topp_static": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p]),
+    "spa_block_minmax": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_rla_state": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_sparse_attend": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "spa_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),

@@ -73,7 +73,7 @@ const char* spa_status_string(int s) {
 
 const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
-int spa_abi_version(void) { return 3; }
+int spa_abi_version(void) { return 4; }
 
 spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean, float* var,
                            void* stream) {
@@ -83,6 +83,28 @@ spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int 
     if ((d != 64 && d != 128) || (block != 32 && block != 64 && block != 128)) return SPA_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(K) || !aligned16(mean) || !aligned16(var)) return SPA_ERR_UNSUPPORTED_SHAPE;
     return launch_block_stats(K, B, Hkv, N, d, block, mean, var, static_cast<cudaStream_t>(stream));
+}
+
+spa_status spa_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mn, float* mx,
+                            void* stream) {
+    if (B < 0 || Hkv <= 0 || N < 0 || block <= 0) return SPA_ERR_INVALID_ARG;
+    if (B == 0 || N / block == 0) return SPA_OK;
+    if (!K || !mn || !mx) return SPA_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || (block != 32 && block != 64 && block != 128)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(K) || !aligned16(mn) || !aligned16(mx)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    return launch_block_minmax(K, B, Hkv, N, d, block, mn, mx, static_cast<cudaStream_t>(stream));
+}
+
+// block score kinds other than low-rank, with their statistics' requirements
+static spa_status check_block_kind(int kind, const void* a, const void* b, float scale) {
+    if (!a || (kind != SPA_SCORE_MEAN_BLOCK && !b)) return SPA_ERR_INVALID_ARG;
+    if (kind == SPA_SCORE_MINMAX_BLOCK && !(scale > 0.f)) return SPA_ERR_INVALID_ARG;
+    if (!aligned16(a) || (b && !aligned16(b))) return SPA_ERR_UNSUPPORTED_SHAPE;
+    return SPA_OK;
+}
+
+static bool is_block_kind(int kind) {
+    return kind == SPA_SCORE_TAYLOR_BLOCK || kind == SPA_SCORE_MINMAX_BLOCK || kind == SPA_SCORE_MEAN_BLOCK;
 }
 
 spa_status spa_index_scores(int kind, const void* q, const void* keys, const float* var, int B, int Hq, int Hkv,
@@ -100,12 +122,12 @@ spa_status spa_index_scores(int kind, const void* q, const void* keys, const flo
         return launch_lowrank_scores(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(keys), B, Hq, Hkv,
                                      M, collapse, scale, scores, nullptr, false, st);
     }
-    if (kind == SPA_SCORE_TAYLOR_BLOCK) {
-        if (!var) return SPA_ERR_INVALID_ARG;
+    if (is_block_kind(kind)) {
+        spa_status s = check_block_kind(kind, keys, var, scale);
+        if (s != SPA_OK) return s;
         if (dim != 64 && dim != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
-        if (!aligned16(keys) || !aligned16(var)) return SPA_ERR_UNSUPPORTED_SHAPE;
         return launch_taylor_scores(static_cast<const uint16_t*>(q), static_cast<const float*>(keys), var, B, Hq,
-                                    Hkv, M, dim, collapse, scale, scores, st);
+                                    Hkv, M, dim, collapse, scale, scores, st, nullptr, kind);
     }
     return SPA_ERR_INVALID_ARG;
 }
@@ -229,7 +251,7 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     const bool group = a->collapse == SPA_COLLAPSE_GROUP_MEAN;
     if (!group && a->collapse != SPA_COLLAPSE_NONE) return SPA_ERR_INVALID_ARG;
     const int U = group ? a->B * a->Hkv : a->B * a->Hq;
-    const bool taylor = a->score_kind == SPA_SCORE_TAYLOR_BLOCK;
+    const bool taylor = is_block_kind(a->score_kind);   // block scores (Taylor, min-max or mean)
     if (!taylor && a->score_kind != SPA_SCORE_LOWRANK) return SPA_ERR_INVALID_ARG;
     const int block = taylor ? a->block : 1;
     if (block <= 0 || (!taylor && a->block > 1)) return SPA_ERR_INVALID_ARG;
@@ -245,9 +267,9 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     }
     if (a->sink < 0 || a->window < 0 || a->cap < 0) return SPA_ERR_INVALID_ARG;
     if (taylor) {
-        if (!a->bmean || !a->bvar) return SPA_ERR_INVALID_ARG;
+        const spa_status sb = check_block_kind(a->score_kind, a->bmean, a->bvar, a->score_scale);
+        if (sb != SPA_OK) return sb;
         if (a->d != 64 && a->d != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
-        if (!aligned16(a->bmean) || !aligned16(a->bvar)) return SPA_ERR_UNSUPPORTED_SHAPE;
     } else {
         if (!a->q_idx || !a->Kidx) return SPA_ERR_INVALID_ARG;
         if (a->r != 16) return SPA_ERR_UNSUPPORTED_SHAPE;
@@ -289,7 +311,7 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     if ((s = mark(0)) != SPA_OK) return s;
     if (taylor) {
         s = launch_taylor_scores(a->q, a->bmean, a->bvar, a->B, a->Hq, a->Hkv, M, a->d, a->collapse,
-                                 a->score_scale, scores, st, a->local_units);
+                                 a->score_scale, scores, st, a->local_units, a->score_kind);
     } else {
         s = launch_lowrank_scores(a->q_idx, a->Kidx, a->B, a->Hq, a->Hkv, M, a->collapse, a->score_scale, scores,
                                   fused_hist ? &hist : nullptr, topp, st, a->local_units);

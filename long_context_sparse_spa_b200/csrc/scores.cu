@@ -153,15 +153,22 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
     }
 }
 
-// ============================================================================ Taylor
+// ============================================================================ block scores
 // One work item = (kv unit, chunk of kTyChunk blocks).  Eight lanes share a block: each
-// holds D/8 dims of the block mean and variance (float4 loads) and the partial sums
-// a_h = q'_h . mean and c_h = sum q'_h^2 var for the G heads are joined by three
-// xor-shuffles.  q' = scale * q lives in shared memory.
+// holds D/8 dims of the block statistics (float4 loads) and the per-head partial sums for
+// the G heads are joined by three xor-shuffles.  q' = scale * q lives in shared memory.
+//   KIND_TAYLOR ("SPLA" 2.1): stats (mean, var); a_h = q'_h . mean, c_h = sum q'_h^2 var,
+//                 score log t (t averaged over the heads under GROUP_MEAN).
+//   KIND_MINMAX (min/max pooling, "SPLA" 1; token-to-page selection, "The Sparse
+//                 Frontier"): stats (min, max); a_h = sum_i max(q'_i min_i, q'_i max_i),
+//                 the largest logit inside the block's channel box.
+//   KIND_MEAN   (mean pooling, "SPLA" 1, PBS-Attn 4): stats (mean); a_h = q'_h . mean.
+//   Under GROUP_MEAN the min-max and mean scores are averaged over the G heads.
 constexpr int kTyThreads = 256;
 constexpr int kTyChunk = 256;
+constexpr int KIND_TAYLOR = 0, KIND_MINMAX = 1, KIND_MEAN = 2;
 
-template <int D, int G>
+template <int D, int G, int KIND>
 __global__ void __launch_bounds__(kTyThreads)
 taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ mean, const float4* __restrict__ var,
                      int Hq, int Hkv, int M, int collapse, float scale, float* __restrict__ scores,
@@ -205,7 +212,7 @@ taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ 
                     // lane8 owns dims {4*(lane8 + 8*v) .. +3}: 8 lanes read 128 contiguous bytes
                     const int f4 = lane8 + 8 * v;
                     const float4 mu = __ldg(mean + base + f4);
-                    const float4 vr = __ldg(var + base + f4);
+                    const float4 vr = KIND == KIND_MEAN ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(var + base + f4);
                     const float mus[4] = {mu.x, mu.y, mu.z, mu.w};
                     const float vrs[4] = {vr.x, vr.y, vr.z, vr.w};
 #pragma unroll
@@ -214,8 +221,12 @@ taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ 
 #pragma unroll
                         for (int h = 0; h < G; ++h) {
                             const float qp = qs[h][i];
-                            a[h] = fmaf(qp, mus[e], a[h]);
-                            c[h] = fmaf(qp * qp, vrs[e], c[h]);
+                            if (KIND == KIND_MINMAX) {
+                                a[h] += fmaxf(qp * mus[e], qp * vrs[e]);
+                            } else {
+                                a[h] = fmaf(qp, mus[e], a[h]);
+                                if (KIND == KIND_TAYLOR) c[h] = fmaf(qp * qp, vrs[e], c[h]);
+                            }
                         }
                     }
                 }
@@ -229,6 +240,21 @@ taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ 
                 }
             }
             if (!live) continue;
+            if (KIND != KIND_TAYLOR) {
+                if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
+                    if (lane8 == 0) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) acc += a[h];
+                        scores[size_t(kvu) * M + blk] = acc / float(G);
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        if ((h & 7) == lane8) scores[(size_t(b) * Hq + size_t(g) * G + h) * M + blk] = a[h];
+                }
+                continue;
+            }
             if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
                 if (lane8 == 0) {
                     float mx = a[0];
@@ -325,6 +351,62 @@ block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, i
     }
 }
 
+// Per-block channel minimum and maximum of K (min/max pooling, "SPLA" 1): the loads of
+// block_stats_kernel, one pass, exact (bf16 values are exact in fp32).
+template <int D, int BLOCK>
+__global__ void __launch_bounds__(128)
+block_minmax_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, float* __restrict__ mn,
+                    float* __restrict__ mx) {
+    pdl_enter();
+    constexpr int DV = D / 8;
+    constexpr int PH = 128 / DV;
+    constexpr int RPT = BLOCK / PH;
+    static_assert(RPT * PH == BLOCK, "block must be a multiple of the row phases");
+    __shared__ float rlo[PH][D], rhi[PH][D];
+    const int c = threadIdx.x % DV;
+    const int ph = threadIdx.x / DV;
+
+    for (int blk = blockIdx.x; blk < n_blocks; blk += gridDim.x) {
+        const int unit = blk / nb_per_unit;
+        const int j = blk - unit * nb_per_unit;
+        const uint4* base = K + (size_t(unit) * N + size_t(j) * BLOCK) * DV + c;
+        uint4 w[RPT];
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) w[i] = __ldg(base + size_t(ph + i * PH) * DV);
+        float lo[8], hi[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = INFINITY; hi[e] = -INFINITY; }
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                lo[2 * e] = fminf(lo[2 * e], bf_lo(ws[e]));
+                hi[2 * e] = fmaxf(hi[2 * e], bf_lo(ws[e]));
+                lo[2 * e + 1] = fminf(lo[2 * e + 1], bf_hi(ws[e]));
+                hi[2 * e + 1] = fmaxf(hi[2 * e + 1], bf_hi(ws[e]));
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            rlo[ph][c * 8 + e] = lo[e];
+            rhi[ph][c * 8 + e] = hi[e];
+        }
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float l = INFINITY, h = -INFINITY;
+#pragma unroll
+            for (int p = 0; p < PH; ++p) {
+                l = fminf(l, rlo[p][threadIdx.x]);
+                h = fmaxf(h, rhi[p][threadIdx.x]);
+            }
+            mn[size_t(blk) * D + threadIdx.x] = l;
+            mx[size_t(blk) * D + threadIdx.x] = h;
+        }
+        __syncthreads();
+    }
+}
+
 int grid_for(int items, int per_sm) {
     const int cap = device_info().num_sms * per_sm;
     return items < cap ? (items > 0 ? items : 1) : cap;
@@ -364,22 +446,48 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
 
 spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
                                 int M, int d, int collapse, float scale, float* scores, cudaStream_t st,
-                                const uint8_t* local) {
+                                const uint8_t* local, int kind) {
     const int G = Hq / Hkv;
     const int chunks = (M + kTyChunk - 1) / kTyChunk;
     const int items = B * Hkv * chunks;
     const int grid = grid_for(items, 8);
     const float4* m4 = reinterpret_cast<const float4*>(mean);
     const float4* v4 = reinterpret_cast<const float4*>(var);
-#define SPA_TY_CASE(D, GG)                                                                                  \
-    if (d == D && G == GG) {                                                                               \
-        SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG>, dim3(grid), dim3(kTyThreads), 0, st, q, m4, v4, Hq,  \
-                                Hkv, M, collapse, scale, scores, chunks, items, local));                    \
-        return SPA_OK;                                                                                     \
+#define SPA_TY_CASE(D, GG)                                                                                   \
+    if (d == D && G == GG) {                                                                                \
+        if (kind == SPA_SCORE_MINMAX_BLOCK)                                                                 \
+            SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KIND_MINMAX>, dim3(grid), dim3(kTyThreads), 0, st, \
+                                    q, m4, v4, Hq, Hkv, M, collapse, scale, scores, chunks, items, local));       \
+        else if (kind == SPA_SCORE_MEAN_BLOCK)                                                              \
+            SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KIND_MEAN>, dim3(grid), dim3(kTyThreads), 0, st,   \
+                                    q, m4, v4, Hq, Hkv, M, collapse, scale, scores, chunks, items, local));       \
+        else                                                                                                \
+            SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KIND_TAYLOR>, dim3(grid), dim3(kTyThreads), 0, st, \
+                                    q, m4, v4, Hq, Hkv, M, collapse, scale, scores, chunks, items, local));       \
+        return SPA_OK;                                                                                      \
     }
     SPA_TY_CASE(64, 1) SPA_TY_CASE(64, 2) SPA_TY_CASE(64, 4) SPA_TY_CASE(64, 8) SPA_TY_CASE(64, 16)
     SPA_TY_CASE(128, 1) SPA_TY_CASE(128, 2) SPA_TY_CASE(128, 4) SPA_TY_CASE(128, 8) SPA_TY_CASE(128, 16)
 #undef SPA_TY_CASE
+    return SPA_ERR_UNSUPPORTED_SHAPE;
+}
+
+spa_status launch_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mn, float* mx,
+                               cudaStream_t st) {
+    const int nb = N / block;
+    const int n_blocks = B * Hkv * nb;
+    if (n_blocks == 0) return SPA_OK;
+    const int grid = grid_for(n_blocks, 16);
+    const uint4* k4 = reinterpret_cast<const uint4*>(K);
+#define SPA_MM_CASE(D, BL)                                                                        \
+    if (d == D && block == BL) {                                                                 \
+        SPA_CUDA_TRY(launch_pdl(block_minmax_kernel<D, BL>, dim3(grid), dim3(128), 0, st, k4,    \
+                                n_blocks, nb, N, mn, mx));                                       \
+        return SPA_OK;                                                                           \
+    }
+    SPA_MM_CASE(64, 32) SPA_MM_CASE(64, 64) SPA_MM_CASE(64, 128)
+    SPA_MM_CASE(128, 32) SPA_MM_CASE(128, 64) SPA_MM_CASE(128, 128)
+#undef SPA_MM_CASE
     return SPA_ERR_UNSUPPORTED_SHAPE;
 }
 

@@ -343,6 +343,14 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
         s = lowrank_scores(x["q_idx"][b, heads], x["Kidx"][b, g], cfg.collapse == "group", f32(cfg.score_scale))
         s = s.reshape(-1)                 # one row: the group's shared scores, or the one head's
         ranked = as_ranked(s)
+    elif cfg.score == "minmax":          # min-max page score (min/max pooling)
+        mn, mx = block_minmax(x["K"][b, g], cfg.block)
+        s = minmax_scores(x["q"][b, heads], mn, mx, f32(cfg.score_scale), True)
+        ranked = as_ranked(s)
+    elif cfg.score == "mean":            # mean-pooling block score
+        mean, _ = stats if stats is not None else block_stats(x["K"][b, g], cfg.block)
+        s = mean_scores(x["q"][b, heads], mean, f32(cfg.score_scale), True)
+        ranked = as_ranked(s)
     else:
         mean, var = stats if stats is not None else block_stats(x["K"][b, g], cfg.block)
         t = taylor_scores(x["q"][b, heads], mean, var, f32(cfg.score_scale), True)
