@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--local-fraction", type=float, default=0.0,
                     help="head-wise routing: this fraction of every sequence's units is local (sink + window)")
+    ap.add_argument("--score", choices=["taylor", "minmax", "mean"], default=None,
+                    help="block score of a block-scored workload (c3): second-order Taylor (its own), the min-max "
+                         "page score or the mean-pooling score")
     ap.add_argument("--rla", action="store_true",
                     help="add the residual linear attention over the rows outside each support (SPLA)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -65,6 +68,15 @@ def parse():
     if a.warmup is None:
         a.warmup = 50 if a.impl == "spa" else 3
     return a
+
+
+def with_score(cfg, score):
+    """The workload with another block score (block-scored workloads only)."""
+    if score is None or score == cfg.score:
+        return cfg
+    if cfg.score == "lowrank":
+        raise SystemExit(f"--score applies to block-scored workloads; {cfg.name} uses low-rank index scores")
+    return cfg.with_(score=score)
 
 
 def workload_desc(cfg):
@@ -173,7 +185,7 @@ def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cfg = DECODE_CONFIGS[a.config]
+    cfg = with_score(DECODE_CONFIGS[a.config], a.score)
     import oracle
 
     x = decode_inputs(cfg)
@@ -219,7 +231,7 @@ def run_spa(a):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    base = DECODE_CONFIGS[a.config]
+    base = with_score(DECODE_CONFIGS[a.config], a.score)
     # weak scaling: every rank holds its own B sequences (a shard of a global batch of world*B)
     cfg_global = global_config(base, world)
     t = time.perf_counter()
@@ -232,7 +244,9 @@ def run_spa(a):
     cfg = base
     lowrank = cfg.score == "lowrank"
     dq, dK, dV = up(x["q"]), up(x["K"]), up(x["V"])
-    kw = dict(score_kind=spa.SPA_SCORE_LOWRANK if lowrank else spa.SPA_SCORE_TAYLOR_BLOCK,
+    kinds = {"lowrank": spa.SPA_SCORE_LOWRANK, "taylor": spa.SPA_SCORE_TAYLOR_BLOCK,
+             "minmax": spa.SPA_SCORE_MINMAX_BLOCK, "mean": spa.SPA_SCORE_MEAN_BLOCK}
+    kw = dict(score_kind=kinds[cfg.score],
               select_kind=spa.SPA_SELECT_TOPP if cfg.select == "topp" else spa.SPA_SELECT_TOPK,
               collapse=spa.SPA_COLLAPSE_GROUP_MEAN if cfg.collapse == "group" else spa.SPA_COLLAPSE_NONE,
               q=dq, K=dK, V=dV, block=cfg.block, score_scale=float(np.float32(cfg.score_scale)),
@@ -242,7 +256,13 @@ def run_spa(a):
         dqi, dKi = up(x["q_idx"]), up(x["Kidx"])
         kw.update(q_idx=dqi, Kidx=dKi)
     else:
-        bm, bv = spa.block_stats(dK, cfg.block)      # once per filled block, off the per-step path
+        # block statistics: once per filled block, off the per-step path
+        if cfg.score == "minmax":
+            bm, bv = spa.block_minmax(dK, cfg.block)
+        else:
+            bm, bv = spa.block_stats(dK, cfg.block)
+            if cfg.score == "mean":
+                bv = None
         kw.update(bmean=bm, bvar=bv)
     # head-wise routing: the first round(f * units per sequence) units of every sequence are local
     units_per_seq = cfg.U // cfg.B
@@ -331,9 +351,10 @@ def run_spa(a):
         if cfg.collapse == "group":      # a local unit's index keys are not read
             score_bytes -= int(local_np.sum()) * cfg.N * cfg.r * 2
     else:
-        score_bytes = 2 * cfg.B * cfg.Hkv * M * d * 4 + cfg.B * cfg.Hq * d * 2
+        n_stats = 1 if cfg.score == "mean" else 2     # (mean) or (mean, var) / (min, max)
+        score_bytes = n_stats * cfg.B * cfg.Hkv * M * d * 4 + cfg.B * cfg.Hq * d * 2
         if cfg.collapse == "group":      # a local unit's block statistics are not read
-            score_bytes -= int(local_np.sum()) * 2 * M * d * 4
+            score_bytes -= int(local_np.sum()) * n_stats * M * d * 4
     attend_bytes = rows * KV_ROW_BYTES(d) + 2 * cfg.B * cfg.Hq * d * 2
     if rla is not None:      # the state (S, z) of every kv head and gamma, read once
         attend_bytes += cfg.B * cfg.Hkv * (d * d + d) * 4 + cfg.Hq * d * 4
