@@ -77,3 +77,44 @@ def test_decode_validation():
     assert need > 1000 * 4
     assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(16), 10, None) == _abi.SPA_ERR_WORKSPACE_TOO_SMALL
     assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(16), need, None) == _abi.SPA_ERR_INVALID_ARG
+
+
+def test_rla_and_block_proxy_validation():
+    L = spa.lib()
+    P = ctypes.c_void_p(16)   # never dereferenced: every call below returns before any device work
+    INV, UNS, OK = _abi.SPA_ERR_INVALID_ARG, _abi.SPA_ERR_UNSUPPORTED_SHAPE, _abi.SPA_OK
+    # spa_rla_state: row range inside [0, N], d in {64, 128}, 16-byte alignment; empty range is a no-op
+    assert L.spa_rla_state(P, P, 1, 1, 100, 128, 5, 4, P, P, None) == INV
+    assert L.spa_rla_state(P, P, 1, 1, 100, 128, 0, 101, P, P, None) == INV
+    assert L.spa_rla_state(P, P, 1, 1, 100, 128, -1, 4, P, P, None) == INV
+    assert L.spa_rla_state(None, None, 1, 1, 100, 128, 7, 7, None, None, None) == OK
+    assert L.spa_rla_state(P, P, 1, 1, 100, 96, 0, 10, P, P, None) == UNS
+    assert L.spa_rla_state(P, P, 1, 1, 100, 128, 0, 10, ctypes.c_void_p(20), P, None) == UNS
+    assert L.spa_rla_state(P, None, 1, 1, 100, 128, 0, 10, P, P, None) == INV
+    # spa_block_minmax: shapes as spa_block_stats
+    assert L.spa_block_minmax(P, 1, 1, 128, 96, 64, P, P, None) == UNS
+    assert L.spa_block_minmax(P, 1, 1, 128, 128, 48, P, P, None) == UNS
+    assert L.spa_block_minmax(None, 0, 1, 128, 128, 64, None, None, None) == OK
+    # min-max scores need both statistics and a positive scale; the mean score needs the means
+    assert L.spa_index_scores(_abi.SPA_SCORE_MINMAX_BLOCK, P, P, P, 1, 4, 1, 10, 128, 0, ctypes.c_float(0.0), P,
+                              None) == INV
+    assert L.spa_index_scores(_abi.SPA_SCORE_MINMAX_BLOCK, P, P, None, 1, 4, 1, 10, 128, 0, ctypes.c_float(1.0), P,
+                              None) == INV
+    assert L.spa_index_scores(_abi.SPA_SCORE_MEAN_BLOCK, P, P, None, 1, 4, 1, 10, 96, 0, ctypes.c_float(1.0), P,
+                              None) == UNS
+    assert L.spa_index_scores(7, P, P, P, 1, 4, 1, 10, 128, 0, ctypes.c_float(1.0), P, None) == INV
+
+
+def test_decode_rla_fields_validation():
+    a = _abi.SpaDecodeArgs()
+    a.score_kind, a.select_kind, a.collapse = _abi.SPA_SCORE_LOWRANK, _abi.SPA_SELECT_TOPP, 1
+    a.B, a.Hq, a.Hkv, a.N, a.d, a.r, a.block = 1, 8, 1, 1000, 128, 16, 1
+    a.topp, a.cap = 0.9, 1000
+    P = 16
+    a.q = a.q_idx = a.K = a.V = a.Kidx = a.idx = a.count = a.out = P
+    a.rla_state, a.rla_z, a.rla_gamma, a.rla_eps = P, None, P, 1e-6     # z missing
+    L = spa.lib()
+    need = L.spa_decode_workspace_bytes(ctypes.byref(a))
+    assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(P), need, None) == _abi.SPA_ERR_INVALID_ARG
+    a.rla_z, a.rla_eps = P, -1.0                                          # negative epsilon
+    assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(P), need, None) == _abi.SPA_ERR_INVALID_ARG
