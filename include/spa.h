@@ -66,6 +66,10 @@ typedef enum spa_score_kind {
     SPA_SCORE_MEAN_BLOCK = 3    /* s_b = mean_h q'_h . mean_b (first-order, mean pooling) */
 } spa_score_kind;
 
+/* OR-ed into a block score kind of spa_index_scores: the statistics are bf16 bit patterns
+ * (spa_block_stats_bf16 / spa_block_minmax_bf16) instead of fp32; half the bytes. */
+#define SPA_STATS_BF16 0x100
+
 typedef enum spa_select_kind {
     SPA_SELECT_TOPK = 0,
     SPA_SELECT_TOPP = 1
@@ -77,8 +81,8 @@ const char* spa_status_string(int status);
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
 const char* spa_last_cuda_error(void);
 
-/* ABI version of this header: 4 (spa_decode_args gained local_units in 2, the RLA fields in 3;
- * the min-max and mean block scores and spa_block_minmax came in 4). */
+/* ABI version of this header: 5 (spa_decode_args gained local_units in 2, the RLA fields in 3;
+ * the min-max and mean block scores and spa_block_minmax came in 4; bf16 statistics in 5). */
 int spa_abi_version(void);
 
 /* ------------------------------------------------------------------------------------
@@ -99,6 +103,14 @@ spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int 
  *   spa_block_stats. */
 spa_status spa_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block,
                             float* mn, float* mx, void* stream);
+
+/* The same statistics stored as bf16 bit patterns (round to nearest even of the fp32 values;
+ * the variance is taken about the fp32 mean; minima and maxima are exact), for scoring with
+ * SPA_STATS_BF16 at half the bytes. */
+spa_status spa_block_stats_bf16(const uint16_t* K, int B, int Hkv, int N, int d, int block,
+                                uint16_t* mean, uint16_t* var, void* stream);
+spa_status spa_block_minmax_bf16(const uint16_t* K, int B, int Hkv, int N, int d, int block,
+                                 uint16_t* mn, uint16_t* mx, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * a2/a3. Index scores, one row of M scores per selection unit.
@@ -121,9 +133,10 @@ spa_status spa_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int
  *   over the G heads under GROUP_MEAN.
  * kind = SPA_SCORE_MEAN_BLOCK: keys = block means, var NULL (not read);
  *   s[u, b] = q' . mean_b; averaged over the G heads under GROUP_MEAN.
+ * kind | SPA_STATS_BF16 (block kinds only): keys and var are bf16 bit patterns.
  * scores [U, M] fp32 out.  G = Hq / Hkv must be an integer, G <= 16.
  */
-spa_status spa_index_scores(int kind, const void* q, const void* keys, const float* var,
+spa_status spa_index_scores(int kind, const void* q, const void* keys, const void* var,
                             int B, int Hq, int Hkv, int M, int dim, int collapse, float scale,
                             float* scores, void* stream);
 
@@ -232,8 +245,8 @@ typedef struct spa_decode_args {
     const uint16_t* K;       /* [B, Hkv, N, d] */
     const uint16_t* V;       /* [B, Hkv, N, d] */
     const uint16_t* Kidx;    /* [B, Hkv, N, r] (LOWRANK) */
-    const float* bmean;      /* [B, Hkv, N / block, d]: TAYLOR and MEAN block means; MINMAX block minima */
-    const float* bvar;       /* [B, Hkv, N / block, d]: TAYLOR block variances; MINMAX block maxima; MEAN unused */
+    const void* bmean;       /* [B, Hkv, N / block, d]: TAYLOR and MEAN block means; MINMAX block minima (fp32, or bf16 with stats_bf16) */
+    const void* bvar;        /* [B, Hkv, N / block, d]: TAYLOR block variances; MINMAX block maxima; MEAN unused */
     float score_scale;       /* LOWRANK: index-score scale; block kinds: q' = score_scale * q */
     float sm_scale;          /* softmax scale of the exact attention */
     int topk;                /* SPA_SELECT_TOPK */
@@ -272,6 +285,7 @@ typedef struct spa_decode_args {
     const float* rla_z;
     const float* rla_gamma;
     float rla_eps;           /* RMSNorm epsilon, >= 0 */
+    int stats_bf16;          /* block kinds: bmean / bvar are bf16 bit patterns (spa_block_*_bf16), else fp32 */
 } spa_decode_args;
 
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream);

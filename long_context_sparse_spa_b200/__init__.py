@@ -18,13 +18,13 @@ from typing import Optional, Tuple
 import torch
 
 from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK, SPA_SCORE_MEAN_BLOCK,
-                   SPA_SCORE_MINMAX_BLOCK, SPA_SCORE_TAYLOR_BLOCK, SPA_SELECT_TOPK, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
+                   SPA_SCORE_MINMAX_BLOCK, SPA_SCORE_TAYLOR_BLOCK, SPA_SELECT_TOPK, SPA_STATS_BF16, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
 
 __all__ = [
     "SpaError", "lib", "lib_path", "block_stats", "index_scores", "select_topk", "select_topp", "sparse_attend",
     "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "prefill", "PrefillPlan", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
     "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SCORE_MINMAX_BLOCK", "SPA_SCORE_MEAN_BLOCK",
-    "SPA_SELECT_TOPK", "SPA_SELECT_TOPP", "block_minmax", "rla_state",
+    "SPA_SELECT_TOPK", "SPA_SELECT_TOPP", "SPA_STATS_BF16", "block_minmax", "rla_state",
 ]
 
 
@@ -59,25 +59,27 @@ def read_device_status(ws: torch.Tensor, reset: bool = True) -> int:
 
 
 # ----------------------------------------------------------------------------- a1
-def block_stats(K: torch.Tensor, block: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
-    """K [B, Hkv, N, d] bf16 -> (mean, var) [B, Hkv, N // block, d] fp32."""
+def block_stats(K: torch.Tensor, block: int = 64, bf16: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K [B, Hkv, N, d] bf16 -> (mean, var) [B, Hkv, N // block, d], fp32 (or bf16 storage)."""
     _need(K, torch.bfloat16, "K")
     B, Hkv, N, d = K.shape
     nb = N // block
-    mean = torch.empty((B, Hkv, nb, d), dtype=torch.float32, device=K.device)
+    mean = torch.empty((B, Hkv, nb, d), dtype=torch.bfloat16 if bf16 else torch.float32, device=K.device)
     var = torch.empty_like(mean)
-    check(lib().spa_block_stats(_ptr(K), B, Hkv, N, d, block, _ptr(mean), _ptr(var), _stream()))
+    fn = lib().spa_block_stats_bf16 if bf16 else lib().spa_block_stats
+    check(fn(_ptr(K), B, Hkv, N, d, block, _ptr(mean), _ptr(var), _stream()))
     return mean, var
 
 
-def block_minmax(K: torch.Tensor, block: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
-    """K [B, Hkv, N, d] bf16 -> per-block channel (min, max) [B, Hkv, N // block, d] fp32."""
+def block_minmax(K: torch.Tensor, block: int = 64, bf16: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K [B, Hkv, N, d] bf16 -> per-block channel (min, max) [B, Hkv, N // block, d], fp32 (or bf16)."""
     _need(K, torch.bfloat16, "K")
     B, Hkv, N, d = K.shape
     nb = N // block
-    mn = torch.empty((B, Hkv, nb, d), dtype=torch.float32, device=K.device)
+    mn = torch.empty((B, Hkv, nb, d), dtype=torch.bfloat16 if bf16 else torch.float32, device=K.device)
     mx = torch.empty_like(mn)
-    check(lib().spa_block_minmax(_ptr(K), B, Hkv, N, d, block, _ptr(mn), _ptr(mx), _stream()))
+    fn = lib().spa_block_minmax_bf16 if bf16 else lib().spa_block_minmax
+    check(fn(_ptr(K), B, Hkv, N, d, block, _ptr(mn), _ptr(mx), _stream()))
     return mn, mx
 
 
@@ -93,9 +95,10 @@ def index_scores(kind: int, q: torch.Tensor, keys: torch.Tensor, var: Optional[t
     if kind == SPA_SCORE_LOWRANK:
         _need(keys, torch.bfloat16, "keys")
     else:
-        _need(keys, torch.float32, "keys")
-        if kind != SPA_SCORE_MEAN_BLOCK:
-            _need(var, torch.float32, "var")
+        sdt = torch.bfloat16 if kind & SPA_STATS_BF16 else torch.float32
+        _need(keys, sdt, "keys")
+        if kind & ~SPA_STATS_BF16 != SPA_SCORE_MEAN_BLOCK:
+            _need(var, sdt, "var")
     U = B * (Hkv if collapse == SPA_COLLAPSE_GROUP_MEAN else Hq)
     if out is None:
         out = torch.empty((U, M), dtype=torch.float32, device=q.device)
@@ -247,6 +250,7 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
     a.q, a.K, a.V = _ptr(q), _ptr(K), _ptr(V)
     a.q_idx, a.Kidx = _ptr(q_idx), _ptr(Kidx)
     a.bmean, a.bvar = _ptr(bmean), _ptr(bvar)
+    a.stats_bf16 = int(bmean is not None and bmean.dtype == torch.bfloat16)
     a.score_scale, a.sm_scale = score_scale, sm_scale
     a.topk, a.topp, a.sink, a.window = topk, topp, sink, window
     a.idx, a.count, a.cap = _ptr(idx), _ptr(count), cap

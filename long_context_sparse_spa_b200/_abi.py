@@ -7,7 +7,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(HERE, "libspa.so")
 
-ABI_VERSION = 4   # spa_abi_version() of the library these declarations describe
+ABI_VERSION = 5   # spa_abi_version() of the library these declarations describe
 
 SPA_OK = 0
 SPA_ERR_INVALID_ARG = 1
@@ -23,6 +23,7 @@ SPA_SCORE_LOWRANK = 0
 SPA_SCORE_TAYLOR_BLOCK = 1
 SPA_SCORE_MINMAX_BLOCK = 2
 SPA_SCORE_MEAN_BLOCK = 3
+SPA_STATS_BF16 = 0x100
 SPA_SELECT_TOPK = 0
 SPA_SELECT_TOPP = 1
 SPA_SELECT_STATIC_MAX_UNITS = 16
@@ -48,6 +49,7 @@ class SpaDecodeArgs(ctypes.Structure):
         ("out", _p), ("out_f32", _p), ("lse", _p),
         ("local_units", _p),
         ("rla_state", _p), ("rla_z", _p), ("rla_gamma", _p), ("rla_eps", _f),
+        ("stats_bf16", _i),
     ]
 
 
@@ -75,6 +77,8 @@ SIGNATURES = {
     "spa_select_workspace_bytes": (_sz, [_i, _i]),
     "spa_select_topp_static": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p]),
     "spa_block_minmax": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
+    "spa_block_stats_bf16": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
+    "spa_block_minmax_bf16": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_rla_state": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_sparse_attend": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "spa_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),

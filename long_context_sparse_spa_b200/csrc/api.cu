@@ -73,26 +73,53 @@ const char* spa_status_string(int s) {
 
 const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
-int spa_abi_version(void) { return 4; }
+int spa_abi_version(void) { return 5; }
+
+// shared checks of the block-statistics entries; SPA_OK with *noop set when there is nothing to do
+static spa_status check_stats_args(const uint16_t* K, int B, int Hkv, int N, int d, int block, const void* a,
+                                   const void* b, bool* noop) {
+    *noop = false;
+    if (B < 0 || Hkv <= 0 || N < 0 || block <= 0) return SPA_ERR_INVALID_ARG;
+    if (B == 0 || N / block == 0) {
+        *noop = true;
+        return SPA_OK;
+    }
+    if (!K || !a || !b) return SPA_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || (block != 32 && block != 64 && block != 128)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(K) || !aligned16(a) || !aligned16(b)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    return SPA_OK;
+}
 
 spa_status spa_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean, float* var,
                            void* stream) {
-    if (B < 0 || Hkv <= 0 || N < 0 || block <= 0) return SPA_ERR_INVALID_ARG;
-    if (B == 0 || N / block == 0) return SPA_OK;
-    if (!K || !mean || !var) return SPA_ERR_INVALID_ARG;
-    if ((d != 64 && d != 128) || (block != 32 && block != 64 && block != 128)) return SPA_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(K) || !aligned16(mean) || !aligned16(var)) return SPA_ERR_UNSUPPORTED_SHAPE;
-    return launch_block_stats(K, B, Hkv, N, d, block, mean, var, static_cast<cudaStream_t>(stream));
+    bool noop;
+    const spa_status s = check_stats_args(K, B, Hkv, N, d, block, mean, var, &noop);
+    if (s != SPA_OK || noop) return s;
+    return launch_block_stats(K, B, Hkv, N, d, block, mean, var, false, static_cast<cudaStream_t>(stream));
+}
+
+spa_status spa_block_stats_bf16(const uint16_t* K, int B, int Hkv, int N, int d, int block, uint16_t* mean,
+                                uint16_t* var, void* stream) {
+    bool noop;
+    const spa_status s = check_stats_args(K, B, Hkv, N, d, block, mean, var, &noop);
+    if (s != SPA_OK || noop) return s;
+    return launch_block_stats(K, B, Hkv, N, d, block, mean, var, true, static_cast<cudaStream_t>(stream));
 }
 
 spa_status spa_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mn, float* mx,
                             void* stream) {
-    if (B < 0 || Hkv <= 0 || N < 0 || block <= 0) return SPA_ERR_INVALID_ARG;
-    if (B == 0 || N / block == 0) return SPA_OK;
-    if (!K || !mn || !mx) return SPA_ERR_INVALID_ARG;
-    if ((d != 64 && d != 128) || (block != 32 && block != 64 && block != 128)) return SPA_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(K) || !aligned16(mn) || !aligned16(mx)) return SPA_ERR_UNSUPPORTED_SHAPE;
-    return launch_block_minmax(K, B, Hkv, N, d, block, mn, mx, static_cast<cudaStream_t>(stream));
+    bool noop;
+    const spa_status s = check_stats_args(K, B, Hkv, N, d, block, mn, mx, &noop);
+    if (s != SPA_OK || noop) return s;
+    return launch_block_minmax(K, B, Hkv, N, d, block, mn, mx, false, static_cast<cudaStream_t>(stream));
+}
+
+spa_status spa_block_minmax_bf16(const uint16_t* K, int B, int Hkv, int N, int d, int block, uint16_t* mn,
+                                 uint16_t* mx, void* stream) {
+    bool noop;
+    const spa_status s = check_stats_args(K, B, Hkv, N, d, block, mn, mx, &noop);
+    if (s != SPA_OK || noop) return s;
+    return launch_block_minmax(K, B, Hkv, N, d, block, mn, mx, true, static_cast<cudaStream_t>(stream));
 }
 
 // block score kinds other than low-rank, with their statistics' requirements
@@ -107,8 +134,11 @@ static bool is_block_kind(int kind) {
     return kind == SPA_SCORE_TAYLOR_BLOCK || kind == SPA_SCORE_MINMAX_BLOCK || kind == SPA_SCORE_MEAN_BLOCK;
 }
 
-spa_status spa_index_scores(int kind, const void* q, const void* keys, const float* var, int B, int Hq, int Hkv,
+spa_status spa_index_scores(int kind, const void* q, const void* keys, const void* var, int B, int Hq, int Hkv,
                             int M, int dim, int collapse, float scale, float* scores, void* stream) {
+    const bool stats_bf16 = (kind & SPA_STATS_BF16) != 0;
+    kind &= ~SPA_STATS_BF16;
+    if (stats_bf16 && !is_block_kind(kind)) return SPA_ERR_INVALID_ARG;
     if (bad_dims(B, Hq, Hkv) || M < 0) return SPA_ERR_INVALID_ARG;
     if (collapse != SPA_COLLAPSE_NONE && collapse != SPA_COLLAPSE_GROUP_MEAN) return SPA_ERR_INVALID_ARG;
     if (B == 0 || M == 0) return SPA_OK;
@@ -126,8 +156,8 @@ spa_status spa_index_scores(int kind, const void* q, const void* keys, const flo
         spa_status s = check_block_kind(kind, keys, var, scale);
         if (s != SPA_OK) return s;
         if (dim != 64 && dim != 128) return SPA_ERR_UNSUPPORTED_SHAPE;
-        return launch_taylor_scores(static_cast<const uint16_t*>(q), static_cast<const float*>(keys), var, B, Hq,
-                                    Hkv, M, dim, collapse, scale, scores, st, nullptr, kind);
+        return launch_taylor_scores(static_cast<const uint16_t*>(q), keys, var, B, Hq, Hkv, M, dim, collapse, scale,
+                                    scores, st, nullptr, kind, stats_bf16);
     }
     return SPA_ERR_INVALID_ARG;
 }
@@ -311,7 +341,7 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
     if ((s = mark(0)) != SPA_OK) return s;
     if (taylor) {
         s = launch_taylor_scores(a->q, a->bmean, a->bvar, a->B, a->Hq, a->Hkv, M, a->d, a->collapse,
-                                 a->score_scale, scores, st, a->local_units, a->score_kind);
+                                 a->score_scale, scores, st, a->local_units, a->score_kind, a->stats_bf16 != 0);
     } else {
         s = launch_lowrank_scores(a->q_idx, a->Kidx, a->B, a->Hq, a->Hkv, M, a->collapse, a->score_scale, scores,
                                   fused_hist ? &hist : nullptr, topp, st, a->local_units);

@@ -138,14 +138,16 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
                                  int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
                                  cudaStream_t st, const uint8_t* local = nullptr);
 // kind: SPA_SCORE_TAYLOR_BLOCK (mean, var), SPA_SCORE_MINMAX_BLOCK (min, max) or
-// SPA_SCORE_MEAN_BLOCK (mean; var not read)
-spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
+// SPA_SCORE_MEAN_BLOCK (mean; var not read); stats_bf16: the statistics are bf16, else fp32
+spa_status launch_taylor_scores(const uint16_t* q, const void* mean, const void* var, int B, int Hq, int Hkv,
                                 int M, int d, int collapse, float scale, float* scores, cudaStream_t st,
-                                const uint8_t* local = nullptr, int kind = SPA_SCORE_TAYLOR_BLOCK);
-spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean,
-                              float* var, cudaStream_t st);
-spa_status launch_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mn, float* mx,
-                               cudaStream_t st);
+                                const uint8_t* local = nullptr, int kind = SPA_SCORE_TAYLOR_BLOCK,
+                                bool stats_bf16 = false);
+// out_bf16: write the statistics as bf16 (round to nearest even), else fp32
+spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, void* mean,
+                              void* var, bool out_bf16, cudaStream_t st);
+spa_status launch_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, void* mn, void* mx,
+                               bool out_bf16, cudaStream_t st);
 
 // select.cu
 struct SelectParams {

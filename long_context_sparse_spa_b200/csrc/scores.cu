@@ -164,13 +164,25 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
 //                 the largest logit inside the block's channel box.
 //   KIND_MEAN   (mean pooling, "SPLA" 1, PBS-Attn 4): stats (mean); a_h = q'_h . mean.
 //   Under GROUP_MEAN the min-max and mean scores are averaged over the G heads.
+// SBF16: the statistics are stored as bf16 (8-byte loads of four values) instead of fp32.
 constexpr int kTyThreads = 256;
 constexpr int kTyChunk = 256;
 constexpr int KIND_TAYLOR = 0, KIND_MINMAX = 1, KIND_MEAN = 2;
 
-template <int D, int G, int KIND>
+// four statistics at position f4 (in units of four values) of a row starting at base
+template <bool SBF16>
+__device__ __forceinline__ float4 load_stats4(const void* p, size_t base, int f4) {
+    if constexpr (SBF16) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(p) + base + f4);
+        return make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+    } else {
+        return __ldg(reinterpret_cast<const float4*>(p) + base + f4);
+    }
+}
+
+template <int D, int G, int KIND, bool SBF16>
 __global__ void __launch_bounds__(kTyThreads)
-taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ mean, const float4* __restrict__ var,
+taylor_scores_kernel(const uint16_t* __restrict__ q, const void* __restrict__ mean, const void* __restrict__ var,
                      int Hq, int Hkv, int M, int collapse, float scale, float* __restrict__ scores,
                      int chunks_per_unit, int n_items, const uint8_t* __restrict__ local) {
     pdl_enter();
@@ -211,8 +223,9 @@ taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ 
                 for (int v = 0; v < kVec; ++v) {
                     // lane8 owns dims {4*(lane8 + 8*v) .. +3}: 8 lanes read 128 contiguous bytes
                     const int f4 = lane8 + 8 * v;
-                    const float4 mu = __ldg(mean + base + f4);
-                    const float4 vr = KIND == KIND_MEAN ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(var + base + f4);
+                    const float4 mu = load_stats4<SBF16>(mean, base, f4);
+                    const float4 vr = KIND == KIND_MEAN ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                                        : load_stats4<SBF16>(var, base, f4);
                     const float mus[4] = {mu.x, mu.y, mu.z, mu.w};
                     const float vrs[4] = {vr.x, vr.y, vr.z, vr.w};
 #pragma unroll
@@ -279,10 +292,21 @@ taylor_scores_kernel(const uint16_t* __restrict__ q, const float4* __restrict__ 
 // One CTA of 128 threads per 64-token (or 32/128) block at a time: thread t holds 8
 // dims (one 16-byte chunk) of BLOCK*D/1024 rows in registers, so the two passes (mean,
 // then squared deviations) read HBM once.
-template <int D, int BLOCK>
+// store one statistic: fp32, or its bf16 rounding (round to nearest even)
+template <bool OBF16>
+__device__ __forceinline__ void store_stat(void* p, size_t i, float v) {
+    if constexpr (OBF16) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        reinterpret_cast<__nv_bfloat16*>(p)[i] = h;
+    } else {
+        reinterpret_cast<float*>(p)[i] = v;
+    }
+}
+
+template <int D, int BLOCK, bool OBF16>
 __global__ void __launch_bounds__(128)
-block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, float* __restrict__ mean,
-                   float* __restrict__ var) {
+block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, void* __restrict__ mean,
+                   void* __restrict__ var) {
     pdl_enter();
     constexpr int DV = D / 8;                 // 16-byte chunks per row
     constexpr int PH = 128 / DV;              // row phases
@@ -320,8 +344,8 @@ block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, i
 #pragma unroll
             for (int p = 0; p < PH; ++p) t += red[p][threadIdx.x];
             const float m = t / float(BLOCK);
-            mu_s[threadIdx.x] = m;
-            mean[size_t(blk) * D + threadIdx.x] = m;
+            mu_s[threadIdx.x] = m;                 // the deviations use the fp32 mean
+            store_stat<OBF16>(mean, size_t(blk) * D + threadIdx.x, m);
         }
         __syncthreads();
         float mv[8];
@@ -345,7 +369,7 @@ block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, i
             float t = 0.f;
 #pragma unroll
             for (int p = 0; p < PH; ++p) t += red[p][threadIdx.x];
-            var[size_t(blk) * D + threadIdx.x] = t / float(BLOCK);
+            store_stat<OBF16>(var, size_t(blk) * D + threadIdx.x, t / float(BLOCK));
         }
         __syncthreads();
     }
@@ -353,10 +377,10 @@ block_stats_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, i
 
 // Per-block channel minimum and maximum of K (min/max pooling, "SPLA" 1): the loads of
 // block_stats_kernel, one pass, exact (bf16 values are exact in fp32).
-template <int D, int BLOCK>
+template <int D, int BLOCK, bool OBF16>
 __global__ void __launch_bounds__(128)
-block_minmax_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, float* __restrict__ mn,
-                    float* __restrict__ mx) {
+block_minmax_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, int N, void* __restrict__ mn,
+                    void* __restrict__ mx) {
     pdl_enter();
     constexpr int DV = D / 8;
     constexpr int PH = 128 / DV;
@@ -400,8 +424,8 @@ block_minmax_kernel(const uint4* __restrict__ K, int n_blocks, int nb_per_unit, 
                 l = fminf(l, rlo[p][threadIdx.x]);
                 h = fmaxf(h, rhi[p][threadIdx.x]);
             }
-            mn[size_t(blk) * D + threadIdx.x] = l;
-            mx[size_t(blk) * D + threadIdx.x] = h;
+            store_stat<OBF16>(mn, size_t(blk) * D + threadIdx.x, l);   // exact: bf16 values
+            store_stat<OBF16>(mx, size_t(blk) * D + threadIdx.x, h);
         }
         __syncthreads();
     }
@@ -444,46 +468,49 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
     return SPA_OK;
 }
 
-spa_status launch_taylor_scores(const uint16_t* q, const float* mean, const float* var, int B, int Hq, int Hkv,
+spa_status launch_taylor_scores(const uint16_t* q, const void* mean, const void* var, int B, int Hq, int Hkv,
                                 int M, int d, int collapse, float scale, float* scores, cudaStream_t st,
-                                const uint8_t* local, int kind) {
+                                const uint8_t* local, int kind, bool stats_bf16) {
     const int G = Hq / Hkv;
     const int chunks = (M + kTyChunk - 1) / kTyChunk;
     const int items = B * Hkv * chunks;
     const int grid = grid_for(items, 8);
-    const float4* m4 = reinterpret_cast<const float4*>(mean);
-    const float4* v4 = reinterpret_cast<const float4*>(var);
-#define SPA_TY_CASE(D, GG)                                                                                   \
-    if (d == D && G == GG) {                                                                                \
-        if (kind == SPA_SCORE_MINMAX_BLOCK)                                                                 \
-            SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KIND_MINMAX>, dim3(grid), dim3(kTyThreads), 0, st, \
-                                    q, m4, v4, Hq, Hkv, M, collapse, scale, scores, chunks, items, local));       \
-        else if (kind == SPA_SCORE_MEAN_BLOCK)                                                              \
-            SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KIND_MEAN>, dim3(grid), dim3(kTyThreads), 0, st,   \
-                                    q, m4, v4, Hq, Hkv, M, collapse, scale, scores, chunks, items, local));       \
-        else                                                                                                \
-            SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KIND_TAYLOR>, dim3(grid), dim3(kTyThreads), 0, st, \
-                                    q, m4, v4, Hq, Hkv, M, collapse, scale, scores, chunks, items, local));       \
-        return SPA_OK;                                                                                      \
+#define SPA_TY_LAUNCH(D, GG, KD, SB)                                                                          \
+    SPA_CUDA_TRY(launch_pdl(taylor_scores_kernel<D, GG, KD, SB>, dim3(grid), dim3(kTyThreads), 0, st, q, mean, var, \
+                            Hq, Hkv, M, collapse, scale, scores, chunks, items, local))
+#define SPA_TY_KIND(D, GG, SB)                                                                                \
+    if (kind == SPA_SCORE_MINMAX_BLOCK) SPA_TY_LAUNCH(D, GG, KIND_MINMAX, SB);                                 \
+    else if (kind == SPA_SCORE_MEAN_BLOCK) SPA_TY_LAUNCH(D, GG, KIND_MEAN, SB);                                \
+    else SPA_TY_LAUNCH(D, GG, KIND_TAYLOR, SB);
+#define SPA_TY_CASE(D, GG)                                                                                    \
+    if (d == D && G == GG) {                                                                                 \
+        if (stats_bf16) { SPA_TY_KIND(D, GG, true) } else { SPA_TY_KIND(D, GG, false) }                       \
+        return SPA_OK;                                                                                       \
     }
     SPA_TY_CASE(64, 1) SPA_TY_CASE(64, 2) SPA_TY_CASE(64, 4) SPA_TY_CASE(64, 8) SPA_TY_CASE(64, 16)
     SPA_TY_CASE(128, 1) SPA_TY_CASE(128, 2) SPA_TY_CASE(128, 4) SPA_TY_CASE(128, 8) SPA_TY_CASE(128, 16)
 #undef SPA_TY_CASE
+#undef SPA_TY_KIND
+#undef SPA_TY_LAUNCH
     return SPA_ERR_UNSUPPORTED_SHAPE;
 }
 
-spa_status launch_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mn, float* mx,
-                               cudaStream_t st) {
+spa_status launch_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, int block, void* mn, void* mx,
+                               bool out_bf16, cudaStream_t st) {
     const int nb = N / block;
     const int n_blocks = B * Hkv * nb;
     if (n_blocks == 0) return SPA_OK;
     const int grid = grid_for(n_blocks, 16);
     const uint4* k4 = reinterpret_cast<const uint4*>(K);
-#define SPA_MM_CASE(D, BL)                                                                        \
-    if (d == D && block == BL) {                                                                 \
-        SPA_CUDA_TRY(launch_pdl(block_minmax_kernel<D, BL>, dim3(grid), dim3(128), 0, st, k4,    \
-                                n_blocks, nb, N, mn, mx));                                       \
-        return SPA_OK;                                                                           \
+#define SPA_MM_CASE(D, BL)                                                                              \
+    if (d == D && block == BL) {                                                                       \
+        if (out_bf16)                                                                                  \
+            SPA_CUDA_TRY(launch_pdl(block_minmax_kernel<D, BL, true>, dim3(grid), dim3(128), 0, st, k4,  \
+                                    n_blocks, nb, N, mn, mx));                                         \
+        else                                                                                           \
+            SPA_CUDA_TRY(launch_pdl(block_minmax_kernel<D, BL, false>, dim3(grid), dim3(128), 0, st, k4, \
+                                    n_blocks, nb, N, mn, mx));                                         \
+        return SPA_OK;                                                                                 \
     }
     SPA_MM_CASE(64, 32) SPA_MM_CASE(64, 64) SPA_MM_CASE(64, 128)
     SPA_MM_CASE(128, 32) SPA_MM_CASE(128, 64) SPA_MM_CASE(128, 128)
@@ -491,18 +518,22 @@ spa_status launch_block_minmax(const uint16_t* K, int B, int Hkv, int N, int d, 
     return SPA_ERR_UNSUPPORTED_SHAPE;
 }
 
-spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, float* mean,
-                              float* var, cudaStream_t st) {
+spa_status launch_block_stats(const uint16_t* K, int B, int Hkv, int N, int d, int block, void* mean,
+                              void* var, bool out_bf16, cudaStream_t st) {
     const int nb = N / block;
     const int n_blocks = B * Hkv * nb;
     if (n_blocks == 0) return SPA_OK;
     const int grid = grid_for(n_blocks, 16);
     const uint4* k4 = reinterpret_cast<const uint4*>(K);
-#define SPA_BS_CASE(D, BL)                                                                       \
-    if (d == D && block == BL) {                                                                \
-        SPA_CUDA_TRY(launch_pdl(block_stats_kernel<D, BL>, dim3(grid), dim3(128), 0, st, k4,    \
-                                n_blocks, nb, N, mean, var));                                   \
-        return SPA_OK;                                                                          \
+#define SPA_BS_CASE(D, BL)                                                                              \
+    if (d == D && block == BL) {                                                                       \
+        if (out_bf16)                                                                                  \
+            SPA_CUDA_TRY(launch_pdl(block_stats_kernel<D, BL, true>, dim3(grid), dim3(128), 0, st, k4,   \
+                                    n_blocks, nb, N, mean, var));                                      \
+        else                                                                                           \
+            SPA_CUDA_TRY(launch_pdl(block_stats_kernel<D, BL, false>, dim3(grid), dim3(128), 0, st, k4,  \
+                                    n_blocks, nb, N, mean, var));                                      \
+        return SPA_OK;                                                                                 \
     }
     SPA_BS_CASE(64, 32) SPA_BS_CASE(64, 64) SPA_BS_CASE(64, 128)
     SPA_BS_CASE(128, 32) SPA_BS_CASE(128, 64) SPA_BS_CASE(128, 128)

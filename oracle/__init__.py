@@ -61,7 +61,8 @@ def lib() -> ctypes.CDLL:
         L.orc_block_minmax.argtypes = [_p, _i64, _int, _int, _p, _p]
         L.orc_minmax_scores.argtypes = [_p, _int, _p, _p, _i64, _int, _dbl, _int, _p]
         L.orc_mean_scores.argtypes = [_p, _int, _p, _i64, _int, _dbl, _int, _p]
-        assert L.orc_abi_version() == 4, "stale oracle library; rebuild it"
+        L.orc_round_bf16.argtypes = [_p, _i64, _p]
+        assert L.orc_abi_version() == 5, "stale oracle library; rebuild it"
         _LIB = L
     return _LIB
 
@@ -108,6 +109,20 @@ def taylor_scores(q: np.ndarray, mean: np.ndarray, var: np.ndarray, scale: float
     out = np.empty(nb if collapse else (G, nb))
     lib().orc_taylor_scores(_ptr(q), G, _ptr(mean), _ptr(var), nb, d, float(scale), int(collapse), _ptr(out))
     return out
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even of float64 values to bf16 bit patterns (uint16), directly from
+    double: the storage of block statistics in bf16."""
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, np.uint16)
+    lib().orc_round_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact)."""
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def block_minmax(K: np.ndarray, block: int) -> Tuple[np.ndarray, np.ndarray]:
@@ -344,15 +359,15 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
         s = s.reshape(-1)                 # one row: the group's shared scores, or the one head's
         ranked = as_ranked(s)
     elif cfg.score == "minmax":          # min-max page score (min/max pooling)
-        mn, mx = block_minmax(x["K"][b, g], cfg.block)
+        mn, mx = _stored(cfg, *block_minmax(x["K"][b, g], cfg.block))
         s = minmax_scores(x["q"][b, heads], mn, mx, f32(cfg.score_scale), True)
         ranked = as_ranked(s)
     elif cfg.score == "mean":            # mean-pooling block score
-        mean, _ = stats if stats is not None else block_stats(x["K"][b, g], cfg.block)
+        mean, _ = _stored(cfg, *(stats if stats is not None else block_stats(x["K"][b, g], cfg.block)))
         s = mean_scores(x["q"][b, heads], mean, f32(cfg.score_scale), True)
         ranked = as_ranked(s)
     else:
-        mean, var = stats if stats is not None else block_stats(x["K"][b, g], cfg.block)
+        mean, var = _stored(cfg, *(stats if stats is not None else block_stats(x["K"][b, g], cfg.block)))
         t = taylor_scores(x["q"][b, heads], mean, var, f32(cfg.score_scale), True)
         s = t
         ranked = as_ranked(np.log(t))
@@ -373,6 +388,14 @@ def decode_unit(cfg, x: Dict[str, np.ndarray], u: int, stats: Optional[Tuple[np.
         res["lse"] = lse
         _add_rla(cfg, x, res, heads, rla)
     return res
+
+
+def _stored(cfg, *stats: np.ndarray) -> Tuple[np.ndarray, ...]:
+    """Block statistics as the workload stores them: as computed, or rounded to bf16
+    (round to nearest even) and widened back."""
+    if getattr(cfg, "stats", "f32") == "bf16":
+        return tuple(widen_bf16(round_bf16(a)) for a in stats)
+    return stats
 
 
 def _add_rla(cfg, x: Dict[str, np.ndarray], res: Dict[str, object], heads: slice,

@@ -100,7 +100,7 @@ int64_t emit_ascending(const std::vector<char>& keep, int32_t* idx) {
 
 extern "C" {
 
-int orc_abi_version() { return 4; }
+int orc_abi_version() { return 5; }
 
 // a1 -- per-block mean and diagonal (population) variance of K [SPLA-2.1].
 // K: [N, d] bf16 of one (batch, kv head); only the nb = N / block full blocks count.
@@ -586,6 +586,30 @@ void orc_mean_scores(const uint16_t* q, int G, const double* mean, int64_t nb, i
             if (collapse) acc += s; else out[h * nb + b] = s;
         }
         if (collapse) out[b] = acc / G;
+    }
+}
+
+// ---------------------------------------------------------------- bf16 storage
+// Round-to-nearest-even of doubles to bf16 bit patterns (8 significant bits), directly from
+// double, for statistics stored in bf16.  Finite inputs within the bf16 range.
+void orc_round_bf16(const double* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) {
+        const double v = x[i];
+        if (v == 0.0) {
+            out[i] = std::signbit(v) ? 0x8000u : 0u;
+            continue;
+        }
+        int e;
+        std::frexp(std::fabs(v), &e);                 // |v| = m * 2^e, m in [0.5, 1)
+        const double ulp = std::ldexp(1.0, std::max(e - 8, -133));   // spacing of bf16 values near |v|
+        const double q = std::fabs(v) / ulp;          // exact: a power-of-two scaling
+        double r = std::floor(q);
+        const double frac = q - r;
+        if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) r += 1.0;
+        const float f = static_cast<float>(std::copysign(r * ulp, v));   // exact in binary32
+        uint32_t u;
+        std::memcpy(&u, &f, sizeof u);
+        out[i] = static_cast<uint16_t>(u >> 16);
     }
 }
 

@@ -66,6 +66,7 @@ class DecodeConfig:
     lowfreq_amp: float = 0.0
     lowfreq_rank: int = 0
     needle_amp: float = 0.0
+    stats: str = "f32"    # storage of block statistics: "f32" or "bf16"
 
     @property
     def G(self) -> int:

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported_and_bound():
 
 def test_status_strings_and_version():
     L = spa.lib()
-    assert L.spa_abi_version() == 4 == _abi.ABI_VERSION
+    assert L.spa_abi_version() == 5 == _abi.ABI_VERSION
     assert L.spa_status_string(_abi.SPA_ERR_CAPACITY) == b"SPA_ERR_CAPACITY"
     assert L.spa_status_string(99) == b"SPA_ERR_UNKNOWN"
 

@@ -66,3 +66,32 @@ def test_mean_score_is_the_zero_variance_taylor_exponent_and_collapses_linearly(
         np.testing.assert_allclose(per_head[h], np.log(t), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(oracle.mean_scores(q, mean, scale, True), scale * _f(q).mean(0) @ mean.T,
                                rtol=1e-12, atol=1e-14)
+
+
+def _nearest_even_bf16(x):
+    """Brute force: the bf16 pattern nearest to x among the neighbours of its float32
+    truncation, ties to the even pattern."""
+    t = int(np.array([x], np.float32).view(np.uint32)[0] >> 16)
+    best = None
+    for c in (t - 1, t, t + 1, t + 2):
+        v = oracle.widen_bf16(np.array([c & 0xFFFF], np.uint16))[0]
+        key = (abs(x - v), c & 1)
+        if best is None or key < best[0]:
+            best = (key, c & 0xFFFF)
+    return best[1]
+
+
+def test_round_bf16_is_nearest_even_from_double():
+    rng = np.random.default_rng(8)
+    xs = np.concatenate([rng.standard_normal(400) * 10.0 ** rng.integers(-6, 6, 400),
+                         rng.uniform(0, 1e-3, 50)])
+    # exact halfway points between adjacent bf16 values, and just beside them
+    base = oracle.round_bf16(rng.uniform(0.1, 100, 60))
+    lo, hi = oracle.widen_bf16(base), oracle.widen_bf16(base + 1)
+    mid = (lo + hi) / 2
+    xs = np.concatenate([xs, mid, np.nextafter(mid, 0), np.nextafter(mid, np.inf), -mid])
+    got = oracle.round_bf16(xs)
+    want = np.array([_nearest_even_bf16(abs(x)) | (0x8000 if x < 0 else 0) for x in xs], np.uint16)
+    np.testing.assert_array_equal(got, want)
+    halfway = got[450:510]
+    assert (halfway & 1 == 0).all()            # ties went to the even pattern
