@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--score", choices=["taylor", "minmax", "mean"], default=None,
                     help="block score of a block-scored workload (c3): second-order Taylor (its own), the min-max "
                          "page score or the mean-pooling score")
+    ap.add_argument("--stats", choices=["f32", "bf16"], default=None,
+                    help="storage of the block statistics of a block-scored workload (bf16 halves their bytes)")
     ap.add_argument("--rla", action="store_true",
                     help="add the residual linear attention over the rows outside each support (SPLA)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -70,18 +72,19 @@ def parse():
     return a
 
 
-def with_score(cfg, score):
-    """The workload with another block score (block-scored workloads only)."""
-    if score is None or score == cfg.score:
+def with_score(cfg, score, stats=None):
+    """The workload with another block score or statistics storage (block-scored workloads only)."""
+    if (score is None or score == cfg.score) and (stats is None or stats == cfg.stats):
         return cfg
     if cfg.score == "lowrank":
-        raise SystemExit(f"--score applies to block-scored workloads; {cfg.name} uses low-rank index scores")
-    return cfg.with_(score=score)
+        raise SystemExit(f"--score / --stats apply to block-scored workloads; {cfg.name} uses low-rank index scores")
+    return cfg.with_(score=score or cfg.score, stats=stats or cfg.stats)
 
 
 def workload_desc(cfg):
-    return (f"{cfg.name}: {cfg.select} decode, {cfg.score} scores, collapse={cfg.collapse}, B={cfg.B} Hq={cfg.Hq} "
-            f"Hkv={cfg.Hkv} d={cfg.d} r={cfg.r} N={cfg.N} p={cfg.topp} k={cfg.topk} sink={cfg.sink} "
+    return (f"{cfg.name}: {cfg.select} decode, {cfg.score} scores"
+            f"{' (bf16 block statistics)' if cfg.stats == 'bf16' else ''}, collapse={cfg.collapse}, B={cfg.B} "
+            f"Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} r={cfg.r} N={cfg.N} p={cfg.topp} k={cfg.topk} sink={cfg.sink} "
             f"window={cfg.window}")
 
 
@@ -185,7 +188,7 @@ def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cfg = with_score(DECODE_CONFIGS[a.config], a.score)
+    cfg = with_score(DECODE_CONFIGS[a.config], a.score, a.stats)
     import oracle
 
     x = decode_inputs(cfg)
@@ -231,7 +234,7 @@ def run_spa(a):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    base = with_score(DECODE_CONFIGS[a.config], a.score)
+    base = with_score(DECODE_CONFIGS[a.config], a.score, a.stats)
     # weak scaling: every rank holds its own B sequences (a shard of a global batch of world*B)
     cfg_global = global_config(base, world)
     t = time.perf_counter()
@@ -257,10 +260,11 @@ def run_spa(a):
         kw.update(q_idx=dqi, Kidx=dKi)
     else:
         # block statistics: once per filled block, off the per-step path
+        bf16_stats = cfg.stats == "bf16"
         if cfg.score == "minmax":
-            bm, bv = spa.block_minmax(dK, cfg.block)
+            bm, bv = spa.block_minmax(dK, cfg.block, bf16=bf16_stats)
         else:
-            bm, bv = spa.block_stats(dK, cfg.block)
+            bm, bv = spa.block_stats(dK, cfg.block, bf16=bf16_stats)
             if cfg.score == "mean":
                 bv = None
         kw.update(bmean=bm, bvar=bv)
@@ -352,9 +356,10 @@ def run_spa(a):
             score_bytes -= int(local_np.sum()) * cfg.N * cfg.r * 2
     else:
         n_stats = 1 if cfg.score == "mean" else 2     # (mean) or (mean, var) / (min, max)
-        score_bytes = n_stats * cfg.B * cfg.Hkv * M * d * 4 + cfg.B * cfg.Hq * d * 2
+        n_stats *= 2 if cfg.stats == "bf16" else 4     # bytes per statistic
+        score_bytes = n_stats * cfg.B * cfg.Hkv * M * d + cfg.B * cfg.Hq * d * 2
         if cfg.collapse == "group":      # a local unit's block statistics are not read
-            score_bytes -= int(local_np.sum()) * n_stats * M * d * 4
+            score_bytes -= int(local_np.sum()) * n_stats * M * d
     attend_bytes = rows * KV_ROW_BYTES(d) + 2 * cfg.B * cfg.Hq * d * 2
     if rla is not None:      # the state (S, z) of every kv head and gamma, read once
         attend_bytes += cfg.B * cfg.Hkv * (d * d + d) * 4 + cfg.Hq * d * 4

@@ -20,7 +20,8 @@ def _run(args, env_extra=None):
 
 
 @pytest.mark.parametrize("extra,needle", [([], None), (["--rla"], "residual linear attention"),
-                                          (["--config", "c3", "--score", "minmax"], "minmax scores")])
+                                          (["--config", "c3", "--score", "minmax"], "minmax scores"),
+                                          (["--config", "c3", "--stats", "bf16"], "bf16 block statistics")])
 def test_reference_arm_line(extra, needle):
     args = ["--steps", "2", "--warmup", "1"]
     if "--config" not in extra:
