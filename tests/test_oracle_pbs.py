@@ -129,3 +129,21 @@ def test_scattered_heavy_hitters_cluster_into_one_permuted_block():
     np.testing.assert_array_equal(sup, heavy)
     # without the permutation a one-block budget cannot hold them: they span several blocks
     assert len(set((heavy // b).tolist())) > 1
+
+
+def test_pbs_output_is_sparse_attention_over_support_and_earlier_own_segment_rows():
+    # the form the GPU path reuses: rows = selected permuted blocks (original positions) and
+    # the own segment's rows before the query block, plus the block's causal diagonal --
+    # the same row set as the shared-support prefill's, with [seg0, t0) added to the support
+    b, S, T, scale, k = 16, 64, 256, 0.3, 2
+    Q, K, V = _case(20, T)
+    perm = oracle.pbs_permutation(oracle.pbs_importance(Q[T - b:], T - b, K, scale), S)
+    for t0 in (80, 160, 240):
+        sup, out = oracle.pbs_prefill_unit(Q[t0:t0 + b], t0, K, V, perm, S, k, scale)
+        seg0 = t0 // S * S
+        base = np.concatenate([sup, np.arange(seg0, t0)]).astype(np.int32)
+        for i in range(b):
+            rows = np.concatenate([base, np.arange(t0, t0 + i + 1)]).astype(np.int32)
+            for h in range(2):
+                ref, _ = oracle.sparse_attention(Q[t0 + i, h:h + 1], K, V, rows, scale)
+                np.testing.assert_allclose(out[i, h], ref[0], rtol=1e-12, atol=1e-14)
