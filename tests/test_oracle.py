@@ -323,3 +323,32 @@ def test_routed_decode_local_units_attend_over_sink_and_window():
         Kf = bf16_value(x["K"][b, g][rows]).astype(np.float64)
         Vf = bf16_value(x["V"][b, g][rows]).astype(np.float64)
         np.testing.assert_allclose(r["out"], _sdpa(qf, Kf, Vf, oracle.f32(cfg.sm_scale)), rtol=1e-10, atol=1e-12)
+
+
+def test_per_query_prefill_b_sel_1():
+    # "Oracle-Guided Sparse Prefill" 2.1 with b_sel = 1: every query has its own support,
+    # scored with the mean of its G heads' index queries; a full budget is dense causal
+    # attention, a budget of k is the lexsort top-k of those scores united with the sink
+    cfg = SMALL["c5s"].with_(N=600, q_start=584, T=16, Hq=4, Hkv=2, bq=1, topk=10_000, n_clusters=4)
+    x = prefill_inputs(cfg)
+    G, d = cfg.G, cfg.d
+    for j in (0, 7, 15):
+        for g in range(cfg.Hkv):
+            support, out = oracle.prefill_block(cfg, x, j, g)
+            t = cfg.q_start + j
+            assert support.tolist() == list(range(t))
+            Kf = bf16_value(x["K"][g, : t + 1]).astype(np.float64)
+            Vf = bf16_value(x["V"][g, : t + 1]).astype(np.float64)
+            for hh in range(G):
+                qf = bf16_value(x["Q"][j, g * G + hh]).astype(np.float64)
+                ref = _sdpa(qf[None], Kf, Vf, oracle.f32(cfg.sm_scale))[0]
+                np.testing.assert_allclose(out[0, hh], ref, rtol=1e-11, atol=1e-12)
+    small = cfg.with_(topk=50)
+    j, g = 9, 1
+    support, _ = oracle.prefill_block(small, x, j, g)
+    t = cfg.q_start + j
+    qi = bf16_value(x["q_idx"][j, g * G:(g + 1) * G]).astype(np.float64)
+    s = oracle.f32(cfg.score_scale) * (bf16_value(x["Kidx"][g, :t]).astype(np.float64) @ qi.mean(0))
+    s = s.astype(np.float32).astype(np.float64)
+    order = np.lexsort((np.arange(t), -s))
+    assert support.tolist() == sorted(set(order[:50].tolist()) | set(range(cfg.sink)))
