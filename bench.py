@@ -183,6 +183,25 @@ def cpu_baseline(cfg, x, seconds: float, local=None, rla=None):
                       f"{cfg.name}, fp64 oracle, {dt:.1f} s"}
 
 
+def captured_mass_report(cfg, x, idx, counts):
+    """Captured mass on the GPU's supports (CPU leg, outside the timed region): for every unit,
+    the oracle's dense head-averaged attention distribution over all N cached rows summed over
+    the rows of the support the GPU selected ("Oracle-Guided Sparse Prefill" 2.1: the mass P
+    a support keeps; "Full Attention Strikes Back" (RTPurbo), key results: attention mass
+    beside sparsity)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max(1, cores)) as ex:
+        vals = list(ex.map(lambda u: oracle.captured_mass(cfg, x, u, idx[u, :counts[u]]), range(cfg.U)))
+    return {"mean": round(float(np.mean(vals)), 5), "min": round(float(np.min(vals)), 5),
+            "units": f"all {cfg.U} units", "how": "fp64 oracle, dense head-averaged softmax over all N rows, "
+            f"summed over the GPU's support ({time.perf_counter() - t0:.1f} s on {cores} host threads)"}
+
+
 # ============================================================================ reference arm
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
@@ -296,6 +315,7 @@ def run_spa(a):
     torch.cuda.synchronize()
     assert spa.read_device_status(plan.ws) == 0, "device status raised during warm-up"
     counts = plan.count.cpu().numpy().astype(np.int64)
+    sup_idx = plan.idx.cpu().numpy()
     rows = int(counts.sum()) * cfg.block
     M = cfg.N // cfg.block
     sparsity = 1.0 - counts.sum() / (cfg.U * M)
@@ -435,6 +455,8 @@ def run_spa(a):
             "clocks": clocks,
             "wall_s_timed_region": w1 - w0,
         }
+        if not a.no_cpu_baseline:
+            line["config"]["captured_mass"] = captured_mass_report(cfg, x, sup_idx, counts)
         if not a.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(cfg, x, a.cpu_seconds, local=local_np if n_local else None,
                                                 rla=rla)
@@ -460,6 +482,44 @@ def prefill_flops(cfg, counts):
     diag = cfg.bq * (cfg.bq + 1) // 2                 # sum over the block's rows of (i + 1)
     keys = cfg.bq * counts.astype(np.int64) + diag    # per unit and query head
     return float(4 * cfg.d * cfg.G * keys.sum())
+
+
+def prefill_sparsity(cfg, counts):
+    """1 - (keys a query reads) / (keys it may read causally), averaged over the chunk's queries:
+    query t0 + i of a block reads its support and the block's own rows [t0, t0 + i]."""
+    tot, read = 0.0, 0.0
+    for u in range(cfg.U):
+        j = u // cfg.Hkv
+        t0 = cfg.q_start + j * cfg.bq
+        for i in range(cfg.bq):
+            tot += t0 + i + 1
+            read += counts[u] + i + 1
+    return 1.0 - read / tot
+
+
+def prefill_captured_mass(cfg, x, idx, counts):
+    """Captured mass of a fixed sample of prefill units (CPU leg, outside the timed region): four
+    query blocks (first, one third, two thirds, last) x every kv head, all 64 queries each."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+
+    blocks = sorted({0, cfg.n_blocks // 3, 2 * cfg.n_blocks // 3, cfg.n_blocks - 1})
+    units = [(j, g) for j in blocks for g in range(cfg.Hkv)]
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    t0 = time.perf_counter()
+
+    def one(jg):
+        j, g = jg
+        u = j * cfg.Hkv + g
+        return oracle.captured_mass_prefill(cfg, x, j, g, idx[u, :counts[u]])
+
+    with ThreadPoolExecutor(max(1, cores)) as ex:
+        vals = list(ex.map(one, units))
+    return {"mean": round(float(np.mean(vals)), 5), "min": round(float(np.min(vals)), 5),
+            "units": f"{len(units)} units: query blocks {blocks} x {cfg.Hkv} kv heads",
+            "how": "fp64 oracle, dense causal head-averaged softmax per query, summed over the support and the "
+                   f"block's own rows ({time.perf_counter() - t0:.1f} s on {cores} host threads)"}
 
 
 def run_prefill(a):
@@ -545,6 +605,9 @@ def run_prefill(a):
     peak = peak or 1590.0
     # the oracle on a bounded sample of units (one host core per unit, all cores)
     cpu = None
+    mass = None
+    if not a.no_cpu_baseline:
+        mass = prefill_captured_mass(cfg, x, plan.idx.cpu().numpy(), counts)
     if not a.no_cpu_baseline:
         units = [(j, g) for j in range(cfg.n_blocks) for g in range(cfg.Hkv)]
         t0, done, cf = time.perf_counter(), 0, 0.0
@@ -562,7 +625,8 @@ def run_prefill(a):
            "config": {"workload": f"{cfg.name}: prefill chunk T={cfg.T} at q_start={cfg.q_start}, N={cfg.N}, "
                                   f"Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} bq={cfg.bq} top-k={cfg.topk} sink={cfg.sink}",
                       "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
-                      "support_mean": float(counts.mean()), "algorithmic_gflop_per_step": flops / 1e9},
+                      "support_mean": float(counts.mean()), "algorithmic_gflop_per_step": flops / 1e9,
+                      "sparsity": round(float(prefill_sparsity(cfg, counts)), 4), "captured_mass": mass},
            "roofline": {"bound": "tensor", "kernel": "prefill (all kernels of the step)", "achieved": tflops,
                         "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
                         "traffic": None},

@@ -81,8 +81,9 @@ const char* spa_status_string(int status);
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
 const char* spa_last_cuda_error(void);
 
-/* ABI version of this header: 5 (spa_decode_args gained local_units in 2, the RLA fields in 3;
- * the min-max and mean block scores and spa_block_minmax came in 4; bf16 statistics in 5). */
+/* ABI version of this header: 6 (spa_decode_args gained local_units in 2, the RLA fields in 3;
+ * the min-max and mean block scores and spa_block_minmax came in 4; bf16 statistics in 5;
+ * spa_select_static_status in 6). */
 int spa_abi_version(void);
 
 /* ------------------------------------------------------------------------------------
@@ -192,12 +193,21 @@ size_t spa_select_workspace_bytes(int U, int M);
  * (cudaMemsetAsync on `stream`) and allocates nothing.  All calls share the one array:
  * calls that overlap on the GPU (other streams, other host threads on the same device)
  * race, and the caller must serialise them.  A support larger than cap shows as
- * count[u] > cap (there is no status word to read back).
+ * count[u] > cap and as SPA_ERR_CAPACITY in the array's status word, which
+ * spa_select_static_status reads back.
  */
 #define SPA_SELECT_STATIC_MAX_UNITS 16
 spa_status spa_select_topp_static(const float* scores, const int32_t* unit_len, int U, int M, float p,
                                   int sink, int window, int32_t* idx, int32_t* count, int cap,
                                   float* index_mass, void* stream);
+
+/* Status word of spa_select_topp_static's fixed scratch (the same interface addition; the
+ * method pages have no counterpart): synchronises `stream`, copies the word (sticky OR of
+ * (1 << SPA_ERR_*) raised on the device: SPA_ERR_CAPACITY, SPA_ERR_TIMEOUT) to *bits and,
+ * if reset != 0, clears it.  Every spa_select_topp_static call starts from a cleared word,
+ * so the word describes the last call; read it before the next one.  Allocates nothing.
+ * Returns SPA_OK, SPA_ERR_INVALID_ARG (bits NULL) or SPA_ERR_CUDA. */
+spa_status spa_select_static_status(void* stream, uint32_t* bits, int reset);
 
 /* ------------------------------------------------------------------------------------
  * a7/a8. Exact softmax attention on the gathered support ("Oracle-Guided Sparse

@@ -7,7 +7,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(HERE, "libspa.so")
 
-ABI_VERSION = 5   # spa_abi_version() of the library these declarations describe
+ABI_VERSION = 6   # spa_abi_version() of the library these declarations describe
 
 SPA_OK = 0
 SPA_ERR_INVALID_ARG = 1
@@ -76,6 +76,7 @@ SIGNATURES = {
     "spa_select_topp": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p, _sz, _p]),
     "spa_select_workspace_bytes": (_sz, [_i, _i]),
     "spa_select_topp_static": (_i, [_p, _p, _i, _i, _f, _i, _i, _p, _p, _i, _p, _p]),
+    "spa_select_static_status": (_i, [_p, ctypes.POINTER(ctypes.c_uint32), _i]),
     "spa_block_minmax": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_block_stats_bf16": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_block_minmax_bf16": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),

@@ -73,7 +73,7 @@ const char* spa_status_string(int s) {
 
 const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
-int spa_abi_version(void) { return 5; }
+int spa_abi_version(void) { return 6; }
 
 // shared checks of the block-statistics entries; SPA_OK with *noop set when there is nothing to do
 static spa_status check_stats_args(const uint16_t* K, int B, int Hkv, int N, int d, int block, const void* a,

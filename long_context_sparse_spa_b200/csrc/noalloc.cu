@@ -78,3 +78,21 @@ extern "C" spa_status spa_select_topp_static(const float* scores, const int32_t*
     if (s != SPA_OK) return s;
     return launch_select(sp, true, st);
 }
+
+// Status word of the fixed scratch: the select kernel ORs SPA_ERR_TIMEOUT / SPA_ERR_CAPACITY
+// into it.  Copied with one cudaMemcpyAsync on the caller's stream (and cleared with one
+// cudaMemsetAsync if asked); nothing is allocated.
+extern "C" spa_status spa_select_static_status(void* stream, uint32_t* bits, int reset) {
+    if (!bits) return SPA_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    spa_status s = scratch_address(&scratch);
+    if (s != SPA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SPA_CUDA_TRY(cudaMemcpyAsync(bits, scratch, sizeof(uint32_t), cudaMemcpyDeviceToHost, st));
+    SPA_CUDA_TRY(cudaStreamSynchronize(st));
+    if (reset) {
+        SPA_CUDA_TRY(cudaMemsetAsync(scratch, 0, sizeof(uint32_t), st));
+        SPA_CUDA_TRY(cudaStreamSynchronize(st));
+    }
+    return SPA_OK;
+}

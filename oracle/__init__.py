@@ -440,6 +440,25 @@ def captured_mass(cfg, x: Dict[str, np.ndarray], u: int, idx: np.ndarray) -> flo
     return float(P[rows[rows < cfg.N]].sum())
 
 
+def captured_mass_prefill(cfg, x: Dict[str, np.ndarray], j: int, g: int, support: np.ndarray,
+                          queries: Optional[Sequence[int]] = None) -> float:
+    """Captured mass of one prefill unit (query block j, kv head g) [OGS-2.1 P_{l,t}]: for
+    each query t of the block, the dense causal head-averaged distribution over keys
+    [0, t] summed over the keys its attention reads (the shared support and the block's
+    own positions [t0, t]); the mean over the block's queries (or the given ones)."""
+    G, bq = cfg.G, cfg.bq
+    t0 = cfg.q_start + j * bq
+    sup = np.asarray(support, np.int64)
+    vals = []
+    for i in (range(bq) if queries is None else queries):
+        t = t0 + i
+        P = dense_probs(x["Q"][j * bq + i, g * G:(g + 1) * G], x["K"][g][:t + 1], f32(cfg.sm_scale))
+        own = np.arange(t0, t + 1)
+        rows = np.union1d(sup[sup <= t], own)
+        vals.append(float(P[rows].sum()))
+    return float(np.mean(vals))
+
+
 def prefill_block(cfg, x: Dict[str, np.ndarray], j: int, g: int, want_scores: bool = False):
     """Unit (query block j, kv head g) of a shared-support prefill -> (support, out [bq, G, d])
     (and the ranked scores of the candidates [0, t0) when want_scores)."""

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported_and_bound():
 
 def test_status_strings_and_version():
     L = spa.lib()
-    assert L.spa_abi_version() == 5 == _abi.ABI_VERSION
+    assert L.spa_abi_version() == 6 == _abi.ABI_VERSION
     assert L.spa_status_string(_abi.SPA_ERR_CAPACITY) == b"SPA_ERR_CAPACITY"
     assert L.spa_status_string(99) == b"SPA_ERR_UNKNOWN"
 
@@ -118,3 +118,8 @@ def test_decode_rla_fields_validation():
     assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(P), need, None) == _abi.SPA_ERR_INVALID_ARG
     a.rla_z, a.rla_eps = P, -1.0                                          # negative epsilon
     assert L.spa_decode(ctypes.byref(a), ctypes.c_void_p(P), need, None) == _abi.SPA_ERR_INVALID_ARG
+
+
+def test_static_status_rejects_null_bits():
+    # validation precedes the device lookup: no GPU needed
+    assert spa.lib().spa_select_static_status(None, None, 0) == _abi.SPA_ERR_INVALID_ARG

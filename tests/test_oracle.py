@@ -352,3 +352,27 @@ def test_per_query_prefill_b_sel_1():
     s = s.astype(np.float32).astype(np.float64)
     order = np.lexsort((np.arange(t), -s))
     assert support.tolist() == sorted(set(order[:50].tolist()) | set(range(cfg.sink)))
+
+
+def test_captured_mass_prefill():
+    """Captured mass of a prefill unit: 1 when the support holds every earlier key (the block's
+    own rows are always read); otherwise the mean over queries of the brute-force causal
+    head-averaged softmax summed over support and own rows ("Oracle-Guided Sparse Prefill" 2.1)."""
+    cfg = SMALL["c5s"].with_(N=640, q_start=512, T=128, Hq=4, Hkv=2, topk=10_000, n_clusters=4)
+    x = prefill_inputs(cfg)
+    j, g = 1, 0
+    t0 = cfg.q_start + j * cfg.bq
+    assert abs(oracle.captured_mass_prefill(cfg, x, j, g, np.arange(t0)) - 1.0) < 1e-12
+    sup = np.array([0, 1, 2, 3, 77, 300, 301, 555], np.int64)
+    got = oracle.captured_mass_prefill(cfg, x, j, g, sup, queries=[0, 5, 63])
+    vals = []
+    for i in (0, 5, 63):
+        t = t0 + i
+        Kf = bf16_value(x["K"][g, : t + 1]).astype(np.float64)
+        P = np.zeros(t + 1)
+        for hh in range(cfg.G):
+            qf = bf16_value(x["Q"][j * cfg.bq + i, g * cfg.G + hh]).astype(np.float64)
+            P += torch.softmax(torch.tensor(oracle.f32(cfg.sm_scale) * (Kf @ qf)), 0).numpy() / cfg.G
+        rows = sorted(set(sup.tolist()) | set(range(t0, t + 1)))
+        vals.append(P[rows].sum())
+    assert abs(got - np.mean(vals)) < 1e-12
