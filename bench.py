@@ -63,6 +63,8 @@ def parse():
                     help="storage of the block statistics of a block-scored workload (bf16 halves their bytes)")
     ap.add_argument("--rla", action="store_true",
                     help="add the residual linear attention over the rows outside each support (SPLA)")
+    ap.add_argument("--path", choices=["separate", "fused"], default="separate",
+                    help="decode kernels: separate kernels (default) or the fused persistent kernel where it applies")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
     if a.steps is None:
@@ -101,8 +103,8 @@ def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel source (profiles/traffic.tsv: kernel, workload, bytes, source sha256 prefix)."""
     path = os.path.join(ROOT, "profiles", "traffic.tsv")
-    src = os.path.join(ROOT, "long_context_sparse_spa_b200", "csrc", "attend.cu" if kernel == "attend" else
-                       ("scores.cu" if kernel == "scores" else "select.cu"))
+    src = os.path.join(ROOT, "long_context_sparse_spa_b200", "csrc",
+                       {"attend": "attend.cu", "scores": "scores.cu", "fused": "fused.cu"}.get(kernel, "select.cu"))
     if not os.path.exists(path) or not os.path.exists(src):
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -273,7 +275,8 @@ def run_spa(a):
               collapse=spa.SPA_COLLAPSE_GROUP_MEAN if cfg.collapse == "group" else spa.SPA_COLLAPSE_NONE,
               q=dq, K=dK, V=dV, block=cfg.block, score_scale=float(np.float32(cfg.score_scale)),
               sm_scale=float(np.float32(cfg.sm_scale)), topk=cfg.topk, topp=cfg.topp, sink=cfg.sink,
-              window=cfg.window, cap=cfg.cap, want_f32=False, want_lse=False, run=False)
+              window=cfg.window, cap=cfg.cap, want_f32=False, want_lse=False, run=False,
+              kernel_path=spa.SPA_DECODE_FUSED if a.path == "fused" else spa.SPA_DECODE_SEPARATE)
     if lowrank:
         dqi, dKi = up(x["q_idx"]), up(x["Kidx"])
         kw.update(q_idx=dqi, Kidx=dKi)
@@ -357,8 +360,11 @@ def run_spa(a):
         flush_l2()
         plan.run_timed(kev[i])
     torch.cuda.synchronize()
+    fused = plan.fused
+    k_names = ("fused", "none", "combine") if fused else ("scores", "select", "attend")
     k_ms = {name: np.array([kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(n_split)])
-            for j, name in enumerate(("scores", "select", "attend"))}
+            for j, name in enumerate(k_names)}
+    k_ms.pop("none", None)
     dev_s = float(step_ms.sum()) / 1e3
     t_max = dev_s
     if world > 1:
@@ -386,8 +392,14 @@ def run_spa(a):
     step_bytes = score_bytes + attend_bytes
     peak, peak_kind = peaks()
     mean_ms = {k: float(v.mean()) for k, v in k_ms.items()}
-    kbytes = {"scores": score_bytes, "attend": attend_bytes, "select": 0}
-    dom = max(("scores", "attend"), key=lambda k: mean_ms[k])
+    if fused:
+        # one kernel moves both streams (index keys and the gathered rows); the combine
+        # kernel merges its records
+        kbytes = {"fused": step_bytes, "combine": 0}
+        dom = "fused"
+    else:
+        kbytes = {"scores": score_bytes, "attend": attend_bytes, "select": 0}
+        dom = max(("scores", "attend"), key=lambda k: mean_ms[k])
     achieved = kbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": peak_kind,
@@ -449,9 +461,11 @@ def run_spa(a):
             "kernels_ms": {k: round(v, 5) for k, v in mean_ms.items()},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": float(np.mean(e2e_ms))},
-            # per step: scores (with the level-0 histogram fused when one score row serves a
-            # kv head), [histogram], selection, attention, log-sum-exp combine
-            "gpu_launches": (4 if (lowrank and cfg.collapse == "group") else 5) * a.steps,
+            # per step: the fused persistent kernel and the combine; or scores (with the
+            # level-0 histogram fused when one score row serves a kv head), [histogram],
+            # selection, attention, log-sum-exp combine
+            "gpu_launches": (2 if fused else (4 if (lowrank and cfg.collapse == "group") else 5)) * a.steps,
+            "decode_path": "fused persistent kernel + combine" if fused else "separate kernels",
             "clocks": clocks,
             "wall_s_timed_region": w1 - w0,
         }

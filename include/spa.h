@@ -296,14 +296,36 @@ typedef struct spa_decode_args {
     const float* rla_gamma;
     float rla_eps;           /* RMSNorm epsilon, >= 0 */
     int stats_bf16;          /* block kinds: bmean / bvar are bf16 bit patterns (spa_block_*_bf16), else fp32 */
+    /* Kernel path (spa_decode_path).  SPA_DECODE_AUTO (the default) and SPA_DECODE_SEPARATE
+     * run scoring, selection and attention as separate kernels.  SPA_DECODE_FUSED runs
+     * low-rank, head-collapsed decodes (d = 128, G <= 8, 16384 <= N <= 2^23, no local_units,
+     * no RLA) as one persistent dataflow kernel, in which every unit's selection chain runs
+     * beside the other units' HBM streams, plus a combine kernel (other decodes fall back to
+     * the separate kernels).  Supports are identical on both paths; the fused path sums the
+     * attention in the order its CTAs claimed the rows, so its outputs may differ between
+     * runs in the last bits of fp32.  A workspace serves one path: zero it again before
+     * using it with the other. */
+    int kernel_path;
 } spa_decode_args;
+
+typedef enum spa_decode_path {
+    SPA_DECODE_AUTO = 0,
+    SPA_DECODE_SEPARATE = 1,
+    SPA_DECODE_FUSED = 2
+} spa_decode_path;
 
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream);
 size_t spa_decode_workspace_bytes(const spa_decode_args* a);
 
+/* The path spa_decode takes for these arguments: SPA_DECODE_FUSED when it runs the fused
+ * persistent kernel, SPA_DECODE_SEPARATE otherwise (host-side, no GPU work; -1 for NULL). */
+int spa_decode_path_taken(const spa_decode_args* a);
+
 /* spa_decode that also records four caller-created cudaEvent_t on `stream`: events[0]
  * before the scoring kernel, events[1] after it, events[2] after the selection kernel and
- * events[3] after the attention kernel, so a caller can time each kernel inside a real step. */
+ * events[3] after the attention kernel, so a caller can time each kernel inside a real step.
+ * On the fused path events[0] precedes the persistent kernel, events[1] and events[2] both
+ * follow it and events[3] follows the combine kernel. */
 spa_status spa_decode_timed(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
                             void* const* events);
 

@@ -17,7 +17,8 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_SCORE_LOWRANK, SPA_SCORE_MEAN_BLOCK,
+from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_DECODE_AUTO, SPA_DECODE_FUSED, SPA_DECODE_SEPARATE,
+                   SPA_SCORE_LOWRANK, SPA_SCORE_MEAN_BLOCK,
                    SPA_SCORE_MINMAX_BLOCK, SPA_SCORE_TAYLOR_BLOCK, SPA_SELECT_TOPK, SPA_STATS_BF16, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
 
 __all__ = [
@@ -25,6 +26,7 @@ __all__ = [
     "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "prefill", "PrefillPlan", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
     "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SCORE_MINMAX_BLOCK", "SPA_SCORE_MEAN_BLOCK",
     "SPA_SELECT_TOPK", "SPA_SELECT_TOPP", "SPA_STATS_BF16", "block_minmax", "rla_state",
+    "SPA_DECODE_AUTO", "SPA_DECODE_SEPARATE", "SPA_DECODE_FUSED",
 ]
 
 
@@ -205,6 +207,11 @@ class DecodePlan:
         check(lib().spa_decode(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
                                _stream(stream)))
 
+    @property
+    def fused(self) -> bool:
+        """Whether spa_decode runs these arguments as the fused persistent kernel."""
+        return lib().spa_decode_path_taken(ctypes.byref(self.args)) == SPA_DECODE_FUSED
+
     def run_timed(self, events, stream: Optional[torch.cuda.Stream] = None) -> None:
         """run() recording four torch.cuda.Event (enable_timing=True, already recorded once so that
         they exist) before scoring, after scoring, after selection and after attention."""
@@ -220,13 +227,15 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
            window: int = 0, cap: Optional[int] = None, want_f32: bool = True, want_lse: bool = True,
            local_units: Optional[torch.Tensor] = None, rla_state: Optional[torch.Tensor] = None,
            rla_z: Optional[torch.Tensor] = None, rla_gamma: Optional[torch.Tensor] = None,
-           rla_eps: float = 1e-6, run: bool = True) -> DecodePlan:
+           rla_eps: float = 1e-6, kernel_path: int = SPA_DECODE_AUTO, run: bool = True) -> DecodePlan:
     """Build (and by default run) a fused decode step; see spa_decode in include/spa.h.
     local_units: optional uint8 [U] on the device, nonzero for the units that head-wise routing
     makes local (support = sink + window, not scored).
     rla_state / rla_z / rla_gamma: optional fp32 [B, Hkv, d, d] / [B, Hkv, d] / [Hq, d] that
     add the residual linear attention over the rows outside each support (state from
-    rla_state())."""
+    rla_state()).
+    kernel_path: SPA_DECODE_AUTO / SPA_DECODE_SEPARATE (scoring, selection and attention as
+    separate kernels) or SPA_DECODE_FUSED (the persistent dataflow kernel where it applies)."""
     for t, n in ((q, "q"), (K, "K"), (V, "V")):
         _need(t, torch.bfloat16, n)
     B, Hq, d = q.shape
@@ -253,6 +262,7 @@ def decode(*, score_kind: int, select_kind: int, collapse: int, q: torch.Tensor,
     a.stats_bf16 = int(bmean is not None and bmean.dtype == torch.bfloat16)
     a.score_scale, a.sm_scale = score_scale, sm_scale
     a.topk, a.topp, a.sink, a.window = topk, topp, sink, window
+    a.kernel_path = kernel_path
     a.idx, a.count, a.cap = _ptr(idx), _ptr(count), cap
     a.index_mass = _ptr(mass)
     a.out, a.out_f32, a.lse = _ptr(out), _ptr(out32), _ptr(lse)

@@ -27,6 +27,9 @@ SPA_STATS_BF16 = 0x100
 SPA_SELECT_TOPK = 0
 SPA_SELECT_TOPP = 1
 SPA_SELECT_STATIC_MAX_UNITS = 16
+SPA_DECODE_AUTO = 0
+SPA_DECODE_SEPARATE = 1
+SPA_DECODE_FUSED = 2
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -50,6 +53,7 @@ class SpaDecodeArgs(ctypes.Structure):
         ("local_units", _p),
         ("rla_state", _p), ("rla_z", _p), ("rla_gamma", _p), ("rla_eps", _f),
         ("stats_bf16", _i),
+        ("kernel_path", _i),
     ]
 
 
@@ -85,6 +89,7 @@ SIGNATURES = {
     "spa_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "spa_decode": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p]),
     "spa_decode_workspace_bytes": (_sz, [ctypes.POINTER(SpaDecodeArgs)]),
+    "spa_decode_path_taken": (_i, [ctypes.POINTER(SpaDecodeArgs)]),
     "spa_decode_timed": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p, ctypes.POINTER(_p)]),
     "spa_read_device_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32), _i]),
     "spa_prefill_shared": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),

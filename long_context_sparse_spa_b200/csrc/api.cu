@@ -45,10 +45,16 @@ namespace {
 
 inline bool bad_dims(int B, int Hq, int Hkv) { return B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0; }
 
+// scores per unit of a decode: tokens, or blocks for the block score kinds
+int decode_units_m(const spa_decode_args* a) {
+    const bool block_kind = a->score_kind == SPA_SCORE_TAYLOR_BLOCK || a->score_kind == SPA_SCORE_MINMAX_BLOCK ||
+                            a->score_kind == SPA_SCORE_MEAN_BLOCK;
+    return block_kind ? a->N / (a->block > 0 ? a->block : 1) : a->N;
+}
+
 size_t decode_scores_bytes(const spa_decode_args* a) {
     const int U = a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->B * a->Hkv : a->B * a->Hq;
-    const int M = a->score_kind == SPA_SCORE_TAYLOR_BLOCK ? a->N / (a->block > 0 ? a->block : 1) : a->N;
-    return align_up(size_t(U) * size_t(M) * 4, 256);
+    return align_up(size_t(U) * size_t(decode_units_m(a)) * 4, 256);
 }
 
 }  // namespace
@@ -252,12 +258,24 @@ spa_status spa_sparse_attend(const uint16_t* q, const uint16_t* K, const uint16_
 size_t spa_decode_workspace_bytes(const spa_decode_args* a) {
     if (!a || bad_dims(a->B, a->Hq, a->Hkv)) return 0;
     const int U = a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->B * a->Hkv : a->B * a->Hq;
-    return kWsHeader + decode_scores_bytes(a) + select_scratch_bytes(U) +
-           attend_scratch_bytes(U, a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->Hq / a->Hkv : 1, a->d);
+    const size_t separate = kWsHeader + decode_scores_bytes(a) + select_scratch_bytes(U) +
+                            attend_scratch_bytes(U, a->collapse == SPA_COLLAPSE_GROUP_MEAN ? a->Hq / a->Hkv : 1, a->d);
+    if (a->kernel_path == SPA_DECODE_FUSED && a->N >= 0 && fused_decode_supported(a)) {
+        const size_t fused = kWsHeader + fused_scratch_bytes(a);
+        return fused > separate ? fused : separate;
+    }
+    return separate;
 }
 
 static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream,
                               void* const* events);
+
+int spa_decode_path_taken(const spa_decode_args* a) {
+    if (!a) return -1;
+    return a->kernel_path == SPA_DECODE_FUSED && !bad_dims(a->B, a->Hq, a->Hkv) && fused_decode_supported(a)
+               ? SPA_DECODE_FUSED
+               : SPA_DECODE_SEPARATE;
+}
 
 spa_status spa_decode(const spa_decode_args* a, void* ws, size_t ws_bytes, void* stream) {
     return decode_impl(a, ws, ws_bytes, stream, nullptr);
@@ -306,8 +324,19 @@ static spa_status decode_impl(const spa_decode_args* a, void* ws, size_t ws_byte
         if (!aligned16(a->q_idx) || !aligned16(a->Kidx)) return SPA_ERR_UNSUPPORTED_SHAPE;
     }
 
+    if (a->kernel_path != SPA_DECODE_AUTO && a->kernel_path != SPA_DECODE_SEPARATE && a->kernel_path != SPA_DECODE_FUSED)
+        return SPA_ERR_INVALID_ARG;
+
     uint8_t* w = static_cast<uint8_t*>(ws);
     uint32_t* status = reinterpret_cast<uint32_t*>(w);
+    if (a->kernel_path == SPA_DECODE_FUSED && fused_decode_supported(a)) {
+        // the persistent dataflow kernel; the pointer and alignment checks are the attention's
+        AttendParams chk;
+        spa_status s = attend_params(a->q, a->K, a->V, a->B, a->Hq, a->Hkv, a->N, a->d, a->idx, a->count, a->cap,
+                                     a->collapse, 1, a->sm_scale, a->out, a->out_f32, a->lse, ws, size_t(-1), chk);
+        if (s != SPA_OK) return s;
+        return launch_fused_decode(a, w + kWsHeader, status, st, events);
+    }
     float* scores = reinterpret_cast<float*>(w + kWsHeader);
     const Hist0 hist = hist0_carve(w + kWsHeader + decode_scores_bytes(a), U);
     uint8_t* attend_ws = w + kWsHeader + decode_scores_bytes(a) + select_scratch_bytes(U);

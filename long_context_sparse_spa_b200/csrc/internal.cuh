@@ -97,6 +97,123 @@ __device__ __forceinline__ unsigned long long fixed_mass(float s, float ref) {
     return __float2ull_rn(expf(s - ref) * kMassScale);
 }
 
+// ------------------------------------------------------------------ level-0 crossing bin
+// Shared by the cluster selection kernel and the fused decode kernel, so both take the same
+// decision from the same histogram: the first 256 threads of the block own 256 groups of 8
+// bins (descending from the top bin), every sum runs in a fixed order independent of the
+// block size (within a group, then a warp scan over the groups, then the warps in order).
+// Top-p: the crossing bin is the first (from the top) where the cumulative mass
+// sum_b mass_b * 2^-40 * exp(r_b - m) reaches p * Z; should fp64 rounding keep every
+// cumulative sum below p * Z, the lowest non-empty bin is taken (everything is needed).
+// Top-k: the first bin where the cumulative count reaches k (exact).
+struct Level0Shared {
+    uint32_t wc[8];
+    double wm[8];
+    uint32_t bin, above_cnt, bmin, hit;
+    uint32_t fb_above_cnt;
+    double above_mass, fb_above_mass;
+};
+struct Level0 {
+    uint32_t bin, above_cnt;
+    double above_mass, Z;
+};
+// blockDim.x >= 256 and a multiple of 32; every thread of the block must call it
+__device__ inline Level0 level0_crossing(const uint32_t* hc, const unsigned long long* hm, uint32_t max_key, bool topp,
+                                         float p, int k, Level0Shared& sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float m = key_score(max_key);
+    const bool act = tid < 256;
+    uint32_t vc[8];
+    unsigned long long mb[8];
+    double vm[8];
+    uint32_t gc = 0;
+    double gm = 0.0;
+    // every load of the thread is issued before any is used
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int bin = 2047 - (tid * 8 + j);
+        vc[j] = act ? __ldcg(hc + bin) : 0u;
+        mb[j] = act && topp ? __ldcg(hm + bin) : 0ull;
+    }
+    if (tid == 0) {
+        sh.bin = max_key >> 21;
+        sh.above_cnt = 0;
+        sh.above_mass = 0.0;
+        sh.bmin = 2048u;
+        sh.hit = 0;
+        sh.fb_above_cnt = 0;
+        sh.fb_above_mass = 0.0;
+    }
+    __syncthreads();
+    uint32_t my_min = 2048u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int bin = 2047 - (tid * 8 + j);
+        vm[j] = mb[j] ? double(mb[j]) * (1.0 / 1099511627776.0) * exp(double(bin_top_score(bin)) - double(m)) : 0.0;
+        if (vc[j]) my_min = min(my_min, uint32_t(bin));
+        gc += vc[j];
+        gm += vm[j];
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) my_min = min(my_min, __shfl_xor_sync(0xffffffffu, my_min, off));
+    if (lane == 0 && my_min < 2048u) atomicMin(&sh.bmin, my_min);
+    // inclusive scan over the groups of this warp, in group order
+    uint32_t ic = gc;
+    double im = gm;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t xc = __shfl_up_sync(0xffffffffu, ic, off);
+        const double xm = __shfl_up_sync(0xffffffffu, im, off);
+        if (lane >= off) { ic += xc; im += xm; }
+    }
+    if (act && lane == 31) { sh.wc[warp] = ic; sh.wm[warp] = im; }
+    __syncthreads();
+    uint32_t pc = 0, tc = 0;
+    double pm = 0.0, tm = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        if (w < warp) { pc += sh.wc[w]; pm += sh.wm[w]; }
+        tc += sh.wc[w];
+        tm += sh.wm[w];
+    }
+    const double T = double(p) * tm;
+    uint32_t ac = pc + ic - gc;
+    double am = pm + im - gm;
+    if (act) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t bin = uint32_t(2047 - (tid * 8 + j));
+            const bool hit = topp ? (am < T && am + vm[j] >= T) : (ac < uint32_t(k) && ac + vc[j] >= uint32_t(k));
+            if (hit) {
+                sh.bin = bin;
+                sh.above_cnt = ac;
+                sh.above_mass = am;
+                sh.hit = 1;
+            }
+            if (bin == sh.bmin) {   // bmin is final here (set before the barrier above)
+                sh.fb_above_cnt = ac;
+                sh.fb_above_mass = am;
+            }
+            ac += vc[j];
+            am += vm[j];
+        }
+    }
+    __syncthreads();
+    Level0 r;
+    if (!sh.hit && topp && sh.bmin < 2048u) {
+        r.bin = sh.bmin;
+        r.above_cnt = sh.fb_above_cnt;
+        r.above_mass = sh.fb_above_mass;
+    } else {
+        r.bin = sh.bin;
+        r.above_cnt = sh.above_cnt;
+        r.above_mass = sh.above_mass;
+    }
+    r.Z = tm;
+    __syncthreads();
+    return r;
+}
+
 __device__ __forceinline__ void raise_status(uint32_t* status, int code) {
     if (status) atomicOr(status, 1u << code);
 }
@@ -176,6 +293,13 @@ spa_status launch_rla_state(const uint16_t* K, const uint16_t* V, int BH, int N,
 // prefill.cu
 size_t prefill_scratch_bytes(int U, int N);
 spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st);
+
+// fused.cu: the persistent dataflow decode (low-rank, head-collapsed, d = 128, G <= 8)
+bool fused_decode_supported(const spa_decode_args* a);
+size_t fused_scratch_bytes(const spa_decode_args* a);
+// events (optional, 4): before the fused kernel, after it (twice), after the combine kernel
+spa_status launch_fused_decode(const spa_decode_args* a, void* ws_after_header, uint32_t* status, cudaStream_t st,
+                               void* const* events);
 
 // attend.cu
 struct AttendParams {

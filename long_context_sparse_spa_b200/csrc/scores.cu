@@ -91,7 +91,10 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
         const uint4* krow = kidx + size_t(kvu) * M * 2 + half;
         float* out_base = NQ == 1 ? scores + size_t(kvu) * M : scores + (size_t(b) * Hq + size_t(g) * G) * M;
 
-        for (int nb = n0 + pair; nb < n1; nb += kRowsPerPass * kLrUnroll) {
+        // every lane runs the same number of passes (the shuffle below needs the whole warp),
+        // rows past the chunk are masked
+        for (int pb = n0; pb < n1; pb += kRowsPerPass * kLrUnroll) {
+            const int nb = pb + pair;
             uint4 w[kLrUnroll];
 #pragma unroll
             for (int i = 0; i < kLrUnroll; ++i) {

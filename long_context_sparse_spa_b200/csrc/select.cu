@@ -37,7 +37,7 @@ constexpr int kSelThreads = 512;
 constexpr int kPerMax = 2048 / kSelThreads;   // histogram bins per thread in a scan
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 16;   // 16 is a non-portable cluster size, allowed on sm_100
 constexpr double kInvMassScale = 1.0 / 1099511627776.0;   // 2^-40
 
 using u64 = unsigned long long;
@@ -63,6 +63,7 @@ struct SelShared {
     u64 found_above_mass;
     double found_above_f64;
     uint32_t found_cnt;
+    Level0Shared l0;
 };
 
 // Block-wide exclusive scan of (a, b) in thread order; totals returned too.  Fixed order.
@@ -230,59 +231,14 @@ select_kernel(SelectParams p, int chunk, int resident) {
     uint32_t b0 = max_key >> 21, cum_cnt0 = 0;
     double cum_mass0 = 0.0;
     if (thresholded) {
-        if (tid == 0) {
-            sh.found_bin = b0;
-            sh.found_above_cnt = 0;
-            sh.found_above_f64 = 0.0;
-        }
-        constexpr int per = kBins / kSelThreads;   // bins per thread, descending
-        uint32_t vc[per];
-        double vm[per];
-        uint32_t sc = 0;
-        double sm = 0.0;
-        u64 mb[per];
-#pragma unroll
-        for (int j = 0; j < per; ++j) {
-            const int bin = kBins - 1 - (tid * per + j);
-            vc[j] = __ldcg(hc + bin);
-            mb[j] = TOPP ? __ldcg(hm + bin) : 0ull;
-        }
-#pragma unroll
-        for (int j = 0; j < per; ++j) {
-            const int bin = kBins - 1 - (tid * per + j);
-            vm[j] = 0.0;
-            // fp64 exp only in warps that hold mass (most bins are empty)
-            if (TOPP && __any_sync(0xffffffffu, mb[j] != 0) && mb[j])
-                vm[j] = double(mb[j]) * kInvMassScale * exp(double(bin_top_score(bin)) - double(m));
-            sc += vc[j];
-            sm += vm[j];
-        }
-        uint32_t ec, tc;
-        double em, tm;
-        block_exscan<double>(sc, sm, ec, em, tc, tm, sh.warp_u32, sh.warp_f64);
+        const Level0 l0 = level0_crossing(hc, hm, max_key, TOPP, p.topp, p.topk, sh.l0);
+        b0 = l0.bin;
+        cum_cnt0 = l0.above_cnt;
+        cum_mass0 = l0.above_mass;
         if (TOPP) {
-            Z = tm;
+            Z = l0.Z;
             T = double(p.topp) * Z;
         }
-        uint32_t ac = ec;
-        double am = em;
-#pragma unroll
-        for (int j = 0; j < per; ++j) {
-            const bool hit = TOPP ? (am < T && am + vm[j] >= T)
-                                  : (ac < uint32_t(p.topk) && ac + vc[j] >= uint32_t(p.topk));
-            if (hit) {
-                sh.found_bin = uint32_t(kBins - 1 - (tid * per + j));
-                sh.found_above_cnt = ac;
-                sh.found_above_f64 = am;
-            }
-            ac += vc[j];
-            am += vm[j];
-        }
-        __syncthreads();
-        b0 = sh.found_bin;
-        cum_cnt0 = sh.found_above_cnt;
-        cum_mass0 = sh.found_above_f64;
-        __syncthreads();
     }
     const float r0 = bin_top_score(b0);                       // mass reference inside B0
     const double scale0 = TOPP ? kInvMassScale * exp(double(r0) - double(m)) : 0.0;
@@ -707,7 +663,8 @@ SelectConfig choose(int U, int M) {
     const size_t fixed = align_up(sizeof(SelShared), 16);
     SelectConfig best{};
     best.C = 0;
-    // largest cluster (<= 8) that keeps every unit's cluster in one wave and >= 2048 scores per CTA
+    // largest cluster (<= 16) that keeps every unit's cluster in one wave and >= 2048 scores per CTA
+    cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     for (int C = kMaxCluster; C >= 1; C /= 2) {
         if (C > 1 && (M + C - 1) / C < 2048) continue;
         const int chunk = ((M + C - 1) / C + 3) / 4 * 4;
@@ -731,6 +688,7 @@ SelectConfig choose(int U, int M) {
 template <bool TOPP>
 spa_status launch_t(const SelectParams& p, cudaStream_t st) {
     const SelectConfig c = choose<TOPP>(p.U, p.M);
+    SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(c.C, p.U, 1);
