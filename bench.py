@@ -51,8 +51,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
-    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS) + ["c5"],
-                    help="decode workload (default), or c5: the selection-block-shared prefill")
+    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS) + ["c5", "c5q"],
+                    help="decode workload (default); c5: the selection-block-shared prefill; c5q: the per-query "
+                         "prefill (b_sel = 1) on the last 1024 queries of the c5 chunk")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--local-fraction", type=float, default=0.0,
                     help="head-wise routing: this fraction of every sequence's units is local (sink + window)")
@@ -538,10 +539,11 @@ def prefill_captured_mass(cfg, x, idx, counts):
 
 def run_prefill(a):
     """--config c5: the selection-block-shared prefill (one chunk of T queries), in TFLOP/s of
-    its algorithmic flops; the L2 is flushed before every step."""
+    its algorithmic flops; c5q: the per-query prefill (one support per query) on the last 1024
+    queries of the same chunk; the L2 is flushed before every step."""
     import oracle
 
-    cfg = C5
+    cfg = C5 if a.config == "c5" else C5.with_(name="c5q", T=1024, q_start=C5.N - 1024, bq=1)
     if a.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return 0
     x = prefill_inputs(cfg)
@@ -571,8 +573,8 @@ def run_prefill(a):
 
     plan = spa.prefill(Q=bf16_dev(x["Q"]), q_idx=bf16_dev(x["q_idx"]), K=bf16_dev(x["K"]), V=bf16_dev(x["V"]),
                        Kidx=bf16_dev(x["Kidx"]), q_start=cfg.q_start, score_scale=float(np.float32(cfg.score_scale)),
-                       sm_scale=float(np.float32(cfg.sm_scale)), topk=cfg.topk, sink=cfg.sink, want_f32=False,
-                       run=False)
+                       sm_scale=float(np.float32(cfg.sm_scale)), topk=cfg.topk, sink=cfg.sink, bq=cfg.bq,
+                       want_f32=False, run=False)
     wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
     for _ in range(a.warmup):
@@ -633,7 +635,8 @@ def run_prefill(a):
         dt = time.perf_counter() - t0
         cpu = {"value": cf / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": f"{done} (query block, kv head) units of {cfg.name}, fp64 oracle, {dt:.1f} s"}
-    out = {"metric": "sparse-prefill TFLOP/s (algorithmic), selection-block-shared", "value": tflops,
+    kind = "selection-block-shared" if cfg.bq > 1 else "per-query (b_sel = 1)"
+    out = {"metric": f"sparse-prefill TFLOP/s (algorithmic), {kind}", "value": tflops,
            "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": {"workload": f"{cfg.name}: prefill chunk T={cfg.T} at q_start={cfg.q_start}, N={cfg.N}, "
@@ -647,14 +650,14 @@ def run_prefill(a):
            "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": int(sum(h.numel() * 2 for h in hq)),
                    "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms},
-           "gpu_launches": 6 * a.steps, "clocks": clocks, "cpu_baseline": cpu}
+           "gpu_launches": (6 if cfg.bq > 1 else 7) * a.steps, "clocks": clocks, "cpu_baseline": cpu}
     print(json.dumps(out))
     return 0
 
 
 def main():
     a = parse()
-    if a.config == "c5":
+    if a.config in ("c5", "c5q"):
         return run_prefill(a)
     if a.impl == "reference":
         return run_reference(a)

@@ -382,6 +382,25 @@ spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_byt
 size_t spa_prefill_workspace_bytes(const spa_prefill_args* a);
 
 /* ------------------------------------------------------------------------------------
+ * Per-query sparse prefill ("Oracle-Guided Sparse Prefill" 2.1 with b_sel = 1: every query
+ * has its own support; 2.2: head-collapsed indexer).  Same arguments as spa_prefill_shared
+ * with bq = 1.  For query t of the chunk (position q_start + t) and kv head g, unit
+ * u = t * Hkv + g:
+ *   index query = mean of q_idx over the G heads of g;
+ *   support     = exact top-k of score_scale * index_query . Kidx[g][n] over n < q_start + t,
+ *                 united with the sink [0, sink), ascending in idx[u], count[u] entries;
+ *   idx[u][count[u]] = q_start + t (the query's own position, which the attention also reads);
+ *   out[t][h]   = softmax(sm_scale * q K^T) V over the support and the own position.
+ * One query per support leaves no dense contraction: the path is the decode's scorer,
+ * selection and split-KV gather attention on K/V shared by all queries of the chunk.
+ * Requires d in {64, 128}, r = 16, G <= 16, q_start + T <= N, T * Hkv <= 8192 and
+ * cap >= min(N, topk + sink) + 1.  The workspace holds one score row of N per unit
+ * (T * Hkv * N * 4 bytes): chunk long prefills.  ws >= spa_prefill_per_query_workspace_bytes.
+ */
+spa_status spa_prefill_per_query(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream);
+size_t spa_prefill_per_query_workspace_bytes(const spa_prefill_args* a);
+
+/* ------------------------------------------------------------------------------------
  * Device status word of a workspace (sticky OR of SPA_ERR_* bits as (1 << code)).
  * Synchronises `stream`, copies the word to *bits and, if reset != 0, clears it.
  * Returns SPA_OK or SPA_ERR_CUDA.

@@ -324,22 +324,27 @@ class PrefillPlan:
     out_f32: Optional[torch.Tensor]
     keep: tuple
 
+    per_query: bool = False
+
     def run(self, stream: Optional[torch.cuda.Stream] = None) -> None:
-        check(lib().spa_prefill_shared(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()),
-                                       self.ws.numel(), _stream(stream)))
+        fn = lib().spa_prefill_per_query if self.per_query else lib().spa_prefill_shared
+        check(fn(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), _stream(stream)))
 
 
 def prefill(*, Q: torch.Tensor, q_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, Kidx: torch.Tensor,
             q_start: int, score_scale: float, sm_scale: float, topk: int, sink: int, bq: int = 64,
             want_f32: bool = True, run: bool = True) -> PrefillPlan:
-    """Selection-block-shared prefill of one query chunk; see spa_prefill_shared in include/spa.h.
+    """Sparse prefill of one query chunk.  bq = 64: one support per 64 queries
+    (spa_prefill_shared in include/spa.h); bq = 1: one support per query
+    (spa_prefill_per_query; idx[u][count[u]] then holds the query's own position).
     Q [T, Hq, d], q_idx [T, Hq, r], K/V [Hkv, N, d], Kidx [Hkv, N, r], all bf16."""
     for t, n in ((Q, "Q"), (q_idx, "q_idx"), (K, "K"), (V, "V"), (Kidx, "Kidx")):
         _need(t, torch.bfloat16, n)
     T, Hq, d = Q.shape
     Hkv, N, _ = K.shape
     U = (T // bq) * Hkv
-    cap = min(N, topk + sink)
+    per_query = bq == 1
+    cap = min(N, topk + sink) + (1 if per_query else 0)
     dev = Q.device
     idx = torch.full((U, max(cap, 1)), -1, dtype=torch.int32, device=dev)
     count = torch.zeros(U, dtype=torch.int32, device=dev)
@@ -353,8 +358,10 @@ def prefill(*, Q: torch.Tensor, q_idx: torch.Tensor, K: torch.Tensor, V: torch.T
     a.topk, a.sink = topk, sink
     a.idx, a.count, a.cap = _ptr(idx), _ptr(count), cap
     a.out, a.out_f32 = _ptr(out), _ptr(out32)
-    ws = workspace(lib().spa_prefill_workspace_bytes(ctypes.byref(a)), dev)
-    plan = PrefillPlan(a, ws, idx, count, out, out32, (Q, q_idx, K, V, Kidx))
+    nbytes = (lib().spa_prefill_per_query_workspace_bytes if per_query else lib().spa_prefill_workspace_bytes)(
+        ctypes.byref(a))
+    ws = workspace(nbytes, dev)
+    plan = PrefillPlan(a, ws, idx, count, out, out32, (Q, q_idx, K, V, Kidx), per_query)
     if run:
         plan.run()
     return plan

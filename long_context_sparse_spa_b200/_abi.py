@@ -94,6 +94,8 @@ SIGNATURES = {
     "spa_read_device_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32), _i]),
     "spa_prefill_shared": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
     "spa_prefill_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
+    "spa_prefill_per_query": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
+    "spa_prefill_per_query_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
 }
 
 _LIB = None

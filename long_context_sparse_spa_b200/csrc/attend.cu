@@ -58,12 +58,12 @@ __device__ __forceinline__ UnitGeom unit_geom(const AttendParams& p, int u, int 
         const int kvh = u - g.b * p.Hkv;
         g.h0 = kvh * G;
         g.bh = g.b * p.Hkv + kvh;
-        g.kv = size_t(g.bh) * size_t(p.N);
+        g.kv = size_t(p.kv_shared ? kvh : g.bh) * size_t(p.N);
     } else {
         g.b = u / p.Hq;
         g.h0 = u - g.b * p.Hq;
         g.bh = g.b * p.Hkv + g.h0 / G;
-        g.kv = size_t(g.bh) * size_t(p.N);
+        g.kv = size_t(p.kv_shared ? g.h0 / G : g.bh) * size_t(p.N);
     }
     g.nh = nh;
     int c = p.count[u];

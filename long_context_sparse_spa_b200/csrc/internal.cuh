@@ -251,9 +251,10 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // hist (optional, GROUP_MEAN only): also accumulate the level-0 histogram of the scores;
 // with_mass adds the fixed-point masses (top-p), else counts only.
 // local (optional, GROUP_MEAN): [B * Hkv] flags of units that are not scored (head-wise routing)
+// kv_shared: the key set [Hkv][M] is shared by every batch row (per-query prefill), else [B][Hkv][M]
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
                                  int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
-                                 cudaStream_t st, const uint8_t* local = nullptr);
+                                 cudaStream_t st, const uint8_t* local = nullptr, bool kv_shared = false);
 // kind: SPA_SCORE_TAYLOR_BLOCK (mean, var), SPA_SCORE_MINMAX_BLOCK (min, max) or
 // SPA_SCORE_MEAN_BLOCK (mean; var not read); stats_bf16: the statistics are bf16, else fp32
 spa_status launch_taylor_scores(const uint16_t* q, const void* mean, const void* var, int B, int Hq, int Hkv,
@@ -320,6 +321,8 @@ struct AttendParams {
     int* unit_ctas;    // [U][2]: first and last CTA of a unit split over several CTAs, else -1
     float* partials;   // [(U + grid) * heads_per_unit * (d + 2)]; the RLA partials follow
     uint32_t* status;
+    // kv_shared: K and V are [Hkv, N, d], shared by every batch row (per-query prefill)
+    int kv_shared;
     // residual linear attention (null rla_S: off): state S [B*Hkv][d][d], z [B*Hkv][d],
     // RMSNorm scale gamma [Hq][d] and epsilon
     const float* rla_S;

@@ -28,7 +28,7 @@ template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
 lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict__ kidx, int Hq, int Hkv,
                       int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items, Hist0 hist,
-                      const uint8_t* __restrict__ local) {
+                      const uint8_t* __restrict__ local, int kv_shared) {
     pdl_enter();
     const int G = Hq / Hkv;
     const int half = threadIdx.x & 1;          // which 8 of the 16 index dims this lane holds
@@ -88,7 +88,8 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
 
         const int n0 = chunk * kLrChunk;
         const int n1 = min(M, n0 + kLrChunk);
-        const uint4* krow = kidx + size_t(kvu) * M * 2 + half;
+        // kv_shared: one key set [Hkv][M] serves every batch row (per-query prefill)
+        const uint4* krow = kidx + size_t(kv_shared ? g : kvu) * M * 2 + half;
         float* out_base = NQ == 1 ? scores + size_t(kvu) * M : scores + (size_t(b) * Hq + size_t(g) * G) * M;
 
         // every lane runs the same number of passes (the shuffle below needs the whole warp),
@@ -443,7 +444,7 @@ int grid_for(int items, int per_sm) {
 
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
                                  int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
-                                 cudaStream_t st, const uint8_t* local) {
+                                 cudaStream_t st, const uint8_t* local, bool kv_shared) {
     const int G = Hq / Hkv;
     const int chunks = (M + kLrChunk - 1) / kLrChunk;
     const int items = B * Hkv * chunks;
@@ -454,14 +455,14 @@ spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int
         auto kern = hist && with_mass ? lowrank_scores_kernel<1, true, true>
                                       : (hist ? lowrank_scores_kernel<1, true, false> : lowrank_scores_kernel<1, false, false>);
         SPA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kLrThreads), 0, st, qidx, k4, Hq, Hkv, M, scale, scores, chunks,
-                                items, h, local));
+                                items, h, local, kv_shared ? 1 : 0));
     } else {
         if (hist) return SPA_ERR_INVALID_ARG;
         switch (G) {
 #define SPA_LR_CASE(n)                                                                                          \
     case n:                                                                                                     \
         SPA_CUDA_TRY(launch_pdl(lowrank_scores_kernel<n, false, false>, dim3(grid), dim3(kLrThreads), 0, st, qidx, \
-                                k4, Hq, Hkv, M, scale, scores, chunks, items, h, nullptr));                     \
+                                k4, Hq, Hkv, M, scale, scores, chunks, items, h, nullptr, kv_shared ? 1 : 0));  \
         break;
             SPA_LR_CASE(1) SPA_LR_CASE(2) SPA_LR_CASE(4) SPA_LR_CASE(8) SPA_LR_CASE(16)
 #undef SPA_LR_CASE
