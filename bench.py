@@ -537,6 +537,21 @@ def prefill_captured_mass(cfg, x, idx, counts):
                    f"block's own rows ({time.perf_counter() - t0:.1f} s on {cores} host threads)"}
 
 
+def pq_roofline(cfg, counts, ms):
+    """Per-query prefill: a gather per (query, kv head), bound by memory.  Algorithmic bytes per
+    step: every unit's index keys before its query (32 B each) and its gathered K/V rows
+    (support + own position, 512 B each); most re-reads are L2 hits, so the fraction of the HBM
+    copy peak can exceed 1."""
+    hbm, kind = peaks()
+    keys = sum(cfg.q_start + u // cfg.Hkv for u in range(cfg.U))
+    rows = int(counts.sum()) + cfg.U
+    byts = keys * cfg.r * 2 + rows * KV_ROW_BYTES(cfg.d)
+    ach = byts / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "per-query prefill (all kernels of the step)", "achieved": ach, "peak": hbm,
+            "unit": "GB/s", "frac": ach / hbm, "peak_source": kind, "traffic": None,
+            "algorithmic_bytes_per_step": byts}
+
+
 def run_prefill(a):
     """--config c5: the selection-block-shared prefill (one chunk of T queries), in TFLOP/s of
     its algorithmic flops; c5q: the per-query prefill (one support per query) on the last 1024
@@ -644,9 +659,9 @@ def run_prefill(a):
                       "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
                       "support_mean": float(counts.mean()), "algorithmic_gflop_per_step": flops / 1e9,
                       "sparsity": round(float(prefill_sparsity(cfg, counts)), 4), "captured_mass": mass},
-           "roofline": {"bound": "tensor", "kernel": "prefill (all kernels of the step)", "achieved": tflops,
-                        "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
-                        "traffic": None},
+           "roofline": ({"bound": "tensor", "kernel": "prefill (all kernels of the step)", "achieved": tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
+                         "traffic": None} if cfg.bq > 1 else pq_roofline(cfg, counts, ms)),
            "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": int(sum(h.numel() * 2 for h in hq)),
                    "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms},

@@ -401,6 +401,49 @@ spa_status spa_prefill_per_query(const spa_prefill_args* a, void* ws, size_t ws_
 size_t spa_prefill_per_query_workspace_bytes(const spa_prefill_args* a);
 
 /* ------------------------------------------------------------------------------------
+ * Permuted block-sparse prefill ("Sparser Block-Sparse Attention via Token Permutation"
+ * (PBS-Attn), sections 1-4) of a causal sequence of T tokens: queries and keys at positions
+ * 0 .. T-1.  Per kv head g:
+ *   importance[g][n] = mean, over the last query block's b queries and the G heads of g, of
+ *                      their causal softmax probability softmax(sm_scale * q . k)[n]
+ *                      (0 for keys after a query); fp32;
+ *   perm[g][s0 + i]  = inside each segment [s0, s0 + S) (the last may be shorter), the keys'
+ *                      original positions sorted by descending importance, equal importance by
+ *                      ascending position;
+ * per query block j (queries [t0, t0 + b), t0 = j * b, segment start seg0 = t0 / S * S) and kv
+ * head g, unit u = j * Hkv + g:
+ *   the key blocks are the blocks of b consecutive permuted keys in segments 0 .. seg0/S - 1,
+ *   scored sm_scale * qbar . kbar (qbar: mean of the block's b x G queries; kbar: mean of the
+ *   key block; mean pooling); the top-k blocks (score desc, block asc) are kept, none forced;
+ *   idx[u]  = the kept blocks' original positions, ascending (count[u] = kept blocks * b);
+ *   out[t][h] = softmax(sm_scale * q K^T) V over the support, the own segment's keys
+ *              [seg0, t0) and the block's own positions up to t (causal), on tcgen05.
+ * Queries are not permuted, so no inverse permutation of the output is needed.
+ * Requires d = 128, b = 64, G = Hq / Hkv even and <= 8, T and S multiples of b, S <= 8192,
+ * topk * b <= 8192, cap >= topk * b.  ws >= spa_pbs_workspace_bytes.
+ */
+typedef struct spa_pbs_args {
+    int T, Hq, Hkv, d;
+    int b;                    /* block size: 64 */
+    int S;                    /* segment size */
+    int topk;                 /* key blocks kept per query block */
+    float sm_scale;
+    const uint16_t* Q;        /* [T, Hq, d] */
+    const uint16_t* K;        /* [Hkv, T, d] */
+    const uint16_t* V;        /* [Hkv, T, d] */
+    float* importance;        /* [Hkv, T] out (optional) */
+    int32_t* perm;            /* [Hkv, T] out */
+    int32_t* idx;             /* [U, cap] out, U = (T / b) * Hkv */
+    int32_t* count;           /* [U] out */
+    int cap;
+    uint16_t* out;            /* [T, Hq, d] out */
+    float* out_f32;           /* optional */
+} spa_pbs_args;
+
+spa_status spa_pbs_prefill(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream);
+size_t spa_pbs_workspace_bytes(const spa_pbs_args* a);
+
+/* ------------------------------------------------------------------------------------
  * Device status word of a workspace (sticky OR of SPA_ERR_* bits as (1 << code)).
  * Synchronises `stream`, copies the word to *bits and, if reset != 0, clears it.
  * Returns SPA_OK or SPA_ERR_CUDA.

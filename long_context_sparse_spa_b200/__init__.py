@@ -19,14 +19,14 @@ import torch
 
 from ._abi import (SPA_COLLAPSE_GROUP_MEAN, SPA_COLLAPSE_NONE, SPA_DECODE_AUTO, SPA_DECODE_FUSED, SPA_DECODE_SEPARATE,
                    SPA_SCORE_LOWRANK, SPA_SCORE_MEAN_BLOCK,
-                   SPA_SCORE_MINMAX_BLOCK, SPA_SCORE_TAYLOR_BLOCK, SPA_SELECT_TOPK, SPA_STATS_BF16, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPrefillArgs, check, lib, lib_path)
+                   SPA_SCORE_MINMAX_BLOCK, SPA_SCORE_TAYLOR_BLOCK, SPA_SELECT_TOPK, SPA_STATS_BF16, SPA_SELECT_TOPP, SpaDecodeArgs, SpaError, SpaPbsArgs, SpaPrefillArgs, check, lib, lib_path)
 
 __all__ = [
     "SpaError", "lib", "lib_path", "block_stats", "index_scores", "select_topk", "select_topp", "sparse_attend",
     "decode", "DecodePlan", "workspace", "read_device_status", "select_topp_static", "prefill", "PrefillPlan", "SPA_COLLAPSE_NONE", "SPA_COLLAPSE_GROUP_MEAN",
     "SPA_SCORE_LOWRANK", "SPA_SCORE_TAYLOR_BLOCK", "SPA_SCORE_MINMAX_BLOCK", "SPA_SCORE_MEAN_BLOCK",
     "SPA_SELECT_TOPK", "SPA_SELECT_TOPP", "SPA_STATS_BF16", "block_minmax", "rla_state",
-    "SPA_DECODE_AUTO", "SPA_DECODE_SEPARATE", "SPA_DECODE_FUSED",
+    "SPA_DECODE_AUTO", "SPA_DECODE_SEPARATE", "SPA_DECODE_FUSED", "pbs_prefill", "PbsPlan",
 ]
 
 
@@ -362,6 +362,55 @@ def prefill(*, Q: torch.Tensor, q_idx: torch.Tensor, K: torch.Tensor, V: torch.T
         ctypes.byref(a))
     ws = workspace(nbytes, dev)
     plan = PrefillPlan(a, ws, idx, count, out, out32, (Q, q_idx, K, V, Kidx), per_query)
+    if run:
+        plan.run()
+    return plan
+
+
+# ----------------------------------------------------------------------------- PBS-Attn prefill
+@dataclass
+class PbsPlan:
+    """Arguments, outputs and workspace of one permuted block-sparse prefill, reusable."""
+
+    args: SpaPbsArgs
+    ws: torch.Tensor
+    importance: torch.Tensor
+    perm: torch.Tensor
+    idx: torch.Tensor
+    count: torch.Tensor
+    out: torch.Tensor
+    out_f32: Optional[torch.Tensor]
+    keep: tuple
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        check(lib().spa_pbs_prefill(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
+                                    _stream(stream)))
+
+
+def pbs_prefill(*, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, sm_scale: float, S: int, topk: int,
+                b: int = 64, want_f32: bool = True, run: bool = True) -> PbsPlan:
+    """Permuted block-sparse prefill of a causal sequence; see spa_pbs_prefill in include/spa.h.
+    Q [T, Hq, d], K/V [Hkv, T, d] bf16."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n)
+    T, Hq, d = Q.shape
+    Hkv = K.shape[0]
+    U = (T // b) * Hkv
+    cap = max(topk * b, 1)
+    dev = Q.device
+    imp = torch.empty((Hkv, T), dtype=torch.float32, device=dev)
+    perm = torch.empty((Hkv, T), dtype=torch.int32, device=dev)
+    idx = torch.full((U, cap), -1, dtype=torch.int32, device=dev)
+    count = torch.zeros(U, dtype=torch.int32, device=dev)
+    out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=dev)
+    out32 = torch.empty((T, Hq, d), dtype=torch.float32, device=dev) if want_f32 else None
+    a = SpaPbsArgs()
+    a.T, a.Hq, a.Hkv, a.d, a.b, a.S, a.topk, a.sm_scale = T, Hq, Hkv, d, b, S, topk, sm_scale
+    a.Q, a.K, a.V = _ptr(Q), _ptr(K), _ptr(V)
+    a.importance, a.perm, a.idx, a.count, a.cap = _ptr(imp), _ptr(perm), _ptr(idx), _ptr(count), cap
+    a.out, a.out_f32 = _ptr(out), _ptr(out32)
+    ws = workspace(lib().spa_pbs_workspace_bytes(ctypes.byref(a)), dev)
+    plan = PbsPlan(a, ws, imp, perm, idx, count, out, out32, (Q, K, V))
     if run:
         plan.run()
     return plan

@@ -69,6 +69,16 @@ class SpaPrefillArgs(ctypes.Structure):
     ]
 
 
+class SpaPbsArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", _i), ("Hq", _i), ("Hkv", _i), ("d", _i),
+        ("b", _i), ("S", _i), ("topk", _i), ("sm_scale", _f),
+        ("Q", _p), ("K", _p), ("V", _p),
+        ("importance", _p), ("perm", _p), ("idx", _p), ("count", _p), ("cap", _i),
+        ("out", _p), ("out_f32", _p),
+    ]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "spa_status_string": (ctypes.c_char_p, [_i]),
@@ -95,6 +105,8 @@ SIGNATURES = {
     "spa_prefill_shared": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
     "spa_prefill_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
     "spa_prefill_per_query": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
+    "spa_pbs_prefill": (_i, [ctypes.POINTER(SpaPbsArgs), _p, _sz, _p]),
+    "spa_pbs_workspace_bytes": (_sz, [ctypes.POINTER(SpaPbsArgs)]),
     "spa_prefill_per_query_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
 }
 

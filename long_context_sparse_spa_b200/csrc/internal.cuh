@@ -294,6 +294,23 @@ spa_status launch_rla_state(const uint16_t* K, const uint16_t* V, int BH, int N,
 // prefill.cu
 size_t prefill_scratch_bytes(int U, int N);
 spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st);
+// The tcgen05 attention of 64-query blocks: unit u = block * Hkv + g attends, for each of its 64
+// queries (positions q_start + block * 64 + i) and G heads, to the rows idx[u][0 .. count[u])
+// and to the block's own positions up to the query (causal).  d = 128, G even.
+struct PrefillAttendParams {
+    const uint16_t* Q;     // [T, Hq, d]
+    const uint16_t* K;     // [Hkv, N, d]
+    const uint16_t* V;
+    const int32_t* idx;    // [U, cap]
+    const int32_t* count;  // [U]
+    int cap;
+    int Hq, Hkv, N, bq, q_start;
+    float sm_scale;
+    uint16_t* out;         // [T, Hq, d]
+    float* out_f32;
+    uint32_t* status;
+};
+spa_status launch_prefill_attend(const PrefillAttendParams& pp, int U, cudaStream_t st);
 
 // fused.cu: the persistent dataflow decode (low-rank, head-collapsed, d = 128, G <= 8)
 bool fused_decode_supported(const spa_decode_args* a);

@@ -174,20 +174,6 @@ prefill_scores_kernel(const float* __restrict__ qhat, const int32_t* __restrict_
 }
 
 // ============================================================================ attention
-struct PrefillAttendParams {
-    const uint16_t* Q;     // [T, Hq, d]
-    const uint16_t* K;     // [Hkv, N, d]
-    const uint16_t* V;
-    const int32_t* idx;    // [U, cap]
-    const int32_t* count;  // [U]
-    int cap;
-    int Hq, Hkv, N, bq, q_start;
-    float sm_scale;
-    uint16_t* out;         // [T, Hq, d]
-    float* out_f32;
-    uint32_t* status;
-};
-
 struct __align__(1024) PfShared {
     uint8_t q[kTileBytes];
     uint8_t k[kTileBytes];
@@ -462,9 +448,13 @@ spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) 
 
     PrefillAttendParams pp{a->Q, a->K, a->V, a->idx, a->count, a->cap, a->Hq, a->Hkv, a->N, a->bq, a->q_start,
                            a->sm_scale, a->out, a->out_f32, status};
+    return launch_prefill_attend(pp, U, st);
+}
+
+spa_status launch_prefill_attend(const PrefillAttendParams& pp, int U, cudaStream_t st) {
     const size_t smem = sizeof(PfShared);
     SPA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    SPA_CUDA_TRY(launch_pdl(prefill_attend_kernel, dim3(U, G / 2), dim3(kPfThreads), smem, st, pp));
+    SPA_CUDA_TRY(launch_pdl(prefill_attend_kernel, dim3(U, pp.Hq / pp.Hkv / 2), dim3(kPfThreads), smem, st, pp));
     return SPA_OK;
 }
 

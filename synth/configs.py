@@ -166,6 +166,49 @@ class PrefillConfig:
         return replace(self, **kw)
 
 
+@dataclass(frozen=True)
+class PbsConfig:
+    """Permuted block-sparse prefill (PBS-Attn) of a causal sequence of T tokens: blocks of b
+    queries and keys, segments of S keys, top-k key blocks per query block.  Keys are N(0, 1)
+    with, in every segment before the last, b heavy keys at scattered positions aligned with
+    the group's mean query of the last block (the structure the in-segment permutation is
+    meant to gather into one block)."""
+
+    name: str
+    seed: int
+    T: int
+    Hq: int
+    Hkv: int
+    d: int = 128
+    b: int = 64
+    S: int = 256
+    topk: int = 2
+    heavy_amp: float = 3.0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def n_blocks(self) -> int:
+        return self.T // self.b
+
+    @property
+    def U(self) -> int:
+        return self.n_blocks * self.Hkv
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def with_(self, **kw) -> "PbsConfig":
+        return replace(self, **kw)
+
+
+PBS_SMALL = PbsConfig(name="pbs_small", seed=5, T=1024, Hq=8, Hkv=2, S=256, topk=2)
+PBS_32K = PbsConfig(name="pbs_32k", seed=6, T=32768, Hq=32, Hkv=8, S=2048, topk=32)
+
+
 C1 = DecodeConfig(
     name="c1", seed=0, B=1, Hq=4, Hkv=1, d=64, N=4096, score="lowrank", select="topk",
     collapse="head", sink=4, window=64, topk=256, keys="needles", n_needles=8, needle_amp=4.0)

@@ -30,7 +30,7 @@ from typing import Dict, Iterable, Optional, Tuple
 
 import numpy as np
 
-from .configs import DecodeConfig, PrefillConfig
+from .configs import DecodeConfig, PbsConfig, PrefillConfig
 
 BF16 = np.uint16
 
@@ -218,3 +218,27 @@ def prefill_inputs(cfg: PrefillConfig) -> Dict[str, np.ndarray]:
         V[g] = bf16_bits(_rng(cfg.seed, 4, 0, g).standard_normal((N, d), dtype=np.float32))
         Kidx[g] = _project(K[g], P)
     return {"Q": Q, "q_idx": q_idx, "K": K, "V": V, "Kidx": Kidx, "P": P}
+
+
+def pbs_inputs(cfg: PbsConfig) -> Dict[str, np.ndarray]:
+    """Inputs of a permuted block-sparse prefill: Q [T, Hq, d], K, V [Hkv, T, d] (bf16 bits).
+
+    Q, V ~ N(0, 1).  K ~ N(0, 1), except that every segment before the last holds b heavy keys
+    at scattered positions, k = heavy_amp * qbar_g / |qbar_g| + 0.3 N(0, 1), with qbar_g the mean
+    of the last query block's queries of kv head g."""
+    T, Hq, Hkv, d, G, b, S = cfg.T, cfg.Hq, cfg.Hkv, cfg.d, cfg.G, cfg.b, cfg.S
+    Q = bf16_bits(_rng(cfg.seed, 1).standard_normal((T, Hq, d), dtype=np.float32))
+    Qf = bf16_value(Q).astype(np.float64)
+    K = np.zeros((Hkv, T, d), np.uint16)
+    V = np.zeros((Hkv, T, d), np.uint16)
+    for g in range(Hkv):
+        rng = _rng(cfg.seed, 2, g)
+        k = rng.standard_normal((T, d), dtype=np.float32)
+        qbar = Qf[T - b:, g * G:(g + 1) * G].reshape(-1, d).mean(0)
+        unit = qbar / np.linalg.norm(qbar)
+        for s0 in range(0, (T - 1) // S * S, S):
+            pos = s0 + np.sort(rng.choice(S, b, replace=False))
+            k[pos] = (cfg.heavy_amp * unit[None, :] + 0.3 * rng.standard_normal((b, d))).astype(np.float32)
+        K[g] = bf16_bits(k)
+        V[g] = bf16_bits(_rng(cfg.seed, 3, g).standard_normal((T, d), dtype=np.float32))
+    return {"Q": Q, "K": K, "V": V}

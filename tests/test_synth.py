@@ -39,3 +39,17 @@ def test_block_generator_and_prefill_shapes():
     assert x["K"].shape == (2, 2, 64 * 300 + 17, 128) and "Kidx" not in x
     p = prefill_inputs(SMALL["c5s"])
     assert p["Q"].shape == (1024, 8, 128) and p["Kidx"].shape == (2, 4096, 16)
+
+
+def test_pbs_inputs_are_seeded_and_plant_heavy_keys():
+    from synth import PBS_SMALL, pbs_inputs
+    a, b2 = pbs_inputs(PBS_SMALL), pbs_inputs(PBS_SMALL)
+    for k in a:
+        assert np.array_equal(a[k], b2[k])
+    cfg = PBS_SMALL
+    assert a["Q"].shape == (cfg.T, cfg.Hq, cfg.d) and a["K"].shape == (cfg.Hkv, cfg.T, cfg.d)
+    # every full segment before the last holds b keys far longer than the N(0, 1) ones
+    Kf = bf16_value(a["K"][0]).astype(np.float64)
+    norms = np.linalg.norm(Kf, axis=1)
+    for s0 in range(0, cfg.T - cfg.S, cfg.S):
+        assert np.sum(norms[s0:s0 + cfg.S] > 0.5 * (norms.mean() + cfg.heavy_amp)) >= cfg.b // 2
