@@ -81,6 +81,22 @@ const char* spa_status_string(int status);
 /* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
 const char* spa_last_cuda_error(void);
 
+/* Test hook of the failure-detection path (the method pages have no counterpart): every wait
+ * inside the kernels is bounded and, when its bound runs out, raises SPA_ERR_TIMEOUT in the
+ * device status word and leaves the kernel in a defined state.  With a bit set, the next
+ * launches of that kernel arm their completion barrier for an arrival that is never issued
+ * (nothing is left in flight), use a short bound, and so take that path:
+ *   SPA_TEST_STALL_SELECT_LOAD  the selection's bulk load of its chunk of scores; the CTA
+ *                               then reads the scores from global memory, so its results
+ *                               stay those of a normal run;
+ *   SPA_TEST_STALL_PREFILL_MMA  the tcgen05 prefill's first S = Q K^T; the CTA writes no
+ *                               output and frees its tensor memory.
+ * Process-wide; bits = 0 restores normal launches.  Returns SPA_ERR_INVALID_ARG for unknown
+ * bits.  Not for production use. */
+#define SPA_TEST_STALL_SELECT_LOAD 1
+#define SPA_TEST_STALL_PREFILL_MMA 2
+spa_status spa_test_stall(int bits);
+
 /* ABI version of this header: 6 (spa_decode_args gained local_units in 2, the RLA fields in 3;
  * the min-max and mean block scores and spa_block_minmax came in 4; bf16 statistics in 5;
  * spa_select_static_status in 6). */

@@ -27,6 +27,8 @@ SPA_STATS_BF16 = 0x100
 SPA_SELECT_TOPK = 0
 SPA_SELECT_TOPP = 1
 SPA_SELECT_STATIC_MAX_UNITS = 16
+SPA_TEST_STALL_SELECT_LOAD = 1
+SPA_TEST_STALL_PREFILL_MMA = 2
 SPA_DECODE_AUTO = 0
 SPA_DECODE_SEPARATE = 1
 SPA_DECODE_FUSED = 2
@@ -84,6 +86,7 @@ SIGNATURES = {
     "spa_status_string": (ctypes.c_char_p, [_i]),
     "spa_last_cuda_error": (ctypes.c_char_p, []),
     "spa_abi_version": (_i, []),
+    "spa_test_stall": (_i, [_i]),
     "spa_block_stats": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _p]),
     "spa_index_scores": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p]),
     "spa_select_topk": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _p, _sz, _p]),

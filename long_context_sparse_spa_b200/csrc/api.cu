@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/spa.h: argument validation, workspace
 // layout and kernel launches.  No entry point allocates device memory.
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -10,9 +11,12 @@ namespace spa {
 
 namespace {
 thread_local std::string g_last_cuda_error;
+std::atomic<int> g_test_stall{0};
 std::mutex g_info_mu;
 std::vector<DeviceInfo> g_info;
 }  // namespace
+
+int test_stall_bits() { return g_test_stall.load(std::memory_order_relaxed); }
 
 spa_status cuda_fail(cudaError_t e) {
     g_last_cuda_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
@@ -78,6 +82,12 @@ const char* spa_status_string(int s) {
 }
 
 const char* spa_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+spa_status spa_test_stall(int bits) {
+    if (bits & ~(SPA_TEST_STALL_SELECT_LOAD | SPA_TEST_STALL_PREFILL_MMA)) return SPA_ERR_INVALID_ARG;
+    g_test_stall.store(bits, std::memory_order_relaxed);
+    return SPA_OK;
+}
 
 int spa_abi_version(void) { return 6; }
 

@@ -189,7 +189,6 @@ struct FShared {
         } g;
     };
 };
-constexpr size_t kFSharedHead = (offsetof(FShared, s) + 127) / 128 * 128;
 static_assert(offsetof(FShared, s) % 128 == 0, "the cp.async / ldmatrix ring needs 16-byte aligned rows");
 
 // Block-wide exclusive scan of (a, b) in thread order, with totals.  Fixed order.

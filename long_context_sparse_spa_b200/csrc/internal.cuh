@@ -282,6 +282,7 @@ struct SelectParams {
     float* index_mass;
     uint32_t* status;
     const uint8_t* local;   // [U] or null: local units (head-wise routing) select only sink + window
+    int test_stall;         // SPA_TEST_STALL_* bits armed by spa_test_stall (test hook), else 0
 };
 spa_status launch_hist0(const SelectParams& p, bool with_mass, cudaStream_t st);
 spa_status launch_select(const SelectParams& p, bool topp, cudaStream_t st);
@@ -309,8 +310,12 @@ struct PrefillAttendParams {
     uint16_t* out;         // [T, Hq, d]
     float* out_f32;
     uint32_t* status;
+    int test_stall;        // SPA_TEST_STALL_* bits (test hook), else 0
 };
 spa_status launch_prefill_attend(const PrefillAttendParams& pp, int U, cudaStream_t st);
+
+// The test hook's armed bits (spa_test_stall), read by the launchers.
+int test_stall_bits();
 
 // fused.cu: the persistent dataflow decode (low-rank, head-collapsed, d = 128, G <= 8)
 bool fused_decode_supported(const spa_decode_args* a);

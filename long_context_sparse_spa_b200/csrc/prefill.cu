@@ -226,6 +226,11 @@ prefill_attend_kernel(PrefillAttendParams p) {
     const uint32_t t_s = tmem, t_o = tmem + 128;                 // S at columns 0..127, O at 128..255
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
     uint32_t phase = 0;
+    // the test hook stalls the first S = Q K^T: its completion barrier waits for an MMA that
+    // is never issued, so the bounded wait runs out with nothing in flight
+    const bool stall = (p.test_stall & SPA_TEST_STALL_PREFILL_MMA) != 0;
+    const uint32_t spin_limit = stall ? 1024u : kSpinLimit;
+    bool pending = false;   // an MMA commit issued and not yet observed (uniform over the CTA)
     const float sl2 = p.sm_scale * kLog2e;
     constexpr uint32_t kIdS = idesc_bf16(kPfRows, kPfKeys, false);
     constexpr uint32_t kIdO = idesc_bf16(kPfRows, 128, true);
@@ -266,7 +271,8 @@ prefill_attend_kernel(PrefillAttendParams p) {
     };
     // S = Q K^T into TMEM columns 0..127; every thread waits for completion
     auto mma_s = [&]() -> bool {
-        if (tid == 0) {
+        pending = !stall;
+        if (tid == 0 && !stall) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
@@ -278,14 +284,17 @@ prefill_attend_kernel(PrefillAttendParams p) {
         }
         return true;
     };
+    // bounded wait for the outstanding commit; on expiry the CTA stops (every later step checks
+    // sh.timed_out) and the commit stays owed, so TMEM is not freed under a running MMA
     auto wait_mma = [&]() {
         uint32_t it = 0;
         while (!mbar_try_wait(&sh.bar, phase)) {
-            if (++it >= kSpinLimit) {
+            if (++it >= spin_limit) {
                 atomicExch(&sh.timed_out, 1);
-                break;
+                return;
             }
         }
+        pending = false;
         phase ^= 1u;
         tc_fence_after();
     };
@@ -376,6 +385,7 @@ prefill_attend_kernel(PrefillAttendParams p) {
             }
             umma_commit(&sh.bar);
         }
+        pending = true;
         wait_mma();       // O ready; P, K and V may be overwritten
         tc_fence_before();
         if (stop()) break;
@@ -406,7 +416,16 @@ prefill_attend_kernel(PrefillAttendParams p) {
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    // after a give-up, an issued MMA may still be running: wait once more (bounded); TMEM is
+    // freed only when no commit is owed (a CTA that exits holding TMEM is the remaining hazard
+    // of a wait that never completes)
+    if (pending) {
+        uint32_t it = 0;
+        while (!mbar_try_wait(&sh.bar, phase) && ++it < spin_limit) {
+        }
+        pending = it >= spin_limit;
+    }
+    if (warp == 0 && !pending) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
@@ -420,7 +439,6 @@ size_t prefill_scratch_bytes(int U, int N) {
 }
 
 spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) {
-    const int G = a->Hq / a->Hkv;
     const int n_blocks = a->T / a->bq;
     const int U = n_blocks * a->Hkv;
     uint8_t* w = static_cast<uint8_t*>(ws);
@@ -451,7 +469,9 @@ spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) 
     return launch_prefill_attend(pp, U, st);
 }
 
-spa_status launch_prefill_attend(const PrefillAttendParams& pp, int U, cudaStream_t st) {
+spa_status launch_prefill_attend(const PrefillAttendParams& pp0, int U, cudaStream_t st) {
+    PrefillAttendParams pp = pp0;
+    pp.test_stall = test_stall_bits();
     const size_t smem = sizeof(PfShared);
     SPA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     SPA_CUDA_TRY(launch_pdl(prefill_attend_kernel, dim3(U, pp.Hq / pp.Hkv / 2), dim3(kPfThreads), smem, st, pp));

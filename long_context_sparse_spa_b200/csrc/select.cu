@@ -151,7 +151,7 @@ hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
 // ============================================================================ selection
 template <bool TOPP>
 __global__ void __launch_bounds__(kSelThreads, 2)
-select_kernel(SelectParams p, int chunk, int resident) {
+select_kernel(SelectParams p, int chunk, int resident_launch) {
     pdl_enter();
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
@@ -172,7 +172,10 @@ select_kernel(SelectParams p, int chunk, int resident) {
     // ---- the chunk into shared memory: bulk asynchronous copies when the row slice is
     // 16-byte aligned (they run while the level-0 scan below executes), else plain loads
     const int n16 = (reinterpret_cast<uintptr_t>(srow) & 15) == 0 ? (n & ~3) : 0;
-    const bool bulk = resident && n16 > 0;
+    const bool bulk = resident_launch && n16 > 0;
+    // the test hook stalls the chunk load: the barrier expects bytes no copy delivers
+    const bool stall = (p.test_stall & SPA_TEST_STALL_SELECT_LOAD) != 0;
+    const uint32_t spin_limit = stall ? 1024u : kLoadSpinLimit;
     const uint32_t bar = uint32_t(__cvta_generic_to_shared(&sh.load_bar));
     if (bulk) {
         if (tid == 0) {
@@ -181,7 +184,7 @@ select_kernel(SelectParams p, int chunk, int resident) {
             const uint32_t bytes = uint32_t(n16) * 4u;
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
             const uint32_t dst = uint32_t(__cvta_generic_to_shared(sv));
-            for (uint32_t off = 0; off < bytes; off += kBulkPiece) {
+            for (uint32_t off = 0; off < (stall ? 0u : bytes); off += kBulkPiece) {
                 const uint32_t piece = min(uint32_t(kBulkPiece), bytes - off);
                 asm volatile(
                     "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
@@ -191,25 +194,35 @@ select_kernel(SelectParams p, int chunk, int resident) {
             }
         }
         for (int j = n16 + tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
-    } else if (resident) {
+    } else if (resident_launch) {
         for (int j = tid; j < n; j += kSelThreads) sv[j] = __ldg(srow + j);
     }
-    auto wait_chunk = [&]() {
-        if (bulk) {
-            uint32_t ok = 0;
-            for (uint32_t it = 0; !ok; ++it) {
-                asm volatile(
-                    "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n selp.u32 %0, 1, 0, q;\n}\n"
-                    : "=r"(ok)
-                    : "r"(bar)
-                    : "memory");
-                if (!ok && it >= kLoadSpinLimit) {
-                    raise_status(p.status, SPA_ERR_TIMEOUT);
-                    break;
-                }
-            }
+    // bounded poll of the chunk-load barrier
+    auto poll_chunk = [&](uint32_t limit) -> bool {
+        uint32_t ok = 0;
+        for (uint32_t it = 0; !ok; ++it) {
+            asm volatile(
+                "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n selp.u32 %0, 1, 0, q;\n}\n"
+                : "=r"(ok)
+                : "r"(bar)
+                : "memory");
+            if (!ok && it >= limit) return false;
         }
-        __syncthreads();   // the resident chunk (bulk part and tail) is visible to every warp
+        return true;
+    };
+    // Once the chunk has arrived, every warp sees it (barrier).  If the bulk copy has not
+    // landed within the bound, the CTA raises SPA_ERR_TIMEOUT and stops using its shared copy
+    // of the chunk: it reads the scores from global memory instead (the streaming path), so
+    // the result stays correct and nothing reads a half-written chunk.
+    int resident = resident_launch;
+    bool chunk_ok = true;
+    auto wait_chunk = [&]() {
+        const bool ok = !bulk || poll_chunk(spin_limit);
+        chunk_ok = __syncthreads_and(ok ? 1 : 0) != 0;
+        if (!chunk_ok) {
+            if (tid == 0) raise_status(p.status, SPA_ERR_TIMEOUT);
+            resident = 0;
+        }
     };
     auto val_at = [&](int i) -> float { return resident ? sv[i] : __ldg(srow + i); };
 
@@ -591,6 +604,9 @@ select_kernel(SelectParams p, int chunk, int resident) {
         walk(false, true, base, nsel, fmass);
     }
 
+    // a chunk load that gave up: wait once more (bounded) so that a late copy lands before
+    // the CTA exits (a copy still in flight after that bound is the one hazard left)
+    if (!chunk_ok && bulk) poll_chunk(spin_limit);
     if (rank == 0) {
         // the unit's level-0 histogram is consumed: clear it for the next producer
         for (int i = tid; i < kBins; i += kSelThreads) {
@@ -686,7 +702,9 @@ SelectConfig choose(int U, int M) {
 }
 
 template <bool TOPP>
-spa_status launch_t(const SelectParams& p, cudaStream_t st) {
+spa_status launch_t(const SelectParams& p0, cudaStream_t st) {
+    SelectParams p = p0;
+    p.test_stall = test_stall_bits();
     const SelectConfig c = choose<TOPP>(p.U, p.M);
     SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)));

@@ -123,3 +123,8 @@ def test_decode_rla_fields_validation():
 def test_static_status_rejects_null_bits():
     # validation precedes the device lookup: no GPU needed
     assert spa.lib().spa_select_static_status(None, None, 0) == _abi.SPA_ERR_INVALID_ARG
+
+
+def test_test_stall_rejects_unknown_bits():
+    assert spa.lib().spa_test_stall(4) == _abi.SPA_ERR_INVALID_ARG
+    assert spa.lib().spa_test_stall(0) == _abi.SPA_OK
