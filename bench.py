@@ -51,9 +51,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
-    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS) + ["c5", "c5q"],
+    ap.add_argument("--config", default="c2_128k", choices=sorted(DECODE_CONFIGS) + ["c5", "c5q", "pbs_32k"],
                     help="decode workload (default); c5: the selection-block-shared prefill; c5q: the per-query "
-                         "prefill (b_sel = 1) on the last 1024 queries of the c5 chunk")
+                         "prefill (b_sel = 1) on the last 1024 queries of the c5 chunk; pbs_32k: the permuted "
+                         "block-sparse prefill of a 32K-token sequence")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--local-fraction", type=float, default=0.0,
                     help="head-wise routing: this fraction of every sequence's units is local (sink + window)")
@@ -670,8 +671,136 @@ def run_prefill(a):
     return 0
 
 
+def pbs_flops(cfg, counts):
+    """Algorithmic flops of a permuted block-sparse prefill: the importance pass (2 d per query
+    row of the last block and key, b*G rows per kv head) and the attention (4 d per (query head,
+    key) over the kept keys, the own segment's earlier keys and the causal diagonal)."""
+    imp = 2.0 * cfg.d * cfg.b * cfg.G * cfg.T * cfg.Hkv
+    att = 0.0
+    diag = cfg.b * (cfg.b + 1) // 2
+    for u in range(cfg.U):
+        j = u // cfg.Hkv
+        t0 = j * cfg.b
+        keys = cfg.b * (int(counts[u]) + t0 - t0 // cfg.S * cfg.S) + diag
+        att += 4.0 * cfg.d * cfg.G * keys
+    return imp + att
+
+
+def run_pbs(a):
+    """--config pbs_32k: the permuted block-sparse prefill (PBS-Attn) of one 32K-token sequence,
+    in TFLOP/s of its algorithmic flops; the L2 is flushed before every step."""
+    import oracle
+    from synth import PBS_32K, pbs_inputs
+
+    cfg = PBS_32K
+    if a.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    x = pbs_inputs(cfg)
+    b, G, T, S = cfg.b, cfg.G, cfg.T, cfg.S
+    sm = float(np.float32(cfg.sm_scale))
+
+    def oracle_sample(budget_s):
+        """The oracle on a bounded sample: kv head 0's importance and permutation, then query
+        blocks of that head from the end of the sequence until the budget is spent."""
+        t0 = time.perf_counter()
+        imp = oracle.pbs_importance(x["Q"][T - b:, 0:G], T - b, x["K"][0], sm)
+        perm = oracle.pbs_permutation(imp, S)
+        fl = 2.0 * cfg.d * b * G * T
+        done = 0
+        for j in range(cfg.n_blocks - 1, -1, -1):
+            if time.perf_counter() - t0 > budget_s and done:
+                break
+            sup, _ = oracle.pbs_prefill_unit(x["Q"][j * b:(j + 1) * b, 0:G], j * b, x["K"][0], x["V"][0], perm, S,
+                                             cfg.topk, sm)
+            t_0 = j * b
+            fl += 4.0 * cfg.d * G * (b * (sup.size + t_0 - t_0 // S * S) + b * (b + 1) // 2)
+            done += 1
+        dt = time.perf_counter() - t0
+        return fl / dt / 1e12, dt, done
+
+    if a.impl == "reference":
+        v, dt, done = oracle_sample(a.cpu_seconds)
+        print(json.dumps({"impl": "reference", "metric": "permuted block-sparse prefill TFLOP/s (algorithmic)",
+                          "value": v, "unit": "TFLOP/s", "n_gpus": a.gpus, "steps": 1, "warmup": 0,
+                          "ms_per_step": dt * 1e3, "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": f"{cfg.name}: kv head 0 importance + {done} query blocks"},
+                          "cpu_baseline": {"kind": "oracle", "cores": 1, "value": v,
+                                           "sample": f"kv head 0: importance, permutation, {done} query blocks"},
+                          "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return 0
+    import torch
+
+    import long_context_sparse_spa_b200 as spa
+
+    dQ, dK, dV = bf16_dev(x["Q"]), bf16_dev(x["K"]), bf16_dev(x["V"])
+    plan = spa.pbs_prefill(Q=dQ, K=dK, V=dV, sm_scale=sm, S=S, topk=cfg.topk, b=b, want_f32=False, run=False)
+    wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    for _ in range(a.warmup):
+        wbuf.zero_(); rbuf.sum(); plan.run()
+    torch.cuda.synchronize()
+    assert spa.read_device_status(plan.ws) == 0, "device status raised during warm-up"
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(a.steps)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(a.steps):
+        wbuf.zero_(); rbuf.sum()
+        ev[i][0].record(); plan.run(); ev[i][1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    counts = plan.count.cpu().numpy()
+    flops = pbs_flops(cfg, counts)
+    tflops = flops / (ms * 1e-3) / 1e12
+    hq = torch.from_numpy(np.ascontiguousarray(x["Q"]).view(np.int16)).pin_memory()
+    hout = torch.empty(plan.out.shape, dtype=plan.out.dtype).pin_memory()
+    e2e = []
+    for i in range(min(a.steps, 20) + 2):
+        wbuf.zero_(); rbuf.sum(); torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        dQ.view(torch.int16).copy_(hq, non_blocking=True)
+        plan.run()
+        hout.copy_(plan.out, non_blocking=True)
+        s1.record(); s1.synchronize()
+        if i >= 2:
+            e2e.append(s0.elapsed_time(s1))
+    e2e_ms = float(np.mean(e2e))
+    peak, peak_kind = None, "fallback"
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+        peak_kind = "measured"
+    peak = peak or 1590.0
+    cpu = None
+    if not a.no_cpu_baseline:
+        v, dt, done = oracle_sample(a.cpu_seconds)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": f"kv head 0: importance, permutation and {done} query blocks, fp64 oracle, {dt:.1f} s"}
+    out = {"metric": "permuted block-sparse prefill TFLOP/s (algorithmic)", "value": tflops, "unit": "TFLOP/s",
+           "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"{cfg.name}: causal prefill T={T}, Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} b={b} "
+                                  f"S={S} top-k={cfg.topk} blocks",
+                      "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
+                      "kept_blocks_mean": float(counts.mean() / b), "algorithmic_gflop_per_step": flops / 1e9},
+           "roofline": {"bound": "tensor", "kernel": "permuted prefill (all kernels of the step)", "achieved": tflops,
+                        "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
+                        "traffic": None},
+           "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": int(hq.numel() * 2), "d2h_bytes_per_step": int(hout.numel() * 2),
+                   "ms_per_step": e2e_ms},
+           "gpu_launches": 11 * a.steps, "clocks": clocks, "cpu_baseline": cpu}
+    print(json.dumps(out))
+    return 0
+
+
 def main():
     a = parse()
+    if a.config == "pbs_32k":
+        return run_pbs(a)
     if a.config in ("c5", "c5q"):
         return run_prefill(a)
     if a.impl == "reference":
