@@ -610,6 +610,8 @@ def run_prefill(a):
     counts = plan.count.cpu().numpy()
     flops = prefill_flops(cfg, counts)
     tflops = flops / (ms * 1e-3) / 1e12
+    # the tcgen05 attention kernel alone, in a separate pass (events around it inside the step)
+    kern_ms = timed_attention_ms(plan, a.steps, lambda: (wbuf.zero_(), rbuf.sum())) if cfg.bq > 1 else None
     # end to end: the chunk's queries (Q, q_idx) from pinned host memory, output read back
     hq = [torch.from_numpy(np.ascontiguousarray(x[k]).view(np.int16)).pin_memory() for k in ("Q", "q_idx")]
     dq = [plan.keep[0], plan.keep[1]]
@@ -660,15 +662,82 @@ def run_prefill(a):
                       "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
                       "support_mean": float(counts.mean()), "algorithmic_gflop_per_step": flops / 1e9,
                       "sparsity": round(float(prefill_sparsity(cfg, counts)), 4), "captured_mass": mass},
-           "roofline": ({"bound": "tensor", "kernel": "prefill (all kernels of the step)", "achieved": tflops,
-                         "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
-                         "traffic": None} if cfg.bq > 1 else pq_roofline(cfg, counts, ms)),
+           "roofline": (attention_roofline(flops, kern_ms, tflops, peak, peak_kind) if cfg.bq > 1
+                        else pq_roofline(cfg, counts, ms)),
            "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": int(sum(h.numel() * 2 for h in hq)),
                    "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms},
            "gpu_launches": (6 if cfg.bq > 1 else 7) * a.steps, "clocks": clocks, "cpu_baseline": cpu}
     print(json.dumps(out))
     return 0
+
+
+def timed_attention_ms(plan, steps, flush):
+    """Mean duration of the prefill's tcgen05 attention kernel: events recorded right before and
+    right after it inside real steps (run_timed), the L2 flushed before each step."""
+    import torch
+
+    k = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for e in k:
+        e.record()
+    out = []
+    for i in range(min(steps, 20) + 2):
+        flush()
+        plan.run_timed(k)
+        torch.cuda.synchronize()
+        if i >= 2:
+            out.append(k[0].elapsed_time(k[1]))
+    return float(np.mean(out))
+
+
+def attention_roofline(att_flops, kern_ms, step_tflops, peak, peak_kind):
+    """Roofline of the tcgen05 attention kernel at its algorithmic flops (4 d per query head and
+    attended key), against the dense bf16 peak; step_frac applies the same to the whole step."""
+    achieved = att_flops / (kern_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": "prefill_attend_kernel", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_kind, "kernel_ms": kern_ms,
+            "step_frac": step_tflops / peak, "traffic": None}
+
+
+def pbs_rows(cfg, u, i, counts):
+    """Keys attended by query i of unit u of a permuted block-sparse prefill, and its causal keys."""
+    j = u // cfg.Hkv
+    t0 = j * cfg.b
+    seg0 = t0 // cfg.S * cfg.S
+    return int(counts[u]) + (t0 - seg0) + i + 1, t0 + i + 1
+
+
+def pbs_sparsity(cfg, counts):
+    """Mean over units of the fraction of causal keys a query does not attend (queries averaged)."""
+    out = []
+    for u in range(cfg.U):
+        att = sum(pbs_rows(cfg, u, i, counts)[0] for i in range(cfg.b))
+        cau = sum(pbs_rows(cfg, u, i, counts)[1] for i in range(cfg.b))
+        out.append(1.0 - att / cau)
+    return float(np.mean(out))
+
+
+def pbs_captured_mass(cfg, x, idx, counts, n_units=8, queries=(0, 31, 63)):
+    """Dense head-averaged causal softmax mass on the attended rows (kept keys, the own segment's
+    earlier keys, the causal diagonal), from the oracle, for a spread sample of units."""
+    import oracle
+
+    G, b = cfg.G, cfg.b
+    units = np.linspace(cfg.Hkv * (cfg.S // b), cfg.U - 1, n_units).astype(int)   # units past the first segment
+    vals = []
+    for u in units:
+        j, g = u // cfg.Hkv, u % cfg.Hkv
+        t0 = j * b
+        seg0 = t0 // cfg.S * cfg.S
+        sup = idx[u, :counts[u]].astype(np.int64)
+        for i in queries:
+            t = t0 + i
+            P = oracle.dense_probs(x["Q"][t, g * G:(g + 1) * G], x["K"][g, :t + 1], float(np.float32(cfg.sm_scale)))
+            rows = np.union1d(sup, np.arange(seg0, t + 1))
+            vals.append(float(P[rows].sum()))
+    return {"mean": round(float(np.mean(vals)), 5), "min": round(float(np.min(vals)), 5),
+            "units": f"{len(units)} units (query blocks past the first segment, spread) x queries {list(queries)}",
+            "how": "fp64 oracle dense head-averaged causal softmax, summed over the attended rows"}
 
 
 def pbs_flops(cfg, counts):
@@ -753,6 +822,8 @@ def run_pbs(a):
     counts = plan.count.cpu().numpy()
     flops = pbs_flops(cfg, counts)
     tflops = flops / (ms * 1e-3) / 1e12
+    att_flops = flops - 2.0 * cfg.d * b * G * T * cfg.Hkv      # without the importance pass
+    kern_ms = timed_attention_ms(plan, a.steps, lambda: (wbuf.zero_(), rbuf.sum()))
     hq = torch.from_numpy(np.ascontiguousarray(x["Q"]).view(np.int16)).pin_memory()
     hout = torch.empty(plan.out.shape, dtype=plan.out.dtype).pin_memory()
     e2e = []
@@ -775,7 +846,9 @@ def run_pbs(a):
         peak_kind = "measured"
     peak = peak or 1590.0
     cpu = None
+    mass = None
     if not a.no_cpu_baseline:
+        mass = pbs_captured_mass(cfg, x, plan.idx.cpu().numpy(), counts)
         v, dt, done = oracle_sample(a.cpu_seconds)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": f"kv head 0: importance, permutation and {done} query blocks, fp64 oracle, {dt:.1f} s"}
@@ -785,10 +858,9 @@ def run_pbs(a):
            "config": {"workload": f"{cfg.name}: causal prefill T={T}, Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} b={b} "
                                   f"S={S} top-k={cfg.topk} blocks",
                       "l2": "flushed before every step (256 MiB device write, then a 256 MiB read)",
-                      "kept_blocks_mean": float(counts.mean() / b), "algorithmic_gflop_per_step": flops / 1e9},
-           "roofline": {"bound": "tensor", "kernel": "permuted prefill (all kernels of the step)", "achieved": tflops,
-                        "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": peak_kind,
-                        "traffic": None},
+                      "kept_blocks_mean": float(counts.mean() / b), "algorithmic_gflop_per_step": flops / 1e9,
+                      "sparsity": round(pbs_sparsity(cfg, counts), 4), "captured_mass": mass},
+           "roofline": attention_roofline(att_flops, kern_ms, tflops, peak, peak_kind),
            "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": int(hq.numel() * 2), "d2h_bytes_per_step": int(hout.numel() * 2),
                    "ms_per_step": e2e_ms},

@@ -391,11 +391,16 @@ typedef struct spa_prefill_args {
     int32_t* count;           /* [U] out */
     int cap;
     uint16_t* out;            /* [T, Hq, d] out */
-    float* out_f32;           /* optional */
+    float* out_f32;           /* optional, [T, Hq, d]; 16-byte aligned */
 } spa_prefill_args;
 
 spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream);
 size_t spa_prefill_workspace_bytes(const spa_prefill_args* a);
+/* spa_prefill_shared that also records two caller-created cudaEvent_t on `stream`: events[0]
+ * right before the tcgen05 attention kernel and events[1] right after it, so a caller can time
+ * that kernel inside a real step.  SPA_ERR_INVALID_ARG if events or either event is NULL. */
+spa_status spa_prefill_shared_timed(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream,
+                                    void* const* events);
 
 /* ------------------------------------------------------------------------------------
  * Per-query sparse prefill ("Oracle-Guided Sparse Prefill" 2.1 with b_sel = 1: every query
@@ -453,11 +458,16 @@ typedef struct spa_pbs_args {
     int32_t* count;           /* [U] out */
     int cap;
     uint16_t* out;            /* [T, Hq, d] out */
-    float* out_f32;           /* optional */
+    float* out_f32;           /* optional, [T, Hq, d]; 16-byte aligned */
 } spa_pbs_args;
 
 spa_status spa_pbs_prefill(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream);
 size_t spa_pbs_workspace_bytes(const spa_pbs_args* a);
+/* spa_pbs_prefill with two caller-created cudaEvent_t recorded on `stream` around the tcgen05
+ * attention kernel (events[0] before, events[1] after).  SPA_ERR_INVALID_ARG if events or
+ * either event is NULL. */
+spa_status spa_pbs_prefill_timed(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream,
+                                 void* const* events);
 
 /* ------------------------------------------------------------------------------------
  * Device status word of a workspace (sticky OR of SPA_ERR_* bits as (1 << code)).

@@ -330,6 +330,15 @@ class PrefillPlan:
         fn = lib().spa_prefill_per_query if self.per_query else lib().spa_prefill_shared
         check(fn(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(), _stream(stream)))
 
+    def run_timed(self, events, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """run() of the shared-support prefill recording two torch.cuda.Event (enable_timing=True,
+        already recorded once) right before and right after its attention kernel."""
+        if self.per_query:
+            raise ValueError("run_timed times the shared-support prefill's attention kernel")
+        handles = (ctypes.c_void_p * 2)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        check(lib().spa_prefill_shared_timed(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()),
+                                             self.ws.numel(), _stream(stream), handles))
+
 
 def prefill(*, Q: torch.Tensor, q_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, Kidx: torch.Tensor,
             q_start: int, score_scale: float, sm_scale: float, topk: int, sink: int, bq: int = 64,
@@ -385,6 +394,13 @@ class PbsPlan:
     def run(self, stream: Optional[torch.cuda.Stream] = None) -> None:
         check(lib().spa_pbs_prefill(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
                                     _stream(stream)))
+
+    def run_timed(self, events, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """run() recording two torch.cuda.Event (enable_timing=True, already recorded once) right
+        before and right after the attention kernel."""
+        handles = (ctypes.c_void_p * 2)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        check(lib().spa_pbs_prefill_timed(ctypes.byref(self.args), ctypes.c_void_p(self.ws.data_ptr()),
+                                          self.ws.numel(), _stream(stream), handles))
 
 
 def pbs_prefill(*, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, sm_scale: float, S: int, topk: int,

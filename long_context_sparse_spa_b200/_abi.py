@@ -7,7 +7,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(HERE, "libspa.so")
 
-ABI_VERSION = 6   # spa_abi_version() of the library these declarations describe
+ABI_VERSION = 7   # spa_abi_version() of the library these declarations describe
 
 SPA_OK = 0
 SPA_ERR_INVALID_ARG = 1
@@ -106,9 +106,11 @@ SIGNATURES = {
     "spa_decode_timed": (_i, [ctypes.POINTER(SpaDecodeArgs), _p, _sz, _p, ctypes.POINTER(_p)]),
     "spa_read_device_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32), _i]),
     "spa_prefill_shared": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
+    "spa_prefill_shared_timed": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p, ctypes.POINTER(_p)]),
     "spa_prefill_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
     "spa_prefill_per_query": (_i, [ctypes.POINTER(SpaPrefillArgs), _p, _sz, _p]),
     "spa_pbs_prefill": (_i, [ctypes.POINTER(SpaPbsArgs), _p, _sz, _p]),
+    "spa_pbs_prefill_timed": (_i, [ctypes.POINTER(SpaPbsArgs), _p, _sz, _p, ctypes.POINTER(_p)]),
     "spa_pbs_workspace_bytes": (_sz, [ctypes.POINTER(SpaPbsArgs)]),
     "spa_prefill_per_query_workspace_bytes": (_sz, [ctypes.POINTER(SpaPrefillArgs)]),
 }

@@ -89,7 +89,7 @@ spa_status spa_test_stall(int bits) {
     return SPA_OK;
 }
 
-int spa_abi_version(void) { return 6; }
+int spa_abi_version(void) { return 7; }
 
 // shared checks of the block-statistics entries; SPA_OK with *noop set when there is nothing to do
 static spa_status check_stats_args(const uint16_t* K, int B, int Hkv, int N, int d, int block, const void* a,
@@ -419,7 +419,8 @@ spa_status spa_rla_state(const uint16_t* K, const uint16_t* V, int B, int Hkv, i
     return launch_rla_state(K, V, B * Hkv, N, d, n0, n1, S, z, static_cast<cudaStream_t>(stream));
 }
 
-spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {
+static spa_status prefill_impl(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream,
+                               void* const* events) {
     if (!a || !ws) return SPA_ERR_INVALID_ARG;
     if (a->T < 0 || a->N <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->bq <= 0 ||
         a->q_start < 0 || a->topk < 0 || a->sink < 0 || a->cap < 0)
@@ -433,10 +434,20 @@ spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_byt
         return SPA_ERR_UNSUPPORTED_SHAPE;
     if (a->cap < (a->topk + a->sink < a->N ? a->topk + a->sink : a->N)) return SPA_ERR_INVALID_ARG;
     if (!aligned16(a->Q) || !aligned16(a->q_idx) || !aligned16(a->K) || !aligned16(a->V) || !aligned16(a->Kidx) ||
-        !aligned16(a->out))
+        !aligned16(a->out) || (a->out_f32 && !aligned16(a->out_f32)))
         return SPA_ERR_UNSUPPORTED_SHAPE;
     if (ws_bytes < spa_prefill_workspace_bytes(a)) return SPA_ERR_WORKSPACE_TOO_SMALL;
-    return launch_prefill(a, ws, static_cast<cudaStream_t>(stream));
+    return launch_prefill(a, ws, static_cast<cudaStream_t>(stream), events);
+}
+
+spa_status spa_prefill_shared(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {
+    return prefill_impl(a, ws, ws_bytes, stream, nullptr);
+}
+
+spa_status spa_prefill_shared_timed(const spa_prefill_args* a, void* ws, size_t ws_bytes, void* stream,
+                                    void* const* events) {
+    if (!events || !events[0] || !events[1]) return SPA_ERR_INVALID_ARG;
+    return prefill_impl(a, ws, ws_bytes, stream, events);
 }
 
 spa_status spa_read_device_status(void* ws, void* stream, uint32_t* bits, int reset) {

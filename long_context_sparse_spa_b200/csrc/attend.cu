@@ -520,7 +520,10 @@ attend_kernel(AttendParams p, int U, int nh) {
 // (o[D], m, l) of one (unit, head) are contiguous: they are staged into shared memory in
 // chunks with every load of a thread issued at once, then merged against the unit's
 // maximum M with a fixed assignment of records to thread groups and a fixed-order sum.
-constexpr int kCombRecs = 48;    // records staged per chunk
+// A unit of at most kCombRecs records (every unit of a 2-CTA-per-SM grid split over at most
+// 128 CTAs) is staged in one round and takes M from the staged records, so its only global
+// round trip is that one; longer units first read every record's m, then stage in chunks.
+constexpr int kCombRecs = 128;   // records staged per chunk (dynamic shared memory)
 
 //
 // RLA: every unit, empty ones included, is finished here.  With the unit's sums of Olin,
@@ -544,19 +547,27 @@ combine_kernel(AttendParams p, int nh, int n_slots) {
     const size_t first = size_t(row) * n_slots + u + (c_lo < 0 ? 0 : c_lo);
     const float* base = p.partials + first * REC;
 
-    __shared__ __align__(16) float st[kCombRecs * REC];
+    extern __shared__ __align__(16) float st[];   // [kCombRecs][REC]
     __shared__ float s_red[8];
     __shared__ float sL[GROUPS], sO[GROUPS][D];
-    float mx = -INFINITY;
-    for (int c = tid; c < n_c; c += 256) mx = fmaxf(mx, __ldcg(base + size_t(c) * REC + D));
+    // the unit's maximum m over its records, as seen by every thread
+    auto block_max = [&](float mx) -> float {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) s_red[warp] = mx;
-    __syncthreads();
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) s_red[warp] = mx;
+        __syncthreads();
+        float r = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) r = fmaxf(r, s_red[w]);
+        return r;
+    };
+    const bool one_round = n_c <= kCombRecs;
     float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) M = fmaxf(M, s_red[w]);
-    const float Mr = M == -INFINITY ? 0.f : M;
+    if (!one_round) {
+        float mx = -INFINITY;
+        for (int c = tid; c < n_c; c += 256) mx = fmaxf(mx, __ldcg(base + size_t(c) * REC + D));
+        M = block_max(mx);
+    }
 
     const int pair = tid % PAIRS, grp = tid / PAIRS;
     float L = 0.f, O0 = 0.f, O1 = 0.f;
@@ -577,6 +588,8 @@ combine_kernel(AttendParams p, int nh, int n_slots) {
             if (i < n2) reinterpret_cast<float2*>(st)[i] = t[k];
         }
         __syncthreads();
+        if (one_round) M = block_max(tid < nr ? st[tid * REC + D] : -INFINITY);   // nr <= kCombRecs <= 256
+        const float Mr = M == -INFINITY ? 0.f : M;
         for (int r = grp; r < nr; r += GROUPS) {
             const float* rec = st + r * REC;
             const float sc = exp2f(rec[D] - Mr);
@@ -676,7 +689,10 @@ spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
         SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<DD, H8, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                           int(sm)));                                                            \
         SPA_CUDA_TRY(launch_pdl(attend_kernel<DD, H8, R>, dim3(grid), dim3(kAtThreads), sm, st, p, U, nh));      \
-        SPA_CUDA_TRY(launch_pdl(combine_kernel<DD, R>, dim3(U, nh), dim3(256), 0, st, p, nh, U + grid));          \
+        const size_t cs = size_t(kCombRecs) * (DD + 2) * 4;                                                    \
+        SPA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel<DD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
+                                          int(cs)));                                                            \
+        SPA_CUDA_TRY(launch_pdl(combine_kernel<DD, R>, dim3(U, nh), dim3(256), cs, st, p, nh, U + grid));         \
         return SPA_OK;                                                                                          \
     }
     SPA_AT_CASE(128, 1, false) SPA_AT_CASE(128, 2, false) SPA_AT_CASE(64, 1, false) SPA_AT_CASE(64, 2, false)

@@ -294,7 +294,8 @@ spa_status launch_rla_state(const uint16_t* K, const uint16_t* V, int BH, int N,
 
 // prefill.cu
 size_t prefill_scratch_bytes(int U, int N);
-spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st);
+// events (optional, 2): recorded on st right before and right after the attention kernel
+spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st, void* const* events = nullptr);
 // The tcgen05 attention of 64-query blocks: unit u = block * Hkv + g attends, for each of its 64
 // queries (positions q_start + block * 64 + i) and G heads, to the rows idx[u][0 .. count[u])
 // and to the block's own positions up to the query (causal).  d = 128, G even.
@@ -312,7 +313,8 @@ struct PrefillAttendParams {
     uint32_t* status;
     int test_stall;        // SPA_TEST_STALL_* bits (test hook), else 0
 };
-spa_status launch_prefill_attend(const PrefillAttendParams& pp, int U, cudaStream_t st);
+spa_status launch_prefill_attend(const PrefillAttendParams& pp, int U, cudaStream_t st,
+                                 void* const* events = nullptr);
 
 // The test hook's armed bits (spa_test_stall), read by the launchers.
 int test_stall_bits();

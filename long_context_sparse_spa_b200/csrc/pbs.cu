@@ -357,7 +357,7 @@ extern "C" size_t spa_pbs_workspace_bytes(const spa_pbs_args* a) {
     return kWsHeader + pbs_layout(a).total;
 }
 
-extern "C" spa_status spa_pbs_prefill(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream) {
+static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream, void* const* events) {
     if (!a || !ws) return SPA_ERR_INVALID_ARG;
     if (a->T <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->b <= 0 || a->S <= 0 || a->topk < 0 ||
         a->cap < 0)
@@ -365,7 +365,9 @@ extern "C" spa_status spa_pbs_prefill(const spa_pbs_args* a, void* ws, size_t ws
     if (!a->Q || !a->K || !a->V || !a->perm || !a->idx || !a->count || !a->out) return SPA_ERR_INVALID_ARG;
     if (!pbs_shape_ok(a)) return SPA_ERR_UNSUPPORTED_SHAPE;
     if (a->cap < a->topk * a->b) return SPA_ERR_INVALID_ARG;
-    if (!aligned16(a->Q) || !aligned16(a->K) || !aligned16(a->V) || !aligned16(a->out)) return SPA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(a->Q) || !aligned16(a->K) || !aligned16(a->V) || !aligned16(a->out) ||
+        (a->out_f32 && !aligned16(a->out_f32)))
+        return SPA_ERR_UNSUPPORTED_SHAPE;
     if (ws_bytes < spa_pbs_workspace_bytes(a)) return SPA_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const PbsLayout l = pbs_layout(a);
@@ -440,5 +442,15 @@ extern "C" spa_status spa_pbs_prefill(const spa_pbs_args* a, void* ws, size_t ws
     SPA_CUDA_TRY(launch_pdl(pbs_expand_kernel, dim3(U), dim3(kPbThreads), size_t(Pe) * 4, st, p));
     PrefillAttendParams pp{a->Q, a->K, a->V, p.aidx, p.acount, p.acap, a->Hq, a->Hkv, a->T, a->b, 0, a->sm_scale,
                            a->out, a->out_f32, status};
-    return launch_prefill_attend(pp, U, st);
+    return launch_prefill_attend(pp, U, st, events);
+}
+
+extern "C" spa_status spa_pbs_prefill(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream) {
+    return pbs_impl(a, ws, ws_bytes, stream, nullptr);
+}
+
+extern "C" spa_status spa_pbs_prefill_timed(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream,
+                                            void* const* events) {
+    if (!events || !events[0] || !events[1]) return SPA_ERR_INVALID_ARG;
+    return pbs_impl(a, ws, ws_bytes, stream, events);
 }

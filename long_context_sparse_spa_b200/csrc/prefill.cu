@@ -15,12 +15,10 @@
 // Step 4 is a dense contraction (64 queries x G heads share each support) and runs on the
 // 5th-generation tensor cores: tcgen05.mma with operands in shared memory (128-byte
 // swizzled, one 128-byte line per row of 64 bf16), fp32 accumulators in tensor memory
-// (TMEM), issued by one thread and completed through an mbarrier.  One CTA owns 128 query
+// (TMEM), issued by one thread and completed through mbarriers.  One CTA owns 128 query
 // rows (two heads x 64 queries).  Keys are processed in tiles of 128 gathered rows
-// (cp.async, bounds-checked) plus the diagonal tile of the block's own 64 positions.
-// Two passes: pass 1 accumulates each row's max m and sum l from S = Q K^T; pass 2
-// recomputes S, forms the normalised P = exp(S - m) / l as the sum of two bf16 terms
-// and accumulates O += P V (two MMAs), so no rescaling of O is needed.
+// (cp.async, bounds-checked) plus the diagonal tile of the block's own 64 positions, in one
+// pass with an online softmax (see the attention section below).
 #include "internal.cuh"
 
 namespace spa {
@@ -28,7 +26,6 @@ namespace {
 
 constexpr int kPfRows = 128;          // query rows per CTA (tensor-core M)
 constexpr int kPfKeys = 128;          // keys per tile (tensor-core N of S, K of P V)
-constexpr int kPfThreads = 128;       // one thread per query row / TMEM lane
 constexpr int kSlab = kPfRows * 128;  // bytes of one 64-column slab of a 128-row operand
 constexpr int kTileBytes = 2 * kSlab; // 128 rows x 128 bf16
 constexpr uint32_t kSpinLimit = 1u << 22;   // bounded mbarrier polls before giving up
@@ -174,25 +171,60 @@ prefill_scores_kernel(const float* __restrict__ qhat, const int32_t* __restrict_
 }
 
 // ============================================================================ attention
+// One pass with an online softmax, pipelined.
+//   * 8 warps.  Warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32 query rows) and owns key
+//     columns 64 (w / 4) .. +63 of every S tile.  Each (row, column half) keeps its own running
+//     maximum m, sum l and output accumulator (O_a over the first 64 keys of every tile, O_b over
+//     the last 64), so the softmax exchanges nothing between threads until the epilogue merges
+//     the halves: O = (2^(m_a - m) O_a + 2^(m_b - m) O_b) / (2^(m_a - m) l_a + 2^(m_b - m) l_b).
+//   * A half's maximum moves (and its O is rescaled through TMEM) only when a tile's maximum
+//     exceeds it by more than kRescaleLog2, so P = 2^(S - m) <= 2^kRescaleLog2; the result is the
+//     same softmax for any such m.  P enters the MMA as bf16 hi + lo (two MMAs), ~16 bits.
+//   * S is double-buffered in TMEM: S(t+1) = Q K(t+1)^T runs on the tensor cores while the
+//     threads turn S(t) into P(t), and O += P(t) V(t) runs while they read S(t+1).
+//   * K and V tiles are double-buffered in shared memory and gathered one tile ahead: K of tile
+//     t+2 as soon as S(t) has consumed its buffer, V of tile t+1 as soon as P(t-1) V(t-1) has.
+//     Every thread commits one cp.async group per gather point, empty or not, so the group
+//     counts of the waits are the same in every iteration.
+// TMEM columns: S buffers 0..127 and 128..255, O_a 256..383, O_b 384..511.
+constexpr int kPfThreads = 256;
+constexpr float kRescaleLog2 = 8.f;
+
 struct __align__(1024) PfShared {
     uint8_t q[kTileBytes];
-    uint8_t k[kTileBytes];
-    uint8_t v[kTileBytes];
-    uint8_t p_hi[kTileBytes];
+    uint8_t k[2][kTileBytes];
+    uint8_t v[2][kTileBytes];
+    uint8_t p_hi[kTileBytes];   // the epilogue reuses it for the halves' (m, l)
     uint8_t p_lo[kTileBytes];
-    uint64_t bar;
+    uint64_t bar_s, bar_o;      // completion of the S MMAs / of the P V MMAs
     uint32_t tmem_base;
-    int rows[kPfKeys];     // cache rows of the current key tile (-1: none)
-    int timed_out;
+    uint32_t valid[4][kPfKeys / 32];   // bit c: key c of tile t (slot t % 4) is attended
 };
 
-// grid (U, G / 2): one CTA per (unit, pair of query heads); 128 threads.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n" ::"r"(
+            taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+        "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+        "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+        "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// grid (U, G / 2): one CTA per (unit, pair of query heads); 256 threads.
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_attend_kernel(PrefillAttendParams p) {
     pdl_enter();
     extern __shared__ __align__(1024) uint8_t dyn[];
     PfShared& sh = *reinterpret_cast<PfShared*>(dyn);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int u = blockIdx.x, pair = blockIdx.y;
     const int blk = u / p.Hkv, g = u - blk * p.Hkv;
     const int G = p.Hq / p.Hkv;
@@ -204,210 +236,286 @@ prefill_attend_kernel(PrefillAttendParams p) {
     const int32_t* sup = p.idx + size_t(u) * p.cap;
     const size_t kv0 = size_t(g) * p.N;
 
-    // this thread's query row: head 2*pair + tid/64, query tid%64 of the block
-    const int hh = 2 * pair + tid / 64, qi = tid & 63;
-    const int head = g * G + hh;
-    const size_t qrow = size_t(blk * p.bq + qi) * p.Hq + head;
+    // softmax role: query row r (TMEM lane) and key-column half
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane, qi = r & 63;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    if (warp == 0) tmem_alloc(&sh.tmem_base, 256);
+    if (warp == 0) tmem_alloc(&sh.tmem_base, 512);
     if (tid == 0) {
-        mbar_init(&sh.bar, 1);
-        sh.timed_out = 0;
+        mbar_init(&sh.bar_s, 1);
+        mbar_init(&sh.bar_o, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    // Q tile: row r = tid
+
+    // cache row of key rr of tile t, or -1 (outside the support, or out of range)
+    auto key_row = [&](int t, int rr) -> int {
+        if (t < n_gather) {
+            const int e = t * kPfKeys + rr;
+            if (e >= n_sup) return -1;
+            const int n = __ldg(sup + e);
+            return (n >= 0 && n < p.N) ? n : -1;
+        }
+        const int n = t0 + rr;                                 // the diagonal tile: the block's own keys
+        return (rr < p.bq && n < p.N) ? n : -1;
+    };
+    // 128 rows x 16 chunks of 16 bytes; thread tid copies chunk tid % 16 of rows tid / 16 + 16 j
+    auto gather = [&](const uint16_t* src, uint8_t* dst, int t) {
+        const int c = tid & 15;
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-        cp_async16(smem_u32(sh.q) + tile_off(tid, c), p.Q + qrow * 128 + c * 8, true);
+        for (int j = 0; j < kPfKeys / 16; ++j) {
+            const int rr = j * 16 + (tid >> 4);
+            const int row = key_row(t, rr);
+            const bool ok = row >= 0;
+            cp_async16(smem_u32(dst) + tile_off(rr, c), src + (ok ? (kv0 + size_t(row)) * 128 + c * 8 : 0), ok);
+        }
+    };
+    auto gather_k = [&](int t) {
+        if (t < n_tiles) {
+            if (warp < 4) {
+                const uint32_t b = __ballot_sync(0xffffffffu, key_row(t, warp * 32 + lane) >= 0);
+                if (lane == 0) sh.valid[t & 3][warp] = b;
+            }
+            gather(p.K, sh.k[t & 1], t);
+        }
+        cp_async_commit();
+    };
+    auto gather_v = [&](int t) {
+        if (t < n_tiles) gather(p.V, sh.v[t & 1], t);
+        cp_async_commit();
+    };
+
+    // Q tile (row rr: head 2 pair + rr / 64, query rr % 64 of the block), in K(0)'s group
+#pragma unroll
+    for (int j = 0; j < kPfRows / 16; ++j) {
+        const int rr = j * 16 + (tid >> 4), c = tid & 15;
+        const size_t qrow = size_t(blk * p.bq + (rr & 63)) * p.Hq + g * G + 2 * pair + rr / 64;
+        cp_async16(smem_u32(sh.q) + tile_off(rr, c), p.Q + qrow * 128 + c * 8, true);
+    }
+    gather_k(0);
+    gather_k(1);
+    gather_v(0);
+    cp_async_wait_group<2>();                                  // Q and K(0)
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
-    const uint32_t t_s = tmem, t_o = tmem + 128;                 // S at columns 0..127, O at 128..255
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    uint32_t phase = 0;
+    const uint32_t t_oa = tmem + 256;
+
     // the test hook stalls the first S = Q K^T: its completion barrier waits for an MMA that
     // is never issued, so the bounded wait runs out with nothing in flight
     const bool stall = (p.test_stall & SPA_TEST_STALL_PREFILL_MMA) != 0;
     const uint32_t spin_limit = stall ? 1024u : kSpinLimit;
-    bool pending = false;   // an MMA commit issued and not yet observed (uniform over the CTA)
     const float sl2 = p.sm_scale * kLog2e;
     constexpr uint32_t kIdS = idesc_bf16(kPfRows, kPfKeys, false);
     constexpr uint32_t kIdO = idesc_bf16(kPfRows, 128, true);
 
-    // gather the keys (and values) of tile t into shared memory; returns the number of valid keys
-    auto load_tile = [&](int t, bool with_v) {
-        __syncthreads();   // previous readers of rows/k/v are done
-        {
-            const int r = tid;
-            int row = -1;
-            if (t < n_gather) {
-                const int e = t * kPfKeys + r;
-                if (e < n_sup) {
-                    const int n = sup[e];
-                    row = (n >= 0 && n < p.N) ? n : -1;
-                }
-            } else if (r < p.bq) {
-                row = t0 + r;                                  // diagonal tile: the block's own keys
-                if (row >= p.N) row = -1;
-            }
-            sh.rows[r] = row;
-        }
-        __syncthreads();
-        // 128 rows x 16 chunks per tensor; thread tid copies chunk (tid & 15) of rows tid/16 + 8j
-        for (int j = 0; j < kPfKeys / 8; ++j) {
-            const int r = j * 8 + (tid >> 4), c = tid & 15;
-            const int row = sh.rows[r];
-            const bool ok = row >= 0;
-            const size_t src = ok ? (kv0 + size_t(row)) * 128 + c * 8 : 0;
-            cp_async16(smem_u32(sh.k) + tile_off(r, c), p.K + src, ok);
-            if (with_v) cp_async16(smem_u32(sh.v) + tile_off(r, c), p.V + src, ok);
-        }
-        cp_async_wait_all();
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    };
-    // S = Q K^T into TMEM columns 0..127; every thread waits for completion
-    auto mma_s = [&]() -> bool {
-        pending = !stall;
-        if (tid == 0 && !stall) {
+    auto issue_s = [&](int t) {                                // S(t) = Q K(t)^T into S buffer t % 2
+        const uint32_t d = tmem + uint32_t(t & 1) * 128;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
-                const uint64_t a = sw128_desc(smem_u32(sh.q) + off, 16, 1024);
-                const uint64_t b = sw128_desc(smem_u32(sh.k) + off, 16, 1024);
-                umma_bf16(t_s, a, b, kIdS, kk > 0);
-            }
-            umma_commit(&sh.bar);
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
+            umma_bf16(d, sw128_desc(smem_u32(sh.q) + off, 16, 1024), sw128_desc(smem_u32(sh.k[t & 1]) + off, 16, 1024),
+                      kIdS, kk > 0);
         }
+        umma_commit(&sh.bar_s);
+    };
+    auto issue_pv = [&](int t) {                               // O_a += P[:, 0:64] V(t)[0:64], O_b += the rest
+        const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo), vb = smem_u32(sh.v[t & 1]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t d = t_oa + uint32_t(kk >> 2) * 128;
+            const uint32_t aoff = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
+            const uint64_t bv = sw128_desc(vb + kk * 2048, kSlab, 1024);
+            umma_bf16(d, sw128_desc(ph + aoff, 16, 1024), bv, kIdO, (t > 0 || (kk & 3) > 0) ? 1u : 0u);
+            umma_bf16(d, sw128_desc(pl + aoff, 16, 1024), bv, kIdO, 1u);
+        }
+        umma_commit(&sh.bar_o);
+    };
+    // bounded wait on a completion barrier; on expiry this thread's flag is set, the CTA stops at
+    // its next barrier (each barrier ORs the flags of all threads, so every thread takes the same
+    // decision there) and the commit stays owed
+    bool my_to = false;
+    auto wait_bar = [&](uint64_t* bar, uint32_t& ph) -> bool {
+        uint32_t it = 0;
+        while (!mbar_try_wait(bar, ph)) {
+            if (++it >= spin_limit) {
+                my_to = true;
+                return false;
+            }
+        }
+        ph ^= 1u;
+        tc_fence_after();
         return true;
     };
-    // bounded wait for the outstanding commit; on expiry the CTA stops (every later step checks
-    // sh.timed_out) and the commit stays owed, so TMEM is not freed under a running MMA
-    auto wait_mma = [&]() {
-        uint32_t it = 0;
-        while (!mbar_try_wait(&sh.bar, phase)) {
-            if (++it >= spin_limit) {
-                atomicExch(&sh.timed_out, 1);
-                return;
-            }
-        }
-        pending = false;
-        phase ^= 1u;
-        tc_fence_after();
-    };
-    // this thread's row of S (scaled to log2 units, masked); key c of tile t
-    auto row_logits = [&](int t, float (&s)[kPfKeys]) {
-#pragma unroll
-        for (int cb = 0; cb < kPfKeys / 32; ++cb) {
-            float v[32];
-            tmem_ld32(t_s + lane_off + cb * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int c = cb * 32 + i;
-                const bool valid = sh.rows[c] >= 0 && (t < n_gather || c <= qi);
-                s[c] = valid ? v[i] * sl2 : -INFINITY;
-            }
-        }
-    };
 
-    // a bounded wait that gave up ends both passes for every thread at the same point
-    auto stop = [&]() -> bool {
-        __syncthreads();
-        return sh.timed_out != 0;
-    };
-
-    // ---- pass 1: row max m and sum l
-    float m = -INFINITY, l = 0.f;
-    for (int t = 0; t < n_tiles; ++t) {
-        load_tile(t, false);
-        mma_s();
-        wait_mma();
-        if (stop()) break;
-        float s[kPfKeys];
-        row_logits(t, s);
-        float tm = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kPfKeys; ++c) tm = fmaxf(tm, s[c]);
-        const float mn = fmaxf(m, tm);
-        if (mn != -INFINITY) {
-            float add = 0.f;
-#pragma unroll
-            for (int c = 0; c < kPfKeys; ++c) add += exp2f(s[c] - mn);
-            l = l * exp2f(m - mn) + add;
-            m = mn;
-        }
-        tc_fence_before();
+    bool pend_s = false, pend_o = false;   // a commit issued and not yet observed (uniform over the CTA)
+    uint32_t ph_s = 0, ph_o = 0;
+    if (!stall) {
+        if (tid == 0) issue_s(0);
+        pend_s = true;
     }
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t t_my_o = t_oa + uint32_t(half) * 128 + lane_off;
+    bool stopped = false;                  // a wait gave up (uniform over the CTA)
 
-    // ---- pass 2: O = sum_t P_t V_t with P = exp2(S - m) / l as bf16 hi + lo
-    for (int t = 0; t < n_tiles && !sh.timed_out; ++t) {
-        load_tile(t, true);
-        mma_s();
-        wait_mma();
-        if (stop()) break;
-        float s[kPfKeys];
-        row_logits(t, s);
-        const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
-#pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float p0 = m == -INFINITY ? 0.f : exp2f(s[c8 * 8 + 2 * j] - m) * inv_l;
-                const float p1 = m == -INFINITY ? 0.f : exp2f(s[c8 * 8 + 2 * j + 1] - m) * inv_l;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                const float2 hf = __bfloat1622float2(h);
-                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-                hw[j] = *reinterpret_cast<const uint32_t*>(&h);
-                lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
-            }
-            const uint32_t off = tile_off(tid, c8);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[0]), "r"(hw[1]),
-                         "r"(hw[2]), "r"(hw[3]));
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[0]), "r"(lw[1]),
-                         "r"(lw[2]), "r"(lw[3]));
-        }
+    for (int t = 0; t < n_tiles; ++t) {
+        // S(t) is complete: its K buffer takes tile t + 2 (ok is made warp-uniform: the gather
+        // holds a warp vote)
+        bool ok = wait_bar(&sh.bar_s, ph_s);
+        if (ok) pend_s = false;
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) gather_k(t + 2);
+        else cp_async_commit();
+        cp_async_wait_group<2>();                              // K(t + 1) (and V(t)) have landed
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        stopped = __syncthreads_or(my_to) != 0;
         tc_fence_after();
-        if (tid == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t aoff = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
-                const uint64_t bh = sw128_desc(smem_u32(sh.v) + kk * 2048, kSlab, 1024);
-                umma_bf16(t_o, sw128_desc(ph + aoff, 16, 1024), bh, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
-                umma_bf16(t_o, sw128_desc(pl + aoff, 16, 1024), bh, kIdO, 1u);
-            }
-            umma_commit(&sh.bar);
+        if (stopped) break;
+        if (t + 1 < n_tiles) {
+            if (tid == 0) issue_s(t + 1);
+            pend_s = true;
         }
-        pending = true;
-        wait_mma();       // O ready; P, K and V may be overwritten
+
+        // this thread's 64 logits of S(t), in log2 units, masked
+        float s[64];
+        {
+            float v[32];
+            const uint32_t ta = tmem + uint32_t(t & 1) * 128 + uint32_t(half) * 64 + lane_off;
+            tmem_ld32(ta, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[i] = v[i];
+            tmem_ld32(ta + 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[32 + i] = v[i];
+        }
         tc_fence_before();
-        if (stop()) break;
+        const uint32_t vm0 = sh.valid[t & 3][2 * half], vm1 = sh.valid[t & 3][2 * half + 1];
+        const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const bool valid = (((i < 32 ? vm0 : vm1) >> (i & 31)) & 1u) && i <= causal;
+            s[i] = valid ? s[i] * sl2 : -INFINITY;
+            tmax = fmaxf(tmax, s[i]);
+        }
+        bool rescale = false;
+        float alpha = 1.f;
+        if (tmax > m_run + kRescaleLog2) {                    // also the first finite maximum
+            alpha = exp2f(m_run - tmax);
+            rescale = m_run != -INFINITY;                      // O of this half holds nonzero terms
+            m_run = tmax;
+            l_run *= alpha;
+        }
+        // P = 2^(s - m) as bf16 hi + lo pairs
+        uint32_t hw[32], lw[32];
+        float add = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float p0 = m_run == -INFINITY ? 0.f : exp2f(s[2 * j] - m_run);
+            const float p1 = m_run == -INFINITY ? 0.f : exp2f(s[2 * j + 1] - m_run);
+            add += p0;
+            add += p1;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+            hw[j] = *reinterpret_cast<const uint32_t*>(&h);
+            lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
+        }
+        l_run += add;
+
+        // P(t-1) V(t-1) is complete: P, O and its V buffer are free
+        ok = t == 0 || wait_bar(&sh.bar_o, ph_o);
+        if (t > 0 && ok) pend_o = false;
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            // tcgen05.ld / st are warp-collective: a warp rescales when any of its rows needs it,
+            // the other rows by 1
+            if (__any_sync(0xffffffffu, rescale)) {
+                const float a = rescale ? alpha : 1.f;
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float v[32];
+                    tmem_ld32(t_my_o + cb * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= a;
+                    tmem_st32(t_my_o + cb * 32, v);
+                }
+                tmem_wait_st();
+            }
+            const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                const uint32_t off = tile_off(r, half * 8 + c8);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[4 * c8]),
+                             "r"(hw[4 * c8 + 1]), "r"(hw[4 * c8 + 2]), "r"(hw[4 * c8 + 3]));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[4 * c8]),
+                             "r"(lw[4 * c8 + 1]), "r"(lw[4 * c8 + 2]), "r"(lw[4 * c8 + 3]));
+            }
+            gather_v(t + 1);
+        } else {
+            cp_async_commit();
+        }
+        cp_async_wait_group<2>();                              // V(t) has landed
+        fence_async_smem();
+        tc_fence_before();
+        stopped = __syncthreads_or(my_to) != 0;
+        tc_fence_after();
+        if (stopped) break;
+        if (tid == 0) issue_pv(t);
+        pend_o = true;
     }
 
-    // ---- epilogue: this thread's output row from TMEM
+    // the last P V, then no copy is left in flight
+    if (!stopped && pend_o && wait_bar(&sh.bar_o, ph_o)) pend_o = false;
+    cp_async_wait_all();
+    tc_fence_before();
+    const bool good = __syncthreads_or(my_to) == 0;
+    float* ex = reinterpret_cast<float*>(sh.p_hi);            // [half][m | l][row]
+    if (good) {
+        ex[half * 256 + r] = m_run;
+        ex[half * 256 + 128 + r] = l_run;
+    }
     __syncthreads();
-    if (!sh.timed_out) {
-        uint16_t* orow = p.out + qrow * 128;
-        float* frow = p.out_f32 ? p.out_f32 + qrow * 128 : nullptr;
+    tc_fence_after();
+    if (good) {
+        const float ma = ex[r], la = ex[128 + r], mb = ex[256 + r], lb = ex[384 + r];
+        const float m = fmaxf(ma, mb);
+        float sa = 0.f, sb = 0.f;
+        if (m != -INFINITY) {
+            const float ea = exp2f(ma - m), eb = exp2f(mb - m);
+            const float l = la * ea + lb * eb;
+            if (l > 0.f) {
+                sa = ea / l;
+                sb = eb / l;
+            }
+        }
+        // this thread writes output columns 64 half .. 64 half + 63 of row r
+        const size_t qrow = size_t(blk * p.bq + qi) * p.Hq + g * G + 2 * pair + r / 64;
+        uint16_t* orow = p.out + qrow * 128 + half * 64;
+        float* frow = p.out_f32 ? p.out_f32 + qrow * 128 + half * 64 : nullptr;
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float v[32];
-            tmem_ld32(t_o + lane_off + cb * 32, v);
+        for (int cb = 0; cb < 2; ++cb) {
+            float va[32], vb[32];
+            tmem_ld32(t_oa + uint32_t(half * 64 + cb * 32) + lane_off, va);
+            tmem_ld32(t_oa + 128 + uint32_t(half * 64 + cb * 32) + lane_off, vb);
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                const float a = l > 0.f ? v[i] : 0.f, b = l > 0.f ? v[i + 1] : 0.f;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-                *reinterpret_cast<__nv_bfloat162*>(orow + cb * 32 + i) = h;
+            for (int i = 0; i < 32; i += 8) {
+                float o[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) o[k] = va[i + k] * sa + vb[i + k] * sb;
+                uint32_t w[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
+                    w[k] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(orow + cb * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
                 if (frow) {
-                    frow[cb * 32 + i] = a;
-                    frow[cb * 32 + i + 1] = b;
+                    *reinterpret_cast<float4*>(frow + cb * 32 + i) = make_float4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<float4*>(frow + cb * 32 + i + 4) = make_float4(o[4], o[5], o[6], o[7]);
                 }
             }
         }
@@ -419,15 +527,22 @@ prefill_attend_kernel(PrefillAttendParams p) {
     // after a give-up, an issued MMA may still be running: wait once more (bounded); TMEM is
     // freed only when no commit is owed (a CTA that exits holding TMEM is the remaining hazard
     // of a wait that never completes)
-    if (pending) {
+    if (pend_s) {
         uint32_t it = 0;
-        while (!mbar_try_wait(&sh.bar, phase) && ++it < spin_limit) {
+        while (!mbar_try_wait(&sh.bar_s, ph_s) && ++it < spin_limit) {
         }
-        pending = it >= spin_limit;
+        pend_s = it >= spin_limit;
     }
-    if (warp == 0 && !pending) {
+    if (pend_o) {
+        uint32_t it = 0;
+        while (!mbar_try_wait(&sh.bar_o, ph_o) && ++it < spin_limit) {
+        }
+        pend_o = it >= spin_limit;
+    }
+    // (the free is warp-collective: warp 0 frees only when none of its lanes still sees a debt)
+    if (warp == 0 && !__any_sync(0xffffffffu, pend_s || pend_o)) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -438,7 +553,7 @@ size_t prefill_scratch_bytes(int U, int N) {
            hist0_bytes(U);
 }
 
-spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) {
+spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st, void* const* events) {
     const int n_blocks = a->T / a->bq;
     const int U = n_blocks * a->Hkv;
     uint8_t* w = static_cast<uint8_t*>(ws);
@@ -466,15 +581,17 @@ spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st) 
 
     PrefillAttendParams pp{a->Q, a->K, a->V, a->idx, a->count, a->cap, a->Hq, a->Hkv, a->N, a->bq, a->q_start,
                            a->sm_scale, a->out, a->out_f32, status};
-    return launch_prefill_attend(pp, U, st);
+    return launch_prefill_attend(pp, U, st, events);
 }
 
-spa_status launch_prefill_attend(const PrefillAttendParams& pp0, int U, cudaStream_t st) {
+spa_status launch_prefill_attend(const PrefillAttendParams& pp0, int U, cudaStream_t st, void* const* events) {
     PrefillAttendParams pp = pp0;
     pp.test_stall = test_stall_bits();
     const size_t smem = sizeof(PfShared);
     SPA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
     SPA_CUDA_TRY(launch_pdl(prefill_attend_kernel, dim3(U, pp.Hq / pp.Hkv / 2), dim3(kPfThreads), smem, st, pp));
+    if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
     return SPA_OK;
 }
 

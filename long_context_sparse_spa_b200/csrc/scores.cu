@@ -35,8 +35,9 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
     const int pair = threadIdx.x >> 1;         // row slot within a pass
     constexpr int kRowsPerPass = kLrThreads / 2;
     constexpr int kHb = HIST ? kHistBins : 1;
-    __shared__ uint32_t h_cnt[kHb];
-    __shared__ uint32_t h_mhi[MASS ? kHb : 1], h_mlo[MASS ? kHb : 1];
+    __shared__ __align__(16) uint32_t h_cnt[kHb];
+    __shared__ __align__(16) uint32_t h_mhi[MASS ? kHb : 1];
+    __shared__ __align__(16) uint32_t h_mlo[MASS ? kHb : 1];
     __shared__ uint32_t h_max;
 
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
@@ -45,9 +46,10 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
         const int b = kvu / Hkv, g = kvu - b * Hkv;
         if (NQ == 1 && local && local[kvu]) continue;  // a local unit is not scored (uniform per CTA)
         if (HIST) {
-            for (int i = threadIdx.x; i < kHistBins; i += kLrThreads) {
-                h_cnt[i] = 0;
-                if (MASS) h_mhi[i] = h_mlo[i] = 0;
+            const uint4 z4 = make_uint4(0, 0, 0, 0);
+            for (int i = threadIdx.x; i < kHistBins / 4; i += kLrThreads) {
+                reinterpret_cast<uint4*>(h_cnt)[i] = z4;
+                if (MASS) reinterpret_cast<uint4*>(h_mhi)[i] = reinterpret_cast<uint4*>(h_mlo)[i] = z4;
             }
             if (threadIdx.x == 0) h_max = 0;
             __syncthreads();
@@ -144,11 +146,22 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
             __syncthreads();
             uint32_t* gc = hist.cnt + size_t(kvu) * kHistBins;
             unsigned long long* gm = hist.mass + size_t(kvu) * kHistBins;
-            for (int i = threadIdx.x; i < kHistBins; i += kLrThreads) {
-                const uint32_t c = h_cnt[i];
-                if (c) {
-                    atomicAdd(gc + i, c);
-                    if (MASS) atomicAdd(gm + i, (static_cast<unsigned long long>(h_mhi[i]) << 20) + h_mlo[i]);
+            for (int i4 = threadIdx.x; i4 < kHistBins / 4; i4 += kLrThreads) {   // four bins at a time
+                const uint4 c4 = reinterpret_cast<const uint4*>(h_cnt)[i4];
+                if ((c4.x | c4.y | c4.z | c4.w) == 0) continue;
+                const uint32_t c[4] = {c4.x, c4.y, c4.z, c4.w};
+                uint32_t mh[4] = {0, 0, 0, 0}, ml[4] = {0, 0, 0, 0};
+                if (MASS) {
+                    const uint4 h4 = reinterpret_cast<const uint4*>(h_mhi)[i4];
+                    const uint4 l4 = reinterpret_cast<const uint4*>(h_mlo)[i4];
+                    mh[0] = h4.x; mh[1] = h4.y; mh[2] = h4.z; mh[3] = h4.w;
+                    ml[0] = l4.x; ml[1] = l4.y; ml[2] = l4.z; ml[3] = l4.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (!c[j]) continue;
+                    atomicAdd(gc + 4 * i4 + j, c[j]);
+                    if (MASS) atomicAdd(gm + 4 * i4 + j, (static_cast<unsigned long long>(mh[j]) << 20) + ml[j]);
                 }
             }
             if (threadIdx.x == 0) atomicMax(hist.max_key + kvu, h_max);

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported_and_bound():
 
 def test_status_strings_and_version():
     L = spa.lib()
-    assert L.spa_abi_version() == 6 == _abi.ABI_VERSION
+    assert L.spa_abi_version() == 7 == _abi.ABI_VERSION
     assert L.spa_status_string(_abi.SPA_ERR_CAPACITY) == b"SPA_ERR_CAPACITY"
     assert L.spa_status_string(99) == b"SPA_ERR_UNKNOWN"
 
@@ -128,3 +128,14 @@ def test_static_status_rejects_null_bits():
 def test_test_stall_rejects_unknown_bits():
     assert spa.lib().spa_test_stall(4) == _abi.SPA_ERR_INVALID_ARG
     assert spa.lib().spa_test_stall(0) == _abi.SPA_OK
+
+
+def test_timed_prefills_reject_missing_events():
+    # the events are checked before any argument that would need a GPU
+    L = spa.lib()
+    a = _abi.SpaPrefillArgs()
+    b = _abi.SpaPbsArgs()
+    none2 = (ctypes.c_void_p * 2)(None, None)
+    for fn, args in ((L.spa_prefill_shared_timed, a), (L.spa_pbs_prefill_timed, b)):
+        assert fn(ctypes.byref(args), ctypes.c_void_p(16), 1 << 20, None, None) == _abi.SPA_ERR_INVALID_ARG
+        assert fn(ctypes.byref(args), ctypes.c_void_p(16), 1 << 20, None, none2) == _abi.SPA_ERR_INVALID_ARG
