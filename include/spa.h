@@ -373,7 +373,7 @@ spa_status spa_rla_state(const uint16_t* K, const uint16_t* V, int B, int Hkv, i
  *                 positions [t0, t] (causal), for every query t of the block and head h of g.
  * Attention runs on tcgen05 tensor cores with TMEM accumulators.  Requires d = 128,
  * bq = 64, G = Hq / Hkv even, T a multiple of bq with T / bq <= 128, q_start + T <= N,
- * cap >= min(N, topk + sink).  ws >= spa_prefill_workspace_bytes.
+ * cap >= min(N, topk + sink), sm_scale > 0.  ws >= spa_prefill_workspace_bytes.
  */
 typedef struct spa_prefill_args {
     int T, Hq, Hkv, N, d, r;
@@ -441,7 +441,7 @@ size_t spa_prefill_per_query_workspace_bytes(const spa_prefill_args* a);
  *              [seg0, t0) and the block's own positions up to t (causal), on tcgen05.
  * Queries are not permuted, so no inverse permutation of the output is needed.
  * Requires d = 128, b = 64, G = Hq / Hkv even and <= 8, T and S multiples of b, S <= 8192,
- * topk * b <= 8192, cap >= topk * b.  ws >= spa_pbs_workspace_bytes.
+ * topk * b <= 8192, cap >= topk * b, sm_scale > 0.  ws >= spa_pbs_workspace_bytes.
  */
 typedef struct spa_pbs_args {
     int T, Hq, Hkv, d;

@@ -423,7 +423,7 @@ static spa_status prefill_impl(const spa_prefill_args* a, void* ws, size_t ws_by
                                void* const* events) {
     if (!a || !ws) return SPA_ERR_INVALID_ARG;
     if (a->T < 0 || a->N <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->bq <= 0 ||
-        a->q_start < 0 || a->topk < 0 || a->sink < 0 || a->cap < 0)
+        a->q_start < 0 || a->topk < 0 || a->sink < 0 || a->cap < 0 || !(a->sm_scale > 0.f))
         return SPA_ERR_INVALID_ARG;
     if (a->T == 0) return SPA_OK;
     if (!a->Q || !a->q_idx || !a->K || !a->V || !a->Kidx || !a->idx || !a->count || !a->out)

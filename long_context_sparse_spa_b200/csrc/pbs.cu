@@ -360,7 +360,7 @@ extern "C" size_t spa_pbs_workspace_bytes(const spa_pbs_args* a) {
 static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, void* stream, void* const* events) {
     if (!a || !ws) return SPA_ERR_INVALID_ARG;
     if (a->T <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->b <= 0 || a->S <= 0 || a->topk < 0 ||
-        a->cap < 0)
+        a->cap < 0 || !(a->sm_scale > 0.f))
         return SPA_ERR_INVALID_ARG;
     if (!a->Q || !a->K || !a->V || !a->perm || !a->idx || !a->count || !a->out) return SPA_ERR_INVALID_ARG;
     if (!pbs_shape_ok(a)) return SPA_ERR_UNSUPPORTED_SHAPE;

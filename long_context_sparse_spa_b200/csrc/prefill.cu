@@ -20,115 +20,62 @@
 // (cp.async, bounds-checked) plus the diagonal tile of the block's own 64 positions, in one
 // pass with an online softmax (see the attention section below).
 #include "internal.cuh"
+#include "tc.cuh"
 
 namespace spa {
 namespace {
+using namespace tc;
 
 constexpr int kPfRows = 128;          // query rows per CTA (tensor-core M)
 constexpr int kPfKeys = 128;          // keys per tile (tensor-core N of S, K of P V)
-constexpr int kSlab = kPfRows * 128;  // bytes of one 64-column slab of a 128-row operand
-constexpr int kTileBytes = 2 * kSlab; // 128 rows x 128 bf16
 constexpr uint32_t kSpinLimit = 1u << 22;   // bounded mbarrier polls before giving up
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0));
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(slot)),
-                 "r"(ncols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols));
-}
-// D[tmem] (+)= A[smem] * B[smem], bf16 inputs, fp32 accumulate
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format, version 1).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
-    d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
-    d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
-    d |= uint64_t(1) << 46;
-    d |= uint64_t(2) << 61;
-    return d;
-}
-// Instruction descriptor of kind::f16: fp32 D, bf16 A and B, A K-major, B K- or MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) |
-           (uint32_t(M >> 4) << 24);
-}
-
-// byte offset of 16-byte chunk c (0..15) of row r in a 128-row, two-slab operand tile
-__device__ __forceinline__ uint32_t tile_off(int r, int c) {
-    return uint32_t((c >> 3) * kSlab + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
 // ============================================================================ index query
-// qhat[u][0..15] (fp32) = mean over the block's bq queries and G heads of q_idx, summed in
-// (query, head) order; also unit_len[u] = t0, the number of candidate keys.
-__global__ void prefill_qhat_kernel(const uint16_t* __restrict__ qidx, int Hq, int Hkv, int bq, int q_start,
-                                    float* __restrict__ qhat, int32_t* __restrict__ unit_len, int U) {
+// qhat[u][0..15] (fp32) = mean over the block's bq queries and G heads of q_idx; also
+// unit_len[u] = t0, the number of candidate keys.  One CTA per unit: thread j takes the rows
+// (query, head) = j, j + 256, ... (in (query, head) order) as two 16-byte loads each, and the
+// partial sums are added in a fixed tree (lanes, then warps in order), so the result does not
+// depend on scheduling.
+__global__ void __launch_bounds__(256)
+prefill_qhat_kernel(const uint16_t* __restrict__ qidx, int Hq, int Hkv, int bq, int q_start,
+                    float* __restrict__ qhat, int32_t* __restrict__ unit_len, int U) {
     pdl_enter();
-    const int u = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16;
-    const int dim = threadIdx.x & 15;
+    __shared__ float part[8][16];
+    const int u = blockIdx.x;
     if (u >= U) return;
     const int blk = u / Hkv, g = u - blk * Hkv;
     const int G = Hq / Hkv;
-    float acc = 0.f;
-    for (int i = 0; i < bq; ++i)
-        for (int h = 0; h < G; ++h)
-            acc += __uint_as_float(uint32_t(qidx[(size_t(blk * bq + i) * Hq + g * G + h) * 16 + dim]) << 16);
-    qhat[u * 16 + dim] = acc / float(bq * G);
-    if (dim == 0) unit_len[u] = q_start + blk * bq;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float acc[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+    for (int j = tid; j < bq * G; j += 256) {
+        const int i = j / G, h = j - i * G;
+        const uint4* row = reinterpret_cast<const uint4*>(qidx + (size_t(blk * bq + i) * Hq + g * G + h) * 16);
+        const uint4 w0 = __ldg(row), w1 = __ldg(row + 1);
+        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            acc[2 * k] += __uint_as_float(ws[k] << 16);
+            acc[2 * k + 1] += __uint_as_float(ws[k] & 0xffff0000u);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], off);
+    if (lane == 0)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) part[warp][c] = acc[c];
+    __syncthreads();
+    if (tid < 16) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += part[w][tid];
+        qhat[u * 16 + tid] = t / float(bq * G);
+    }
+    if (tid == 0) unit_len[u] = q_start + blk * bq;
 }
 
 // ============================================================================ scores
@@ -201,22 +148,6 @@ struct __align__(1024) PfShared {
     uint32_t valid[4][kPfKeys / 32];   // bit c: key c of tile t (slot t % 4) is attended
 };
 
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n" ::"r"(
-            taddr),
-        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
-        "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
-        "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
-        "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 // grid (U, G / 2): one CTA per (unit, pair of query heads); 256 threads.
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -379,7 +310,7 @@ prefill_attend_kernel(PrefillAttendParams p) {
             pend_s = true;
         }
 
-        // this thread's 64 logits of S(t), in log2 units, masked
+        // this thread's 64 logits of S(t)
         float s[64];
         {
             float v[32];
@@ -392,39 +323,48 @@ prefill_attend_kernel(PrefillAttendParams p) {
             for (int i = 0; i < 32; ++i) s[32 + i] = v[i];
         }
         tc_fence_before();
+        // raw logits; masked keys become -inf.  A full tile of support keys (every tile but the
+        // last partial one and the diagonal) needs no mask: the test is warp-uniform
         const uint32_t vm0 = sh.valid[t & 3][2 * half], vm1 = sh.valid[t & 3][2 * half + 1];
-        const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
-        float tmax = -INFINITY;
+        if (!(t < n_gather && (vm0 & vm1) == 0xffffffffu)) {
+            const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const bool valid = (((i < 32 ? vm0 : vm1) >> (i & 31)) & 1u) && i <= causal;
-            s[i] = valid ? s[i] * sl2 : -INFINITY;
-            tmax = fmaxf(tmax, s[i]);
+            for (int i = 0; i < 64; ++i) {
+                const bool valid = (((i < 32 ? vm0 : vm1) >> (i & 31)) & 1u) && i <= causal;
+                s[i] = valid ? s[i] : -INFINITY;
+            }
         }
+        // tile maximum in four independent chains, then in log2 units (sm_scale > 0)
+        float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+        const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         bool rescale = false;
         float alpha = 1.f;
         if (tmax > m_run + kRescaleLog2) {                    // also the first finite maximum
-            alpha = exp2f(m_run - tmax);
+            alpha = ex2_approx(m_run - tmax);
             rescale = m_run != -INFINITY;                      // O of this half holds nonzero terms
             m_run = tmax;
             l_run *= alpha;
         }
-        // P = 2^(s - m) as bf16 hi + lo pairs
+        // P = 2^(sl2 s - m) as bf16 hi + lo pairs (masked keys give 2^-inf = 0; while no key has
+        // been seen m is -inf and every logit is -inf, so the reference 0 gives P = 0)
+        const float mu = m_run == -INFINITY ? 0.f : m_run;
         uint32_t hw[32], lw[32];
-        float add = 0.f;
+        float add4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const float p0 = m_run == -INFINITY ? 0.f : exp2f(s[2 * j] - m_run);
-            const float p1 = m_run == -INFINITY ? 0.f : exp2f(s[2 * j + 1] - m_run);
-            add += p0;
-            add += p1;
+            const float p0 = ex2_approx(fmaf(s[2 * j], sl2, -mu));
+            const float p1 = ex2_approx(fmaf(s[2 * j + 1], sl2, -mu));
+            add4[(2 * j) & 3] += p0;
+            add4[(2 * j + 1) & 3] += p1;
             const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
             const float2 hf = __bfloat1622float2(h);
             const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
             hw[j] = *reinterpret_cast<const uint32_t*>(&h);
             lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
         }
-        l_run += add;
+        l_run += (add4[0] + add4[1]) + (add4[2] + add4[3]);
 
         // P(t-1) V(t-1) is complete: P, O and its V buffer are free
         ok = t == 0 || wait_bar(&sh.bar_o, ph_o);
@@ -567,7 +507,7 @@ spa_status launch_prefill(const spa_prefill_args* a, void* ws, cudaStream_t st, 
     w += align_up(size_t(U) * a->N * 4, 256);
     const Hist0 hist = hist0_carve(w, U);
 
-    SPA_CUDA_TRY(launch_pdl(prefill_qhat_kernel, dim3((U + 15) / 16), dim3(256), 0, st, a->q_idx, a->Hq, a->Hkv, a->bq,
+    SPA_CUDA_TRY(launch_pdl(prefill_qhat_kernel, dim3(U), dim3(256), 0, st, a->q_idx, a->Hq, a->Hkv, a->bq,
                             a->q_start, qhat, unit_len, U));
     SPA_CUDA_TRY(launch_pdl(prefill_scores_kernel, dim3((a->N + kPsThreads - 1) / kPsThreads, a->Hkv), dim3(kPsThreads),
                             0, st, qhat, unit_len, reinterpret_cast<const uint4*>(a->Kidx), a->Hkv, a->N, n_blocks,

@@ -673,13 +673,21 @@ int max_active_clusters(int C, size_t smem) {
     return v;
 }
 
+// Cluster size C for U units of M scores.  A configuration runs ceil(U / concurrent units)
+// waves of CTAs that each scan M / C scores plus a fixed cost (level-0 resolution, barriers,
+// histogram merges) worth about kSelFixed scores; a chunk too long for shared memory streams
+// from L2 on every level (kSelStreamCost per score).  The cheapest estimate wins, ties to the
+// larger cluster; C > 1 needs at least 2048 scores per CTA.  When every unit's cluster fits in
+// one wave this is the largest such C, as before.
+constexpr double kSelFixed = 4096.0;
+constexpr double kSelStreamCost = 3.0;
 template <bool TOPP>
 SelectConfig choose(int U, int M) {
     const DeviceInfo& di = device_info();
     const size_t fixed = align_up(sizeof(SelShared), 16);
     SelectConfig best{};
     best.C = 0;
-    // largest cluster (<= 16) that keeps every unit's cluster in one wave and >= 2048 scores per CTA
+    double best_cost = 0.0;
     cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     for (int C = kMaxCluster; C >= 1; C /= 2) {
         if (C > 1 && (M + C - 1) / C < 2048) continue;
@@ -691,10 +699,24 @@ SelectConfig choose(int U, int M) {
             smem = fixed;
         }
         cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        const int active = C > 1 ? max_active_clusters<TOPP>(C, smem) : U;
-        if (C == 1 || U <= active) {
+        int active = 0;   // units whose CTAs run at once
+        if (C > 1) {
+            active = max_active_clusters<TOPP>(C, smem);
+        } else {
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<TOPP>, kSelThreads, smem) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                per_sm = 1;
+            }
+            active = per_sm * di.num_sms;
+        }
+        if (active <= 0) continue;
+        const double waves = double((U + active - 1) / active);
+        const double cost = waves * (double(chunk) * (resident ? 1.0 : kSelStreamCost) + kSelFixed);
+        if (best.C == 0 || cost < best_cost) {
             best = SelectConfig{C, chunk, resident, smem};
-            break;
+            best_cost = cost;
         }
     }
     if (best.C == 0) best = SelectConfig{1, M, 0, fixed};
