@@ -16,17 +16,17 @@
 //      selection-block-shared prefill -- on the tcgen05 attention kernel.  Queries are not
 //      permuted, so no inverse permutation of the output is needed.
 //
-// Steps 1-3 are CUDA-core kernels (the importance pass is a b*G x T x d contraction done once
-// per prefill); step 3's top-k is the library's exact selection with a per-unit candidate
-// length.
+// Step 1 is a b*G x T x d contraction and runs on tcgen05 (two passes: row statistics, then the
+// probabilities' column sums); steps 2-3 are CUDA-core kernels, and step 3's top-k is the
+// library's exact selection with a per-unit candidate length.
 #include "internal.cuh"
+#include "tc.cuh"
 
 namespace spa {
 namespace {
 
 constexpr int kPbThreads = 256;
-constexpr int kPbKeys = 128;       // keys per CTA in the importance passes
-constexpr int kPbRows = 256;       // query rows held in shared memory at once
+constexpr int kPbKeys = 128;       // keys per importance tile
 constexpr int kPbD = 128;
 constexpr float kPbLog2e = 1.4426950408889634f;
 
@@ -35,8 +35,8 @@ struct PbsParams {
     const uint16_t* K;   // [Hkv, T, d]
     int T, Hq, Hkv, G, b, S, R, ntiles, nblk;
     float sm_scale;
-    float* rm;           // [Hkv][ntiles][R] per-tile row max (log2 units)
-    float* rl;           // [Hkv][ntiles][R] per-tile row sum
+    float* rm;           // [Hkv][ntiles][R] per-chunk row max (log2 units); ntiles = the chunk count
+    float* rl;           // [Hkv][ntiles][R] per-chunk row sum
     float* M;            // [Hkv][R]
     float* L;            // [Hkv][R]
     float* imp;          // [Hkv][T]
@@ -58,69 +58,211 @@ struct PbsParams {
 
 __device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(uint32_t(v) << 16); }
 
-// Stage the key tile [n0, n0 + kPbKeys) of kv head g (fp32, zero past T) and rows [rc, rc +
-// kPbRows) of the last query block (transposed: qT[c][r], zero past R) in shared memory.
-__device__ void pb_stage(const PbsParams& p, int g, int n0, int rc, float* ks, float* qT) {
-    for (int i = threadIdx.x; i < kPbKeys * kPbD; i += kPbThreads) {
-        const int k = i / kPbD, c = i - k * kPbD, n = n0 + k;
-        ks[i] = n < p.T ? bf(p.K[(size_t(g) * p.T + n) * kPbD + c]) : 0.f;
-    }
-    for (int i = threadIdx.x; i < kPbRows * kPbD; i += kPbThreads) {
-        const int rr = i % kPbRows, c = i / kPbRows, r = rc + rr;
-        float v = 0.f;
-        if (r < p.R) {
-            const int qi = p.T - p.b + r / p.G, h = r % p.G;
-            v = bf(p.Q[(size_t(qi) * p.Hq + g * p.G + h) * kPbD + c]);
-        }
-        qT[c * kPbRows + rr] = v;
+// ---------------------------------------------------------------------------- importance
+// The importance passes are R x T x d contractions (R = b * G rows of the last query block
+// against every key of the kv head) and run on tcgen05: S = Q_last K_tile^T into TMEM, one
+// 128 x 128 MMA tile per 128 rows, one thread per row.  R = 128 * NMT rows are staged once
+// (row r: query T - b + r / G, head r % G); a CTA then walks a chunk of kImTiles key tiles with
+// double-buffered cp.async.
+//   PASS 0: per row, the max and sum of 2^(sm_scale log2e s) over the chunk's keys the row may
+//           see (keys after its query count nothing) -> rm / rl [g][chunk][r];
+//   PASS 1: per key, sum over rows of 2^(sm_scale log2e s - M_r) / L_r (M, L: the combined row
+//           statistics).  A warp sums its 32 rows per column with a transposing butterfly of
+//           shuffles (five steps over each half of the tile, the live columns halving at each),
+//           the warps are then added in order, so the sum is in a fixed order.
+constexpr int kImTiles = 16;              // key tiles of 128 per CTA
+constexpr uint32_t kImSpinLimit = 1u << 22;
+
+// One step of a transposing butterfly over a warp: each lane holds 2 HF live columns of its
+// row; it keeps the half selected by (lane & MK), adds its partner's copy of that half, and hands
+// the other half to the partner.  Five steps from 64 columns leave every lane with the warp's
+// sums of 2 columns.
+template <int HF, int MK>
+__device__ __forceinline__ void bfly_step(float (&v)[64], int lane) {
+    const bool up = (lane & MK) != 0;
+#pragma unroll
+    for (int i = 0; i < HF; ++i) {
+        const float send = up ? v[i] : v[HF + i];
+        const float keep = up ? v[HF + i] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, MK);
     }
 }
 
-// scaled logit (log2 units) of staged row rr and staged key k, channels in ascending order
-__device__ __forceinline__ float pb_logit(const float* qT, const float* ks, int rr, int k, float sl2) {
-    float dot = 0.f;
-    const float4* k4 = reinterpret_cast<const float4*>(ks + k * kPbD);
-#pragma unroll 8
-    for (int c4 = 0; c4 < kPbD / 4; ++c4) {
-        const float4 kv = k4[c4];
-        dot = fmaf(qT[(4 * c4 + 0) * kPbRows + rr], kv.x, dot);
-        dot = fmaf(qT[(4 * c4 + 1) * kPbRows + rr], kv.y, dot);
-        dot = fmaf(qT[(4 * c4 + 2) * kPbRows + rr], kv.z, dot);
-        dot = fmaf(qT[(4 * c4 + 3) * kPbRows + rr], kv.w, dot);
-    }
-    return dot * sl2;
-}
+template <int NMT>
+struct __align__(1024) ImShared {
+    uint8_t q[NMT][tc::kTileBytes];
+    uint8_t k[2][tc::kTileBytes];
+    uint64_t bar;
+    uint32_t tmem_base;
+    float colsum[4 * NMT][128];           // PASS 1: per-warp column sums of a tile
+};
 
-// pass 1: per key tile, every row's max and sum of exp2 over the tile's keys it may see
-__global__ void __launch_bounds__(kPbThreads) pbs_rowstats_kernel(PbsParams p) {
+template <int NMT, int PASS>
+__global__ void __launch_bounds__(128 * NMT, 1) pbs_importance_tc_kernel(PbsParams p, uint32_t* status) {
+    using namespace tc;
     pdl_enter();
-    extern __shared__ __align__(16) float pbs_smem[];
-    float* ks = pbs_smem;
-    float* qT = pbs_smem + kPbKeys * kPbD;
-    const int g = blockIdx.y, kt = blockIdx.x;
-    const int n0 = kt * kPbKeys, n1 = min(p.T, n0 + kPbKeys);
+    extern __shared__ __align__(1024) uint8_t dyn[];
+    ImShared<NMT>& sh = *reinterpret_cast<ImShared<NMT>*>(dyn);
+    constexpr int R = 128 * NMT, NT = 128 * NMT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = blockIdx.y, chunk = blockIdx.x;
+    const int n_all = (p.T + 127) / 128;
+    const int t_begin = chunk * kImTiles, t_end = min(n_all, t_begin + kImTiles);
+    const int r = tid;                                          // this thread's row
+    const int t_row = p.T - p.b + r / p.G;                      // its query position
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t col_off = uint32_t(warp >> 2) * 128;         // TMEM columns of its operand tile
     const float sl2 = p.sm_scale * kPbLog2e;
-    for (int rc = 0; rc < p.R; rc += kPbRows) {
-        __syncthreads();
-        pb_stage(p, g, n0, rc, ks, qT);
-        __syncthreads();
-        const int r = rc + threadIdx.x;
-        if (r >= p.R) continue;
-        const int t_row = p.T - p.b + r / p.G;
-        const int kend = min(n1, t_row + 1);
-        float m = -INFINITY, l = 0.f;
-        for (int n = n0; n < kend; ++n) {
-            const float x = pb_logit(qT, ks, threadIdx.x, n - n0, sl2);
-            const float mn = fmaxf(m, x);
-            l = l * exp2f(m - mn) + exp2f(x - mn);
-            m = mn;
+    constexpr uint32_t kId = idesc_bf16(128, 128, false);
+
+    constexpr uint32_t kCols = NMT <= 1 ? 128 : (NMT <= 2 ? 256 : 512);   // a power of 2
+    if (warp == 0) tmem_alloc(&sh.tmem_base, kCols);
+    if (tid == 0) {
+        mbar_init(&sh.bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    // Q rows, then the first key tile, in one cp.async group
+    for (int i = tid; i < R * 16; i += NT) {
+        const int row = i >> 4, c = i & 15;
+        const size_t q = size_t(p.T - p.b + row / p.G) * p.Hq + size_t(g) * p.G + row % p.G;
+        cp_async16(smem_u32(sh.q[row >> 7]) + tile_off(row & 127, c), p.Q + q * kPbD + c * 8, true);
+    }
+    auto issue = [&](int t) {
+        if (t < t_end) {
+            for (int i = tid; i < 128 * 16; i += NT) {
+                const int kr = i >> 4, c = i & 15, n = t * 128 + kr;
+                const bool ok = n < p.T;
+                cp_async16(smem_u32(sh.k[t & 1]) + tile_off(kr, c), p.K + (ok ? (size_t(g) * p.T + n) * kPbD + c * 8 : 0),
+                           ok);
+            }
         }
-        p.rm[(size_t(g) * p.ntiles + kt) * p.R + r] = m;
-        p.rl[(size_t(g) * p.ntiles + kt) * p.R + r] = l;
+        cp_async_commit();
+    };
+    issue(t_begin);
+    const float Mr = PASS == 1 ? p.M[size_t(g) * R + r] : 0.f;
+    const float inv_l = PASS == 1 ? 1.f / p.L[size_t(g) * R + r] : 0.f;
+    float m = -INFINITY, l = 0.f;
+    uint32_t phase = 0;
+    bool my_to = false, pending = false, stopped = false;
+    uint32_t tmem = 0;
+    for (int t = t_begin; t < t_end; ++t) {
+        issue(t + 1);                                           // the next tile's buffer was read by S(t - 1)
+        cp_async_wait_group<1>();                               // tile t (and Q) landed
+        fence_async_smem();
+        tc_fence_before();
+        stopped = __syncthreads_or(my_to) != 0;                 // also: S(t - 1) and colsum read by everyone
+        tc_fence_after();
+        if (stopped) break;
+        tmem = sh.tmem_base;
+        if (tid == 0) {
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
+                    umma_bf16(tmem + mt * 128, sw128_desc(smem_u32(sh.q[mt]) + off, 16, 1024),
+                              sw128_desc(smem_u32(sh.k[t & 1]) + off, 16, 1024), kId, kk > 0);
+                }
+            umma_commit(&sh.bar);
+        }
+        pending = true;
+        {
+            uint32_t it = 0;
+            bool done = true;
+            while (!mbar_try_wait(&sh.bar, phase))
+                if (++it >= kImSpinLimit) {
+                    done = false;
+                    my_to = true;
+                    break;
+                }
+            if (done) {
+                pending = false;
+                phase ^= 1u;
+            }
+        }
+        stopped = __syncthreads_or(my_to) != 0;                 // every thread takes the same path
+        tc_fence_after();
+        if (stopped) break;
+        // this row's 128 logits of the tile, in two halves of 64 columns
+        const int n0 = t * 128;
+        const int lim = min(p.T - 1, t_row) - n0;               // keys c <= lim are seen by this row
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[64];
+            {
+                float w[32];
+                tmem_ld32(tmem + col_off + lane_off + hh * 64, w);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = w[i];
+                tmem_ld32(tmem + col_off + lane_off + hh * 64 + 32, w);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[32 + i] = w[i];
+            }
+            const int lh = lim - hh * 64;
+            if (PASS == 0) {
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    v[c] = c <= lh ? v[c] * sl2 : -INFINITY;
+                    tmax = fmaxf(tmax, v[c]);
+                }
+                if (tmax != -INFINITY) {
+                    const float mn = fmaxf(m, tmax);
+                    float add = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) add += exp2f(v[c] - mn);
+                    l = l * exp2f(m - mn) + add;
+                    m = mn;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) v[c] = c <= lh ? exp2f(fmaf(v[c], sl2, -Mr)) * inv_l : 0.f;
+                bfly_step<32, 16>(v, lane);
+                bfly_step<16, 8>(v, lane);
+                bfly_step<8, 4>(v, lane);
+                bfly_step<4, 2>(v, lane);
+                bfly_step<2, 1>(v, lane);
+                // this lane now holds the warp's sums of columns c0, c0 + 1 of the half
+                const int c0 = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
+                               ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+                sh.colsum[warp][hh * 64 + c0] = v[0];
+                sh.colsum[warp][hh * 64 + c0 + 1] = v[1];
+            }
+        }
+        tc_fence_before();
+        if (PASS == 1) {
+            __syncthreads();
+            if (tid < 128 && n0 + tid < p.T) {
+                float tot = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4 * NMT; ++w) tot += sh.colsum[w][tid];
+                p.imp[size_t(g) * p.T + n0 + tid] = tot / float(R);
+            }
+        }
+    }
+    cp_async_wait_all();
+    tc_fence_before();
+    const bool good = __syncthreads_or(my_to) == 0;
+    if (PASS == 0 && good) {
+        p.rm[(size_t(g) * p.ntiles + chunk) * R + r] = m;
+        p.rl[(size_t(g) * p.ntiles + chunk) * R + r] = l;
+    }
+    if (!good && tid == 0) raise_status(status, SPA_ERR_TIMEOUT);
+    // an MMA that was not seen to complete may still be running: wait once more (bounded) and
+    // free the tensor memory only when nothing is owed
+    if (pending) {
+        uint32_t it = 0;
+        while (!mbar_try_wait(&sh.bar, phase) && ++it < kImSpinLimit) {
+        }
+        pending = it >= kImSpinLimit;
+    }
+    if (warp == 0 && !__any_sync(0xffffffffu, pending)) {
+        tc_fence_after();
+        tmem_dealloc(sh.tmem_base, kCols);
     }
 }
 
-// every row's max and sum over all tiles (tile order)
+// every row's max and sum over all chunks (chunk order)
 __global__ void __launch_bounds__(kPbThreads) pbs_rowcombine_kernel(PbsParams p) {
     pdl_enter();
     const int g = blockIdx.y;
@@ -135,47 +277,6 @@ __global__ void __launch_bounds__(kPbThreads) pbs_rowcombine_kernel(PbsParams p)
     }
     p.M[size_t(g) * p.R + r] = M;
     p.L[size_t(g) * p.R + r] = L;
-}
-
-// pass 2: importance of the tile's keys: sum over rows of exp2(x - M_r) / L_r, divided by R;
-// rows are summed within a warp in lane order, then over warps and row chunks in order
-__global__ void __launch_bounds__(kPbThreads) pbs_importance_kernel(PbsParams p) {
-    pdl_enter();
-    extern __shared__ __align__(16) float pbs_smem[];
-    float* ks = pbs_smem;
-    float* qT = pbs_smem + kPbKeys * kPbD;
-    float* part = qT + kPbD * kPbRows;   // [warps][kPbKeys]
-    const int g = blockIdx.y, kt = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n0 = kt * kPbKeys, n1 = min(p.T, n0 + kPbKeys);
-    const float sl2 = p.sm_scale * kPbLog2e;
-    float acc = 0.f;   // thread k < kPbKeys: the running sum of key n0 + k
-    for (int rc = 0; rc < p.R; rc += kPbRows) {
-        __syncthreads();
-        pb_stage(p, g, n0, rc, ks, qT);
-        __syncthreads();
-        const int r = rc + threadIdx.x;
-        const bool live = r < p.R;
-        const int t_row = live ? p.T - p.b + r / p.G : -1;
-        const float Mr = live ? p.M[size_t(g) * p.R + r] : 0.f;
-        const float inv_l = live ? 1.f / p.L[size_t(g) * p.R + r] : 0.f;
-        for (int k = 0; k < n1 - n0; ++k) {
-            const int n = n0 + k;
-            float pr = 0.f;
-            if (live && n <= t_row) pr = exp2f(pb_logit(qT, ks, threadIdx.x, k, sl2) - Mr) * inv_l;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) pr += __shfl_xor_sync(0xffffffffu, pr, off);
-            if (lane == 0) part[warp * kPbKeys + k] = pr;
-        }
-        __syncthreads();
-        if (threadIdx.x < kPbKeys) {
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < kPbThreads / 32; ++w) s += part[w * kPbKeys + threadIdx.x];
-            acc += s;
-        }
-    }
-    if (threadIdx.x < n1 - n0) p.imp[size_t(g) * p.T + n0 + threadIdx.x] = acc / float(p.R);
 }
 
 // sort each segment by (importance desc, position asc): bitonic sort of 64-bit keys
@@ -413,15 +514,26 @@ static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, voi
     p.aidx = reinterpret_cast<int32_t*>(b + l.aidx);
     p.acount = reinterpret_cast<int32_t*>(b + l.acount);
 
-    // 1. importance
-    const size_t smem1 = size_t(kPbKeys) * kPbD * 4 + size_t(kPbD) * kPbRows * 4;
-    const size_t smem2 = smem1 + size_t(kPbThreads / 32) * kPbKeys * 4;
-    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_rowstats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem1)));
-    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_importance_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem2)));
-    SPA_CUDA_TRY(launch_pdl(pbs_rowstats_kernel, dim3(p.ntiles, a->Hkv), dim3(kPbThreads), smem1, st, p));
-    SPA_CUDA_TRY(launch_pdl(pbs_rowcombine_kernel, dim3((p.R + kPbThreads - 1) / kPbThreads, a->Hkv),
-                            dim3(kPbThreads), 0, st, p));
-    SPA_CUDA_TRY(launch_pdl(pbs_importance_kernel, dim3(p.ntiles, a->Hkv), dim3(kPbThreads), smem2, st, p));
+    // 1. importance (tcgen05): row statistics per key chunk, combined per row, then the column sums
+    const int nchunk = (p.ntiles + kImTiles - 1) / kImTiles;
+    p.ntiles = nchunk;                                        // rm / rl hold one record per chunk
+    const int nmt = p.R / 128;
+#define SPA_PB_IMP(NMT)                                                                                         \
+    if (nmt == NMT) {                                                                                           \
+        const size_t sm = sizeof(ImShared<NMT>);                                                                \
+        SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_importance_tc_kernel<NMT, 0>,                                     \
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));               \
+        SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_importance_tc_kernel<NMT, 1>,                                     \
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));               \
+        SPA_CUDA_TRY(launch_pdl(pbs_importance_tc_kernel<NMT, 0>, dim3(nchunk, a->Hkv), dim3(128 * NMT), sm, st,  \
+                                p, status));                                                                    \
+        SPA_CUDA_TRY(launch_pdl(pbs_rowcombine_kernel, dim3((p.R + kPbThreads - 1) / kPbThreads, a->Hkv),        \
+                                dim3(kPbThreads), 0, st, p));                                                   \
+        SPA_CUDA_TRY(launch_pdl(pbs_importance_tc_kernel<NMT, 1>, dim3(nchunk, a->Hkv), dim3(128 * NMT), sm, st,  \
+                                p, status));                                                                    \
+    }
+    SPA_PB_IMP(1) else SPA_PB_IMP(2) else SPA_PB_IMP(3) else SPA_PB_IMP(4) else return SPA_ERR_UNSUPPORTED_SHAPE;
+#undef SPA_PB_IMP
     // 2. permutation inside segments
     int P = 1;
     while (P < a->S) P <<= 1;
