@@ -17,8 +17,10 @@
 //      permuted, so no inverse permutation of the output is needed.
 //
 // Step 1 is a b*G x T x d contraction and runs on tcgen05 (two passes: row statistics, then the
-// probabilities' column sums); steps 2-3 are CUDA-core kernels, and step 3's top-k is the
-// library's exact selection with a per-unit candidate length.
+// probabilities' column sums); steps 2-3 are CUDA-core kernels: the block scores as a tiled
+// product of the block means, the top-k as a per-unit bitonic sort of (score, block) keys (a
+// unit has at most T / b candidates), and the support as a bitmap of positions compacted in
+// ascending order.
 #include "internal.cuh"
 #include "tc.cuh"
 
@@ -44,9 +46,8 @@ struct PbsParams {
     float* kbar;         // [Hkv][nblk][d]
     float* qbar;         // [nblk][Hkv][d]
     float* scores;       // [U][nblk]
-    int32_t* unit_len;   // [U]
-    const int32_t* bidx; // [U][topk] selected blocks
-    const int32_t* bcount;
+    int32_t* bidx;       // [U][topk] selected blocks
+    int32_t* bcount;
     int topk;
     int32_t* idx;        // [U][cap] support (original positions, ascending)
     int32_t* count;
@@ -316,97 +317,185 @@ __global__ void __launch_bounds__(1024) pbs_sort_kernel(PbsParams p) {
 }
 
 // z = 0: kbar of permuted key block blockIdx.x; z = 1: qbar of query block blockIdx.x (mean over
-// its b queries and G heads, in (query, head) order); one thread per channel
+// its b queries and G heads, in (query, head) order); one thread per channel.  The block's 64
+// permuted positions are staged in shared memory first; loads are then issued eight at a time
+// and the sums keep their sequential order.
 __global__ void __launch_bounds__(kPbD) pbs_means_kernel(PbsParams p) {
     pdl_enter();
+    __shared__ int32_t pm[64];
     const int blk = blockIdx.x, g = blockIdx.y, c = threadIdx.x;
     float s = 0.f;
     if (blockIdx.z == 0) {
-        const int32_t* pm = p.perm + size_t(g) * p.T + size_t(blk) * p.b;
-        for (int i = 0; i < p.b; ++i) s += bf(p.K[(size_t(g) * p.T + pm[i]) * kPbD + c]);
+        if (c < p.b) pm[c] = p.perm[size_t(g) * p.T + size_t(blk) * p.b + c];   // b = 64
+        __syncthreads();
+        const uint16_t* kg = p.K + size_t(g) * p.T * kPbD + c;
+        for (int i = 0; i < p.b; i += 8) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = bf(kg[size_t(pm[i + e]) * kPbD]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += v[e];
+        }
         p.kbar[(size_t(g) * p.nblk + blk) * kPbD + c] = s / float(p.b);
     } else {
-        for (int i = 0; i < p.b; ++i)
-            for (int h = 0; h < p.G; ++h) s += bf(p.Q[(size_t(blk * p.b + i) * p.Hq + g * p.G + h) * kPbD + c]);
+        // rows (query i, head h) in (i, h) order; b * G is a multiple of 8
+        const uint16_t* qb = p.Q + (size_t(blk) * p.b * p.Hq + size_t(g) * p.G) * kPbD + c;
+        int i = 0, h = 0;
+        for (int f = 0; f < p.b * p.G; f += 8) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[e] = bf(qb[(size_t(i) * p.Hq + h) * kPbD]);
+                if (++h == p.G) {
+                    h = 0;
+                    ++i;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += v[e];
+        }
         p.qbar[(size_t(blk) * p.Hkv + g) * kPbD + c] = s / float(p.b * p.G);
     }
 }
 
-// block scores of unit u = j * Hkv + g over the permuted blocks before its own segment
+// Block scores sm_scale * qbar . kbar over the permuted blocks before each query block's own
+// segment.  CTA per (kv head g, kPbJ consecutive query blocks): their qbar rows sit in shared
+// memory; each thread takes key blocks c = tid, tid + 256, ..., loads kbar[c] once and forms the
+// dots with every query block of the tile that has c among its candidates.  Each dot runs over
+// the channels in ascending order.
+constexpr int kPbJ = 32;
 __global__ void __launch_bounds__(kPbThreads) pbs_scores_kernel(PbsParams p) {
     pdl_enter();
-    const int u = blockIdx.x, j = u / p.Hkv, g = u - j * p.Hkv;
-    const int seg0 = (j * p.b) / p.S * p.S;
-    const int nc = seg0 / p.b;
-    __shared__ float qb[kPbD];
-    if (threadIdx.x < kPbD) qb[threadIdx.x] = p.qbar[(size_t(j) * p.Hkv + g) * kPbD + threadIdx.x];
-    if (threadIdx.x == 0) p.unit_len[u] = nc;
+    __shared__ __align__(16) float qs[kPbJ][kPbD];
+    const int g = blockIdx.y, j0 = blockIdx.x * kPbJ;
+    const int nj = min(kPbJ, p.nblk - j0);
+    for (int i = threadIdx.x; i < nj * kPbD; i += kPbThreads)
+        qs[i / kPbD][i % kPbD] = p.qbar[(size_t(j0 + i / kPbD) * p.Hkv + g) * kPbD + i % kPbD];
     __syncthreads();
-    for (int c = threadIdx.x; c < nc; c += kPbThreads) {
-        const float4* kb = reinterpret_cast<const float4*>(p.kbar + (size_t(g) * p.nblk + c) * kPbD);
-        float dot = 0.f;
-#pragma unroll 8
-        for (int d4 = 0; d4 < kPbD / 4; ++d4) {
-            const float4 v = kb[d4];
-            dot = fmaf(qb[4 * d4 + 0], v.x, dot);
-            dot = fmaf(qb[4 * d4 + 1], v.y, dot);
-            dot = fmaf(qb[4 * d4 + 2], v.z, dot);
-            dot = fmaf(qb[4 * d4 + 3], v.w, dot);
+    const int nc_max = ((j0 + nj - 1) * p.b) / p.S * p.S / p.b;   // the tile's largest candidate count
+    for (int c = threadIdx.x; c < nc_max; c += kPbThreads) {
+        float4 kb[kPbD / 4];
+        const float4* k4 = reinterpret_cast<const float4*>(p.kbar + (size_t(g) * p.nblk + c) * kPbD);
+#pragma unroll
+        for (int d4 = 0; d4 < kPbD / 4; ++d4) kb[d4] = k4[d4];
+        for (int jj = 0; jj < nj; ++jj) {
+            const int j = j0 + jj;
+            if (c >= (j * p.b) / p.S * p.S / p.b) continue;
+            const float4* q4 = reinterpret_cast<const float4*>(qs[jj]);
+            float dot = 0.f;
+#pragma unroll
+            for (int d4 = 0; d4 < kPbD / 4; ++d4) {
+                const float4 q = q4[d4];
+                dot = fmaf(q.x, kb[d4].x, dot);
+                dot = fmaf(q.y, kb[d4].y, dot);
+                dot = fmaf(q.z, kb[d4].z, dot);
+                dot = fmaf(q.w, kb[d4].w, dot);
+            }
+            p.scores[size_t(j * p.Hkv + g) * p.nblk + c] = p.sm_scale * dot;
         }
-        p.scores[size_t(u) * p.nblk + c] = p.sm_scale * dot;
     }
 }
 
-// selected blocks -> their keys' original positions, ascending (support); the attention's
-// rows are the support followed by the own segment's keys before the block, [seg0, t0)
-__global__ void __launch_bounds__(kPbThreads) pbs_expand_kernel(PbsParams p) {
+// Block top-k of unit u: its nc candidate scores sorted by (score desc, block asc) with a
+// bitonic sort of 64-bit keys in shared memory; the first min(k, nc) blocks are kept.
+__global__ void __launch_bounds__(kPbThreads) pbs_topk_kernel(PbsParams p, int k) {
     pdl_enter();
-    extern __shared__ __align__(16) uint32_t pos[];
-    const int u = blockIdx.x, j = u / p.Hkv, g = u - j * p.Hkv;
-    const int t0 = j * p.b, seg0 = t0 / p.S * p.S;
-    int nb = p.bcount[u];
-    nb = nb < 0 ? 0 : (nb > p.topk ? p.topk : nb);
-    const int n = nb * p.b;
+    extern __shared__ __align__(16) unsigned long long tk[];
+    const int u = blockIdx.x, j = u / p.Hkv;
+    const int nc = (j * p.b) / p.S * p.S / p.b;
     int P = 1;
-    while (P < n) P <<= 1;
+    while (P < nc) P <<= 1;
     for (int i = threadIdx.x; i < P; i += kPbThreads) {
-        uint32_t v = 0xffffffffu;
-        if (i < n) {
-            const int blk = p.bidx[size_t(u) * p.topk + i / p.b];
-            v = uint32_t(p.perm[size_t(g) * p.T + size_t(blk) * p.b + (i % p.b)]);
+        unsigned long long key = ~0ull;
+        if (i < nc) {
+            const uint32_t sk = score_key(p.scores[size_t(u) * p.nblk + i]);
+            key = (static_cast<unsigned long long>(~sk) << 32) | uint32_t(i);
         }
-        pos[i] = v;
+        tk[i] = key;
     }
     __syncthreads();
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+    for (int kk = 2; kk <= P; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
             for (int i = threadIdx.x; i < P; i += kPbThreads) {
                 const int ixj = i ^ jj;
                 if (ixj > i) {
-                    const bool up = (i & k) == 0;
-                    const uint32_t a = pos[i], c = pos[ixj];
+                    const bool up = (i & kk) == 0;
+                    const unsigned long long a = tk[i], c = tk[ixj];
                     if ((a > c) == up) {
-                        pos[i] = c;
-                        pos[ixj] = a;
+                        tk[i] = c;
+                        tk[ixj] = a;
                     }
                 }
             }
             __syncthreads();
         }
     }
-    for (int i = threadIdx.x; i < n; i += kPbThreads) {
-        p.idx[size_t(u) * p.cap + i] = int32_t(pos[i]);
-        p.aidx[size_t(u) * p.acap + i] = int32_t(pos[i]);
+    const int kept = k < nc ? k : nc;
+    for (int i = threadIdx.x; i < kept; i += kPbThreads) p.bidx[size_t(u) * p.topk + i] = int32_t(tk[i] & 0xffffffffu);
+    if (threadIdx.x == 0) p.bcount[u] = kept;
+}
+
+// selected blocks -> their keys' original positions, ascending (the support): the positions are
+// marked in a bitmap of [0, seg0) in shared memory (the blocks lie in earlier segments and the
+// permutation stays inside segments) and compacted in order; the attention's rows are the
+// support followed by the own segment's keys before the block, [seg0, t0)
+__global__ void __launch_bounds__(kPbThreads) pbs_expand_kernel(PbsParams p) {
+    pdl_enter();
+    extern __shared__ __align__(16) uint32_t bits[];
+    __shared__ int wsum[kPbThreads / 32];
+    const int u = blockIdx.x, j = u / p.Hkv, g = u - j * p.Hkv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = j * p.b, seg0 = t0 / p.S * p.S;
+    int nb = p.bcount[u];
+    nb = nb < 0 ? 0 : (nb > p.topk ? p.topk : nb);
+    const int n = nb * p.b;
+    const int nw = (seg0 + 31) / 32;
+    for (int i = tid; i < nw; i += kPbThreads) bits[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += kPbThreads) {
+        const int blk = p.bidx[size_t(u) * p.topk + i / p.b];
+        const int pos = p.perm[size_t(g) * p.T + size_t(blk) * p.b + (i % p.b)];
+        if (pos >= 0 && pos < seg0) atomicOr(&bits[pos >> 5], 1u << (pos & 31));
     }
-    for (int i = threadIdx.x; i < t0 - seg0; i += kPbThreads) p.aidx[size_t(u) * p.acap + n + i] = seg0 + i;
-    if (threadIdx.x == 0) {
-        p.count[u] = n;
-        p.acount[u] = n + (t0 - seg0);
+    __syncthreads();
+    // thread t owns words [t W, t W + W): count, exclusive scan over threads, then write in order
+    const int W = (nw + kPbThreads - 1) / kPbThreads;
+    const int w0 = min(nw, tid * W), w1 = min(nw, w0 + W);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += x;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int base = incl - cnt;
+    for (int w = 0; w < warp; ++w) base += wsum[w];
+    int total = 0;
+    for (int w = 0; w < kPbThreads / 32; ++w) total += wsum[w];
+    int32_t* out_i = p.idx + size_t(u) * p.cap;
+    int32_t* out_a = p.aidx + size_t(u) * p.acap;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t x = bits[w];
+        while (x) {
+            const int bit = __ffs(x) - 1;
+            x &= x - 1;
+            out_i[base] = w * 32 + bit;
+            out_a[base] = w * 32 + bit;
+            ++base;
+        }
+    }
+    for (int i = tid; i < t0 - seg0; i += kPbThreads) out_a[total + i] = seg0 + i;
+    if (tid == 0) {
+        p.count[u] = total;
+        p.acount[u] = total + (t0 - seg0);
     }
 }
 
 struct PbsLayout {
-    size_t rm, rl, M, L, imp, perm, kbar, qbar, scores, unit_len, hist, bidx, bcount, aidx, acount, total;
+    size_t rm, rl, M, L, imp, perm, kbar, qbar, scores, bidx, bcount, aidx, acount, total;
 };
 
 PbsLayout pbs_layout(const spa_pbs_args* a) {
@@ -429,9 +518,6 @@ PbsLayout pbs_layout(const spa_pbs_args* a) {
     l.kbar = take(size_t(a->Hkv) * nblk * kPbD * 4);
     l.qbar = take(size_t(nblk) * a->Hkv * kPbD * 4);
     l.scores = take(size_t(U) * nblk * 4);
-    l.unit_len = take(size_t(U) * 4);
-    l.hist = o;
-    o += hist0_bytes(U);
     l.bidx = take(size_t(U) * topk * 4);
     l.bcount = take(size_t(U) * 4);
     l.aidx = take(size_t(U) * (size_t(topk) * a->b + a->S) * 4);
@@ -501,7 +587,6 @@ static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, voi
     p.kbar = reinterpret_cast<float*>(b + l.kbar);
     p.qbar = reinterpret_cast<float*>(b + l.qbar);
     p.scores = reinterpret_cast<float*>(b + l.scores);
-    p.unit_len = reinterpret_cast<int32_t*>(b + l.unit_len);
     int32_t* bidx = reinterpret_cast<int32_t*>(b + l.bidx);
     int32_t* bcount = reinterpret_cast<int32_t*>(b + l.bcount);
     p.bidx = bidx;
@@ -541,17 +626,15 @@ static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, voi
     SPA_CUDA_TRY(launch_pdl(pbs_sort_kernel, dim3((a->T + a->S - 1) / a->S, a->Hkv), dim3(1024), size_t(P) * 8, st, p));
     // 3. block means, block scores, top-k blocks
     SPA_CUDA_TRY(launch_pdl(pbs_means_kernel, dim3(nblk, a->Hkv, 2), dim3(kPbD), 0, st, p));
-    SPA_CUDA_TRY(launch_pdl(pbs_scores_kernel, dim3(U), dim3(kPbThreads), 0, st, p));
-    SelectParams sp{hist0_carve(b + l.hist, U), p.scores, p.unit_len, U, nblk, a->topk, 0.f, 0, 0, bidx, bcount,
-                    topk, nullptr, status};
-    spa_status s = launch_hist0(sp, false, st);
-    if (s != SPA_OK) return s;
-    if ((s = launch_select(sp, false, st)) != SPA_OK) return s;
+    SPA_CUDA_TRY(launch_pdl(pbs_scores_kernel, dim3((nblk + kPbJ - 1) / kPbJ, a->Hkv), dim3(kPbThreads), 0, st, p));
+    int Pk = 1;
+    while (Pk < nblk) Pk <<= 1;
+    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Pk * 8)));
+    SPA_CUDA_TRY(launch_pdl(pbs_topk_kernel, dim3(U), dim3(kPbThreads), size_t(Pk) * 8, st, p, a->topk));
     // 4. rows of the attention, then the tcgen05 attention
-    int Pe = 1;
-    while (Pe < topk * a->b) Pe <<= 1;
-    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Pe * 4)));
-    SPA_CUDA_TRY(launch_pdl(pbs_expand_kernel, dim3(U), dim3(kPbThreads), size_t(Pe) * 4, st, p));
+    const size_t bitmap = size_t((a->T + 31) / 32) * 4;
+    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bitmap)));
+    SPA_CUDA_TRY(launch_pdl(pbs_expand_kernel, dim3(U), dim3(kPbThreads), bitmap, st, p));
     PrefillAttendParams pp{a->Q, a->K, a->V, p.aidx, p.acount, p.acap, a->Hq, a->Hkv, a->T, a->b, 0, a->sm_scale,
                            a->out, a->out_f32, status};
     return launch_prefill_attend(pp, U, st, events);

@@ -137,7 +137,10 @@ prefill_scores_kernel(const float* __restrict__ qhat, const int32_t* __restrict_
 constexpr int kPfThreads = 256;
 constexpr float kRescaleLog2 = 8.f;
 
-struct __align__(1024) PfShared {
+// (the operand tiles sit at multiples of 32 KB from the 1024-byte aligned start of dynamic shared
+// memory, as the 128-byte swizzle needs; the struct itself is not padded to 1024 bytes, which
+// keeps it under the 227 KB a CTA may use)
+struct PfShared {
     uint8_t q[kTileBytes];
     uint8_t k[2][kTileBytes];
     uint8_t v[2][kTileBytes];
@@ -146,7 +149,9 @@ struct __align__(1024) PfShared {
     uint64_t bar_s, bar_o;      // completion of the S MMAs / of the P V MMAs
     uint32_t tmem_base;
     uint32_t valid[4][kPfKeys / 32];   // bit c: key c of tile t (slot t % 4) is attended
+    int rows[4][kPfKeys];              // cache rows of tile t's keys (slot t % 4), -1 for none
 };
+static_assert(sizeof(PfShared) <= 227 * 1024, "prefill attention: shared memory over the per-CTA limit");
 
 
 // grid (U, G / 2): one CTA per (unit, pair of query heads); 256 threads.
@@ -190,25 +195,28 @@ prefill_attend_kernel(PrefillAttendParams p) {
         const int n = t0 + rr;                                 // the diagonal tile: the block's own keys
         return (rr < p.bq && n < p.N) ? n : -1;
     };
+    // tile t's cache rows and key mask into slot t % 4 (threads 0..127, one key each); the value
+    // comes from a register loaded earlier, so the load's latency is not waited for here
+    auto stage_rows = [&](int t, int row) {
+        if (t < n_tiles && warp < 4) {
+            sh.rows[t & 3][tid] = row;
+            const uint32_t b = __ballot_sync(0xffffffffu, row >= 0);
+            if (lane == 0) sh.valid[t & 3][warp] = b;
+        }
+    };
     // 128 rows x 16 chunks of 16 bytes; thread tid copies chunk tid % 16 of rows tid / 16 + 16 j
     auto gather = [&](const uint16_t* src, uint8_t* dst, int t) {
         const int c = tid & 15;
 #pragma unroll
         for (int j = 0; j < kPfKeys / 16; ++j) {
             const int rr = j * 16 + (tid >> 4);
-            const int row = key_row(t, rr);
+            const int row = sh.rows[t & 3][rr];
             const bool ok = row >= 0;
             cp_async16(smem_u32(dst) + tile_off(rr, c), src + (ok ? (kv0 + size_t(row)) * 128 + c * 8 : 0), ok);
         }
     };
     auto gather_k = [&](int t) {
-        if (t < n_tiles) {
-            if (warp < 4) {
-                const uint32_t b = __ballot_sync(0xffffffffu, key_row(t, warp * 32 + lane) >= 0);
-                if (lane == 0) sh.valid[t & 3][warp] = b;
-            }
-            gather(p.K, sh.k[t & 1], t);
-        }
+        if (t < n_tiles) gather(p.K, sh.k[t & 1], t);
         cp_async_commit();
     };
     auto gather_v = [&](int t) {
@@ -223,6 +231,10 @@ prefill_attend_kernel(PrefillAttendParams p) {
         const size_t qrow = size_t(blk * p.bq + (rr & 63)) * p.Hq + g * G + 2 * pair + rr / 64;
         cp_async16(smem_u32(sh.q) + tile_off(rr, c), p.Q + qrow * 128 + c * 8, true);
     }
+    // rows of tiles 0..2; tile t + 3 is staged during iteration t
+#pragma unroll
+    for (int t = 0; t < 3; ++t) stage_rows(t, tid < kPfKeys ? key_row(t, tid) : -1);
+    __syncthreads();
     gather_k(0);
     gather_k(1);
     gather_v(0);
@@ -309,6 +321,8 @@ prefill_attend_kernel(PrefillAttendParams p) {
             if (tid == 0) issue_s(t + 1);
             pend_s = true;
         }
+        // rows of tile t + 3: the load is issued now and stored before the next barrier
+        const int row_pf = (tid < kPfKeys && t + 3 < n_tiles) ? key_row(t + 3, tid) : -1;
 
         // this thread's 64 logits of S(t)
         float s[64];
@@ -398,6 +412,7 @@ prefill_attend_kernel(PrefillAttendParams p) {
         } else {
             cp_async_commit();
         }
+        stage_rows(t + 3, row_pf);                             // slot of tile t - 1, no longer read
         cp_async_wait_group<2>();                              // V(t) has landed
         fence_async_smem();
         tc_fence_before();

@@ -99,7 +99,8 @@ __device__ __forceinline__ void block_exscan(uint32_t a, TB b, uint32_t& ea, TB&
 
 // ============================================================================ level-0 histogram
 // One work item = (unit, chunk of 4096 scores); shared-memory bins flushed with integer
-// atomics into the unit's histogram.
+// atomics into the unit's histogram.  When rows are 16-byte aligned (M a multiple of 4) every
+// thread issues its four float4 loads at once; the bins are cleared and scanned four at a time.
 constexpr int kH0Threads = 256;
 constexpr int kH0Chunk = 4096;
 
@@ -107,40 +108,63 @@ template <bool MASS>
 __global__ void __launch_bounds__(kH0Threads)
 hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
     pdl_enter();
-    __shared__ uint32_t h_cnt[kBins];
-    __shared__ u64 h_mass[MASS ? kBins : 1];
+    __shared__ __align__(16) uint32_t h_cnt[kBins];
+    __shared__ __align__(16) u64 h_mass[MASS ? kBins : 2];
     __shared__ uint32_t h_max;
+    const bool vec = (p.M & 3) == 0 && (reinterpret_cast<uintptr_t>(p.scores) & 15) == 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int u = item / chunks_per_unit;
         const int chunk = item - u * chunks_per_unit;
         const int L = p.unit_len ? min(max(p.unit_len[u], 0), p.M) : p.M;
         const int n0 = chunk * kH0Chunk, n1 = min(L, n0 + kH0Chunk);
         if (n0 >= n1 || (p.local && p.local[u])) continue;   // local units are not selected from
-        for (int i = threadIdx.x; i < kBins; i += kH0Threads) {
-            h_cnt[i] = 0;
-            if (MASS) h_mass[i] = 0;
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < kBins / 4; i += kH0Threads) {
+            reinterpret_cast<uint4*>(h_cnt)[i] = z4;
+            if (MASS) {
+                reinterpret_cast<uint4*>(h_mass)[2 * i] = z4;
+                reinterpret_cast<uint4*>(h_mass)[2 * i + 1] = z4;
+            }
         }
         if (threadIdx.x == 0) h_max = 0;
         __syncthreads();
         uint32_t my_max = 0;
         const float* row = p.scores + size_t(u) * p.M;
-        for (int n = n0 + threadIdx.x; n < n1; n += kH0Threads) {
-            const float s = __ldg(row + n);
+        auto add = [&](float s) {
             const uint32_t key = score_key(s);
             const uint32_t bin = key >> 21;
             my_max = max(my_max, key);
             atomicAdd(&h_cnt[bin], 1u);
             if (MASS) atomicAdd(&h_mass[bin], fixed_mass(s, bin_top_score(bin)));
+        };
+        if (vec && n1 - n0 == kH0Chunk) {
+            const float4* r4 = reinterpret_cast<const float4*>(row + n0);
+            float4 v[kH0Chunk / 4 / kH0Threads];
+#pragma unroll
+            for (int j = 0; j < kH0Chunk / 4 / kH0Threads; ++j) v[j] = __ldg(r4 + threadIdx.x + j * kH0Threads);
+#pragma unroll
+            for (int j = 0; j < kH0Chunk / 4 / kH0Threads; ++j) {
+                add(v[j].x);
+                add(v[j].y);
+                add(v[j].z);
+                add(v[j].w);
+            }
+        } else {
+            for (int n = n0 + threadIdx.x; n < n1; n += kH0Threads) add(__ldg(row + n));
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, off));
         if ((threadIdx.x & 31) == 0) atomicMax(&h_max, my_max);
         __syncthreads();
-        for (int i = threadIdx.x; i < kBins; i += kH0Threads) {
-            const uint32_t c = h_cnt[i];
-            if (c) {
-                atomicAdd(p.hist.cnt + size_t(u) * kBins + i, c);
-                if (MASS) atomicAdd(p.hist.mass + size_t(u) * kBins + i, h_mass[i]);
+        for (int i4 = threadIdx.x; i4 < kBins / 4; i4 += kH0Threads) {   // four bins at a time
+            const uint4 c4 = reinterpret_cast<const uint4*>(h_cnt)[i4];
+            if ((c4.x | c4.y | c4.z | c4.w) == 0) continue;
+            const uint32_t c[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (!c[j]) continue;
+                atomicAdd(p.hist.cnt + size_t(u) * kBins + 4 * i4 + j, c[j]);
+                if (MASS) atomicAdd(p.hist.mass + size_t(u) * kBins + 4 * i4 + j, h_mass[4 * i4 + j]);
             }
         }
         if (threadIdx.x == 0) atomicMax(p.hist.max_key + u, h_max);
