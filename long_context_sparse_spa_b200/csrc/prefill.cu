@@ -254,25 +254,31 @@ prefill_attend_kernel(PrefillAttendParams p) {
     constexpr uint32_t kIdS = idesc_bf16(kPfRows, kPfKeys, false);
     constexpr uint32_t kIdO = idesc_bf16(kPfRows, 128, true);
 
+    // Operand descriptors, built once: a k-step moves the start address, the descriptor's low 14
+    // bits (address / 16, below 2^14 for any shared-memory address), so it is one 64-bit add.
+    const uint64_t d_q = sw128_desc(smem_u32(sh.q), 16, 1024);
+    const uint64_t d_k0 = sw128_desc(smem_u32(sh.k[0]), 16, 1024), d_k1 = sw128_desc(smem_u32(sh.k[1]), 16, 1024);
+    const uint64_t d_v0 = sw128_desc(smem_u32(sh.v[0]), kSlab, 1024), d_v1 = sw128_desc(smem_u32(sh.v[1]), kSlab, 1024);
+    const uint64_t d_ph = sw128_desc(smem_u32(sh.p_hi), 16, 1024), d_pl = sw128_desc(smem_u32(sh.p_lo), 16, 1024);
     auto issue_s = [&](int t) {                                // S(t) = Q K(t)^T into S buffer t % 2
         const uint32_t d = tmem + uint32_t(t & 1) * 128;
+        const uint64_t dk = (t & 1) ? d_k1 : d_k0;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
-            umma_bf16(d, sw128_desc(smem_u32(sh.q) + off, 16, 1024), sw128_desc(smem_u32(sh.k[t & 1]) + off, 16, 1024),
-                      kIdS, kk > 0);
+            const uint64_t off = uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4);
+            umma_bf16(d, d_q + off, dk + off, kIdS, kk > 0);
         }
         umma_commit(&sh.bar_s);
     };
     auto issue_pv = [&](int t) {                               // O_a += P[:, 0:64] V(t)[0:64], O_b += the rest
-        const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo), vb = smem_u32(sh.v[t & 1]);
+        const uint64_t dv = (t & 1) ? d_v1 : d_v0;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint32_t d = t_oa + uint32_t(kk >> 2) * 128;
-            const uint32_t aoff = uint32_t((kk >> 2) * kSlab + (kk & 3) * 32);
-            const uint64_t bv = sw128_desc(vb + kk * 2048, kSlab, 1024);
-            umma_bf16(d, sw128_desc(ph + aoff, 16, 1024), bv, kIdO, (t > 0 || (kk & 3) > 0) ? 1u : 0u);
-            umma_bf16(d, sw128_desc(pl + aoff, 16, 1024), bv, kIdO, 1u);
+            const uint64_t aoff = uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4);
+            const uint64_t bv = dv + uint64_t((kk * 2048) >> 4);
+            umma_bf16(d, d_ph + aoff, bv, kIdO, (t > 0 || (kk & 3) > 0) ? 1u : 0u);
+            umma_bf16(d, d_pl + aoff, bv, kIdO, 1u);
         }
         umma_commit(&sh.bar_o);
     };
@@ -324,7 +330,7 @@ prefill_attend_kernel(PrefillAttendParams p) {
         // rows of tile t + 3: the load is issued now and stored before the next barrier
         const int row_pf = (tid < kPfKeys && t + 3 < n_tiles) ? key_row(t + 3, tid) : -1;
 
-        // this thread's 64 logits of S(t)
+        // this thread's 64 logits of S(t) -> the tile's maximum
         float s[64];
         {
             float v[32];
@@ -361,24 +367,6 @@ prefill_attend_kernel(PrefillAttendParams p) {
             m_run = tmax;
             l_run *= alpha;
         }
-        // P = 2^(sl2 s - m) as bf16 hi + lo pairs (masked keys give 2^-inf = 0; while no key has
-        // been seen m is -inf and every logit is -inf, so the reference 0 gives P = 0)
-        const float mu = m_run == -INFINITY ? 0.f : m_run;
-        uint32_t hw[32], lw[32];
-        float add4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const float p0 = ex2_approx(fmaf(s[2 * j], sl2, -mu));
-            const float p1 = ex2_approx(fmaf(s[2 * j + 1], sl2, -mu));
-            add4[(2 * j) & 3] += p0;
-            add4[(2 * j + 1) & 3] += p1;
-            const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-            const float2 hf = __bfloat1622float2(h);
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-            hw[j] = *reinterpret_cast<const uint32_t*>(&h);
-            lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
-        }
-        l_run += (add4[0] + add4[1]) + (add4[2] + add4[3]);
 
         // P(t-1) V(t-1) is complete: P, O and its V buffer are free
         ok = t == 0 || wait_bar(&sh.bar_o, ph_o);
@@ -399,15 +387,35 @@ prefill_attend_kernel(PrefillAttendParams p) {
                 }
                 tmem_wait_st();
             }
+            // P = 2^(sl2 s - m) as bf16 hi + lo, stored 8 keys at a time (masked keys give
+            // 2^-inf = 0; while no key has been seen m is -inf and every logit is -inf, so the
+            // reference 0 gives P = 0)
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
             const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
+            float add4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = c8 * 8 + 2 * j;
+                    const float p0 = ex2_approx(fmaf(s[i], sl2, -mu));
+                    const float p1 = ex2_approx(fmaf(s[i + 1], sl2, -mu));
+                    add4[(2 * j) & 3] += p0;
+                    add4[(2 * j + 1) & 3] += p1;
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    const float2 hf = __bfloat1622float2(h);
+                    const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                    hw[j] = *reinterpret_cast<const uint32_t*>(&h);
+                    lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
+                }
                 const uint32_t off = tile_off(r, half * 8 + c8);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[4 * c8]),
-                             "r"(hw[4 * c8 + 1]), "r"(hw[4 * c8 + 2]), "r"(hw[4 * c8 + 3]));
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[4 * c8]),
-                             "r"(lw[4 * c8 + 1]), "r"(lw[4 * c8 + 2]), "r"(lw[4 * c8 + 3]));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[0]), "r"(hw[1]),
+                             "r"(hw[2]), "r"(hw[3]));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[0]), "r"(lw[1]),
+                             "r"(lw[2]), "r"(lw[3]));
             }
+            l_run += (add4[0] + add4[1]) + (add4[2] + add4[3]);
             gather_v(t + 1);
         } else {
             cp_async_commit();
