@@ -93,8 +93,12 @@ inline Hist0 hist0_carve(void* base, int U) {
 __device__ __forceinline__ float bin_top_score(uint32_t b) {
     return b >= 2047u ? 3.402823466e38f : key_score(((b + 1u) << 21) - 1u);
 }
+// round(2^40 e^(s - ref)) for s <= ref, with the MUFU exponential (about 2^-22 relative; the
+// level-0 and in-bin masses of every kernel use this one function, so they agree exactly)
 __device__ __forceinline__ unsigned long long fixed_mass(float s, float ref) {
-    return __float2ull_rn(expf(s - ref) * kMassScale);
+    float e;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"((s - ref) * 1.4426950408889634f));
+    return __float2ull_rn(e * kMassScale);
 }
 
 // ------------------------------------------------------------------ level-0 crossing bin

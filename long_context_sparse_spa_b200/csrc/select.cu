@@ -701,9 +701,10 @@ int max_active_clusters(int C, size_t smem) {
 // waves of CTAs that each scan M / C scores plus a fixed cost (level-0 resolution, barriers,
 // histogram merges) worth about kSelFixed scores; a chunk too long for shared memory streams
 // from L2 on every level (kSelStreamCost per score).  The cheapest estimate wins, ties to the
-// larger cluster; C > 1 needs at least 2048 scores per CTA.  When every unit's cluster fits in
-// one wave this is the largest such C, as before.
-constexpr double kSelFixed = 4096.0;
+// larger cluster; C > 1 needs at least 2048 scores per CTA.  kSelFixed was fitted on B200 to the
+// selection of 512 units of about 30K scores timed with clusters of 2, 4 and 8 (90, 136 and 230
+// us); when every unit's cluster fits in one wave the choice is the largest C.
+constexpr double kSelFixed = 40960.0;
 constexpr double kSelStreamCost = 3.0;
 template <bool TOPP>
 SelectConfig choose(int U, int M) {
