@@ -14,7 +14,7 @@ __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w <<
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // ============================================================================ low-rank
-// One work item = (kv unit, chunk of kLrChunk rows).  Two lanes share a 32-byte index-key
+// One work item = (kv unit, chunk of at most kLrChunk rows).  Two lanes share a 32-byte index-key
 // row: each loads one 16-byte half (8 bf16) and the halves are joined with one
 // warp shuffle.  Each thread keeps kLrUnroll rows of loads in flight.
 // With HIST (one score per row, GROUP_MEAN), the CTA also histograms its scores into the
@@ -27,8 +27,8 @@ constexpr int kLrChunk = 2048;
 template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
 lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict__ kidx, int Hq, int Hkv,
-                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int n_items, Hist0 hist,
-                      const uint8_t* __restrict__ local, int kv_shared) {
+                      int M, float scale, float* __restrict__ scores, int chunks_per_unit, int chunk_rows, int n_items,
+                      Hist0 hist, const uint8_t* __restrict__ local, int kv_shared) {
     pdl_enter();
     const int G = Hq / Hkv;
     const int half = threadIdx.x & 1;          // which 8 of the 16 index dims this lane holds
@@ -88,8 +88,8 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
             }
         }
 
-        const int n0 = chunk * kLrChunk;
-        const int n1 = min(M, n0 + kLrChunk);
+        const int n0 = chunk * chunk_rows;
+        const int n1 = min(M, n0 + chunk_rows);
         // kv_shared: one key set [Hkv][M] serves every batch row (per-query prefill)
         const uint4* krow = kidx + size_t(kv_shared ? g : kvu) * M * 2 + half;
         float* out_base = NQ == 1 ? scores + size_t(kvu) * M : scores + (size_t(b) * Hq + size_t(g) * G) * M;
@@ -453,30 +453,60 @@ int grid_for(int items, int per_sm) {
     return items < cap ? (items > 0 ? items : 1) : cap;
 }
 
+// Rows per work item of the low-rank scorer, at most kLrChunk.  A grid with fewer items than SMs
+// (a short cache: 4K tokens make two 2048-row items per unit) is split into more, shorter items,
+// about one wave of the CTAs the SMs hold at once, each of at least min_rows rows (a histogram item
+// clears and flushes 2048 bins).  Larger grids keep 2048-row items: splitting them further was
+// measured slower (more clears and flushes, for a partial last wave that the next kernel's launch
+// overlaps anyway).
+template <typename Kern>
+int lr_chunk_rows(Kern kern, int units, int M, int min_rows) {
+    const int base = (M + kLrChunk - 1) / kLrChunk;
+    const int sms = device_info().num_sms;
+    if ((long long)units * base >= sms) return kLrChunk;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLrThreads, 0) != cudaSuccess || per_sm <= 0) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    const long long resident = (long long)per_sm * sms;
+    const long long per_unit = (resident + units - 1) / units;   // chunks per unit for about one wave
+    int rows = int((M + per_unit - 1) / per_unit);
+    rows = (rows + 15) / 16 * 16;
+    rows = rows < min_rows ? min_rows : rows;
+    return rows > kLrChunk ? kLrChunk : rows;
+}
+
 }  // namespace
 
 spa_status launch_lowrank_scores(const uint16_t* qidx, const uint16_t* kidx, int B, int Hq, int Hkv, int M,
                                  int collapse, float scale, float* scores, const Hist0* hist, bool with_mass,
                                  cudaStream_t st, const uint8_t* local, bool kv_shared) {
     const int G = Hq / Hkv;
-    const int chunks = (M + kLrChunk - 1) / kLrChunk;
-    const int items = B * Hkv * chunks;
-    const int grid = grid_for(items, 8);
+    const int units = B * Hkv;
     const uint4* k4 = reinterpret_cast<const uint4*>(kidx);
     const Hist0 h = hist ? *hist : Hist0{nullptr, nullptr, nullptr};
     if (collapse == SPA_COLLAPSE_GROUP_MEAN) {
         auto kern = hist && with_mass ? lowrank_scores_kernel<1, true, true>
                                       : (hist ? lowrank_scores_kernel<1, true, false> : lowrank_scores_kernel<1, false, false>);
-        SPA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kLrThreads), 0, st, qidx, k4, Hq, Hkv, M, scale, scores, chunks,
-                                items, h, local, kv_shared ? 1 : 0));
+        const int rows = lr_chunk_rows(kern, units, M, hist ? 1024 : 256);
+        const int chunks = (M + rows - 1) / rows;
+        const int items = units * chunks;
+        SPA_CUDA_TRY(launch_pdl(kern, dim3(grid_for(items, 32)), dim3(kLrThreads), 0, st, qidx, k4, Hq, Hkv, M, scale,
+                                scores, chunks, rows, items, h, local, kv_shared ? 1 : 0));
     } else {
         if (hist) return SPA_ERR_INVALID_ARG;
         switch (G) {
 #define SPA_LR_CASE(n)                                                                                          \
-    case n:                                                                                                     \
-        SPA_CUDA_TRY(launch_pdl(lowrank_scores_kernel<n, false, false>, dim3(grid), dim3(kLrThreads), 0, st, qidx, \
-                                k4, Hq, Hkv, M, scale, scores, chunks, items, h, nullptr, kv_shared ? 1 : 0));  \
-        break;
+    case n: {                                                                                                   \
+        const int rows = lr_chunk_rows(lowrank_scores_kernel<n, false, false>, units, M, 256);                 \
+        const int chunks = (M + rows - 1) / rows;                                                              \
+        const int items = units * chunks;                                                                      \
+        SPA_CUDA_TRY(launch_pdl(lowrank_scores_kernel<n, false, false>, dim3(grid_for(items, 32)), dim3(kLrThreads), \
+                                0, st, qidx, k4, Hq, Hkv, M, scale, scores, chunks, rows, items, h, nullptr,     \
+                                kv_shared ? 1 : 0));                                                           \
+        break;                                                                                                 \
+    }
             SPA_LR_CASE(1) SPA_LR_CASE(2) SPA_LR_CASE(4) SPA_LR_CASE(8) SPA_LR_CASE(16)
 #undef SPA_LR_CASE
             default: return SPA_ERR_UNSUPPORTED_SHAPE;
