@@ -100,7 +100,8 @@ def test_pbs_small_all_units():
     check(PBS_SMALL)
 
 
-@pytest.mark.parametrize("over", [dict(topk=0), dict(topk=40), dict(S=64, topk=3), dict(S=192, Hq=16, Hkv=2)],
-                         ids=["no_blocks", "all_blocks", "segment_eq_2_blocks", "ragged_last_segment_G8"])
+@pytest.mark.parametrize("over", [dict(topk=0), dict(topk=40), dict(S=64, topk=3), dict(S=192, Hq=16, Hkv=2),
+                                  dict(Hq=4, Hkv=2), dict(Hq=12, Hkv=2, T=768)],
+                         ids=["no_blocks", "all_blocks", "segment_eq_2_blocks", "ragged_last_segment_G8", "G2", "G6"])
 def test_pbs_variants(over):
     check(PBS_SMALL.with_(**over))

@@ -64,6 +64,13 @@ def test_prefill_small_all_units():
     check_units(cfg, [(j, g) for j in range(cfg.n_blocks) for g in range(cfg.Hkv)])
 
 
+@pytest.mark.parametrize("over", [dict(Hq=4, Hkv=2), dict(Hq=16, Hkv=2)], ids=["G2", "G8"])
+def test_prefill_head_groups(over):
+    # one and four pairs of query heads per unit (one CTA per pair)
+    cfg = SMALL["c5s"].with_(N=2048, q_start=1536, T=256, topk=256, n_clusters=8, **over)
+    check_units(cfg, [(j, g) for j in range(cfg.n_blocks) for g in range(cfg.Hkv)])
+
+
 def test_prefill_budget_covers_everything():
     # top-k larger than every candidate set: supports are all of [0, t0); dense causal attention
     cfg = SMALL["c5s"].with_(N=2048, q_start=1024, T=512, topk=4096, n_clusters=8)
