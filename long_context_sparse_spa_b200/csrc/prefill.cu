@@ -134,7 +134,8 @@ prefill_scores_kernel(const float* __restrict__ qhat, const int32_t* __restrict_
 //     Every thread commits one cp.async group per gather point, empty or not, so the group
 //     counts of the waits are the same in every iteration.
 // TMEM columns: S buffers 0..127 and 128..255, O_a 256..383, O_b 384..511.
-constexpr int kPfThreads = 256;
+constexpr int kPfSoft = 256;               // warps 0-7: gathers and softmax
+constexpr int kPfThreads = kPfSoft + 32;   // + warp 8, whose lane 0 issues the MMAs
 constexpr float kRescaleLog2 = 8.f;
 
 // (the operand tiles sit at multiples of 32 KB from the 1024-byte aligned start of dynamic shared
@@ -146,21 +147,45 @@ struct PfShared {
     uint8_t v[2][kTileBytes];
     uint8_t p_hi[kTileBytes];   // the epilogue reuses it for the halves' (m, l)
     uint8_t p_lo[kTileBytes];
-    uint64_t bar_s, bar_o;      // completion of the S MMAs / of the P V MMAs
+    uint64_t bar_s, bar_o;      // completion of the S MMAs / of the P V MMAs (tcgen05.commit)
+    uint64_t k_ready;           // the 256 softmax threads: the next tile's keys are in place (and S read)
+    uint64_t p_ready;           // the 256 softmax threads: P(t) stored and V(t) in place
     uint32_t tmem_base;
+    uint32_t n_s, n_o;          // commits the issuer made on bar_s / bar_o
     uint32_t valid[4][kPfKeys / 32];   // bit c: key c of tile t (slot t % 4) is attended
     int rows[4][kPfKeys];              // cache rows of tile t's keys (slot t % 4), -1 for none
 };
 static_assert(sizeof(PfShared) <= 227 * 1024, "prefill attention: shared memory over the per-CTA limit");
 
+// named barrier 1 of the 256 softmax threads (the issuing warp never joins it)
+__device__ __forceinline__ void soft_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+// the same barrier, returning the OR of v over the 256 threads
+__device__ __forceinline__ bool soft_sync_or(bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 256, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+                 : "=r"(r)
+                 : "r"(uint32_t(v))
+                 : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
 
-// grid (U, G / 2): one CTA per (unit, pair of query heads); 256 threads.
+// grid (U, G / 2): one CTA per (unit, pair of query heads); 288 threads.  Warps 0-7 gather and run
+// the softmax; lane 0 of warp 8 issues every MMA.  The two sides meet only at mbarriers: the
+// softmax warps arrive on k_ready once the next tile's keys have landed (and the S buffer they
+// overwrite was read) and on p_ready once P(t) is stored and V(t) has landed; the issuer waits
+// on those and the softmax warps on the MMAs' commits.  So an MMA issue that waits for room in the
+// tensor core's queue delays no softmax warp, and the softmax warps share one named barrier per
+// tile (row staging, and the decision to stop after a bounded wait gave up).
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_attend_kernel(PrefillAttendParams p) {
     pdl_enter();
     extern __shared__ __align__(1024) uint8_t dyn[];
     PfShared& sh = *reinterpret_cast<PfShared*>(dyn);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool issuer_warp = warp == kPfSoft / 32;
     const int u = blockIdx.x, pair = blockIdx.y;
     const int blk = u / p.Hkv, g = u - blk * p.Hkv;
     const int G = p.Hq / p.Hkv;
@@ -173,7 +198,7 @@ prefill_attend_kernel(PrefillAttendParams p) {
     const size_t kv0 = size_t(g) * p.N;
 
     // softmax role: query row r (TMEM lane) and key-column half
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const int r = quad * 32 + lane, qi = r & 63;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
@@ -181,6 +206,10 @@ prefill_attend_kernel(PrefillAttendParams p) {
     if (tid == 0) {
         mbar_init(&sh.bar_s, 1);
         mbar_init(&sh.bar_o, 1);
+        mbar_init(&sh.k_ready, kPfSoft);
+        mbar_init(&sh.p_ready, kPfSoft);
+        sh.n_s = 0;
+        sh.n_o = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
 
@@ -204,7 +233,7 @@ prefill_attend_kernel(PrefillAttendParams p) {
             if (lane == 0) sh.valid[t & 3][warp] = b;
         }
     };
-    // 128 rows x 16 chunks of 16 bytes; thread tid copies chunk tid % 16 of rows tid / 16 + 16 j
+    // 128 rows x 16 chunks of 16 bytes; softmax thread tid copies chunk tid % 16 of rows tid / 16 + 16 j
     auto gather = [&](const uint16_t* src, uint8_t* dst, int t) {
         const int c = tid & 15;
 #pragma unroll
@@ -224,67 +253,21 @@ prefill_attend_kernel(PrefillAttendParams p) {
         cp_async_commit();
     };
 
-    // Q tile (row rr: head 2 pair + rr / 64, query rr % 64 of the block), in K(0)'s group
-#pragma unroll
-    for (int j = 0; j < kPfRows / 16; ++j) {
-        const int rr = j * 16 + (tid >> 4), c = tid & 15;
-        const size_t qrow = size_t(blk * p.bq + (rr & 63)) * p.Hq + g * G + 2 * pair + rr / 64;
-        cp_async16(smem_u32(sh.q) + tile_off(rr, c), p.Q + qrow * 128 + c * 8, true);
-    }
-    // rows of tiles 0..2; tile t + 3 is staged during iteration t
-#pragma unroll
-    for (int t = 0; t < 3; ++t) stage_rows(t, tid < kPfKeys ? key_row(t, tid) : -1);
-    __syncthreads();
-    gather_k(0);
-    gather_k(1);
-    gather_v(0);
-    cp_async_wait_group<2>();                                  // Q and K(0)
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sh.tmem_base;
-    const uint32_t t_oa = tmem + 256;
-
     // the test hook stalls the first S = Q K^T: its completion barrier waits for an MMA that
-    // is never issued, so the bounded wait runs out with nothing in flight
+    // is never issued, so the bounded waits run out with nothing in flight
     const bool stall = (p.test_stall & SPA_TEST_STALL_PREFILL_MMA) != 0;
     const uint32_t spin_limit = stall ? 1024u : kSpinLimit;
     const float sl2 = p.sm_scale * kLog2e;
     constexpr uint32_t kIdS = idesc_bf16(kPfRows, kPfKeys, false);
     constexpr uint32_t kIdO = idesc_bf16(kPfRows, 128, true);
 
-    // Operand descriptors, built once: a k-step moves the start address, the descriptor's low 14
-    // bits (address / 16, below 2^14 for any shared-memory address), so it is one 64-bit add.
-    const uint64_t d_q = sw128_desc(smem_u32(sh.q), 16, 1024);
-    const uint64_t d_k0 = sw128_desc(smem_u32(sh.k[0]), 16, 1024), d_k1 = sw128_desc(smem_u32(sh.k[1]), 16, 1024);
-    const uint64_t d_v0 = sw128_desc(smem_u32(sh.v[0]), kSlab, 1024), d_v1 = sw128_desc(smem_u32(sh.v[1]), kSlab, 1024);
-    const uint64_t d_ph = sw128_desc(smem_u32(sh.p_hi), 16, 1024), d_pl = sw128_desc(smem_u32(sh.p_lo), 16, 1024);
-    auto issue_s = [&](int t) {                                // S(t) = Q K(t)^T into S buffer t % 2
-        const uint32_t d = tmem + uint32_t(t & 1) * 128;
-        const uint64_t dk = (t & 1) ? d_k1 : d_k0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t off = uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4);
-            umma_bf16(d, d_q + off, dk + off, kIdS, kk > 0);
-        }
-        umma_commit(&sh.bar_s);
-    };
-    auto issue_pv = [&](int t) {                               // O_a += P[:, 0:64] V(t)[0:64], O_b += the rest
-        const uint64_t dv = (t & 1) ? d_v1 : d_v0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t d = t_oa + uint32_t(kk >> 2) * 128;
-            const uint64_t aoff = uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4);
-            const uint64_t bv = dv + uint64_t((kk * 2048) >> 4);
-            umma_bf16(d, d_ph + aoff, bv, kIdO, (t > 0 || (kk & 3) > 0) ? 1u : 0u);
-            umma_bf16(d, d_pl + aoff, bv, kIdO, 1u);
-        }
-        umma_commit(&sh.bar_o);
-    };
-    // bounded wait on a completion barrier; on expiry this thread's flag is set, the CTA stops at
-    // its next barrier (each barrier ORs the flags of all threads, so every thread takes the same
-    // decision there) and the commit stays owed
+    tc_fence_before();
+    __syncthreads();                                           // barriers initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const uint32_t t_oa = tmem + 256;
+
+    // bounded wait on a barrier phase; on expiry this thread's flag is set
     bool my_to = false;
     auto wait_bar = [&](uint64_t* bar, uint32_t& ph) -> bool {
         uint32_t it = 0;
@@ -299,151 +282,214 @@ prefill_attend_kernel(PrefillAttendParams p) {
         return true;
     };
 
-    bool pend_s = false, pend_o = false;   // a commit issued and not yet observed (uniform over the CTA)
+    uint32_t seen_s = 0, seen_o = 0;       // completions of bar_s / bar_o this thread observed
     uint32_t ph_s = 0, ph_o = 0;
-    if (!stall) {
-        if (tid == 0) issue_s(0);
-        pend_s = true;
-    }
     float m_run = -INFINITY, l_run = 0.f;
-    const uint32_t t_my_o = t_oa + uint32_t(half) * 128 + lane_off;
-    bool stopped = false;                  // a wait gave up (uniform over the CTA)
 
-    for (int t = 0; t < n_tiles; ++t) {
-        // S(t) is complete: its K buffer takes tile t + 2 (ok is made warp-uniform: the gather
-        // holds a warp vote)
-        bool ok = wait_bar(&sh.bar_s, ph_s);
-        if (ok) pend_s = false;
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) gather_k(t + 2);
-        else cp_async_commit();
-        cp_async_wait_group<2>();                              // K(t + 1) (and V(t)) have landed
-        fence_async_smem();
-        tc_fence_before();
-        stopped = __syncthreads_or(my_to) != 0;
-        tc_fence_after();
-        if (stopped) break;
-        if (t + 1 < n_tiles) {
-            if (tid == 0) issue_s(t + 1);
-            pend_s = true;
-        }
-        // rows of tile t + 3: the load is issued now and stored before the next barrier
-        const int row_pf = (tid < kPfKeys && t + 3 < n_tiles) ? key_row(t + 3, tid) : -1;
-
-        // this thread's 64 logits of S(t) -> the tile's maximum
-        float s[64];
-        {
-            float v[32];
-            const uint32_t ta = tmem + uint32_t(t & 1) * 128 + uint32_t(half) * 64 + lane_off;
-            tmem_ld32(ta, v);
+    if (issuer_warp) {
+        if (lane == 0) {
+            // Operand descriptors, built once: a k-step moves the start address, the descriptor's
+            // low 14 bits (address / 16, below 2^14 for any shared-memory address), one 64-bit add.
+            const uint64_t d_q = sw128_desc(smem_u32(sh.q), 16, 1024);
+            const uint64_t d_k0 = sw128_desc(smem_u32(sh.k[0]), 16, 1024), d_k1 = sw128_desc(smem_u32(sh.k[1]), 16, 1024);
+            const uint64_t d_v0 = sw128_desc(smem_u32(sh.v[0]), kSlab, 1024);
+            const uint64_t d_v1 = sw128_desc(smem_u32(sh.v[1]), kSlab, 1024);
+            const uint64_t d_ph = sw128_desc(smem_u32(sh.p_hi), 16, 1024), d_pl = sw128_desc(smem_u32(sh.p_lo), 16, 1024);
+            auto issue_s = [&](int t) {                        // S(t) = Q K(t)^T into S buffer t % 2
+                const uint32_t d = tmem + uint32_t(t & 1) * 128;
+                const uint64_t dk = (t & 1) ? d_k1 : d_k0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s[i] = v[i];
-            tmem_ld32(ta + 32, v);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t off = uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4);
+                    umma_bf16(d, d_q + off, dk + off, kIdS, kk > 0);
+                }
+                umma_commit(&sh.bar_s);
+            };
+            auto issue_pv = [&](int t) {                       // O_a += P[:, 0:64] V(t)[0:64], O_b += the rest
+                const uint64_t dv = (t & 1) ? d_v1 : d_v0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s[32 + i] = v[i];
-        }
-        tc_fence_before();
-        // raw logits; masked keys become -inf.  A full tile of support keys (every tile but the
-        // last partial one and the diagonal) needs no mask: the test is warp-uniform
-        const uint32_t vm0 = sh.valid[t & 3][2 * half], vm1 = sh.valid[t & 3][2 * half + 1];
-        if (!(t < n_gather && (vm0 & vm1) == 0xffffffffu)) {
-            const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const bool valid = (((i < 32 ? vm0 : vm1) >> (i & 31)) & 1u) && i <= causal;
-                s[i] = valid ? s[i] : -INFINITY;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t d = t_oa + uint32_t(kk >> 2) * 128;
+                    const uint64_t aoff = uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4);
+                    const uint64_t bv = dv + uint64_t((kk * 2048) >> 4);
+                    umma_bf16(d, d_ph + aoff, bv, kIdO, (t > 0 || (kk & 3) > 0) ? 1u : 0u);
+                    umma_bf16(d, d_pl + aoff, bv, kIdO, 1u);
+                }
+                umma_commit(&sh.bar_o);
+            };
+            // S(t + 1) is issued before P(t) V(t): the softmax of tile t + 1 needs it first
+            uint32_t pk = 0, pp = 0;
+            bool live = wait_bar(&sh.k_ready, pk);             // Q and tile 0's keys
+            if (live && !stall) {
+                issue_s(0);
+                sh.n_s = 1;
+            }
+            for (int t = 0; live && t < n_tiles; ++t) {
+                if (t + 1 < n_tiles) {
+                    if (!wait_bar(&sh.k_ready, pk)) break;
+                    issue_s(t + 1);
+                    sh.n_s = uint32_t(t + 2);
+                }
+                if (!wait_bar(&sh.p_ready, pp)) break;
+                issue_pv(t);
+                sh.n_o = uint32_t(t + 1);
             }
         }
-        // tile maximum in four independent chains, then in log2 units (sm_scale > 0)
-        float mx4[4] = {s[0], s[1], s[2], s[3]};
+    } else {
+        // Q tile (row rr: head 2 pair + rr / 64, query rr % 64 of the block), in K(0)'s group
 #pragma unroll
-        for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
-        const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
-        bool rescale = false;
-        float alpha = 1.f;
-        if (tmax > m_run + kRescaleLog2) {                    // also the first finite maximum
-            alpha = ex2_approx(m_run - tmax);
-            rescale = m_run != -INFINITY;                      // O of this half holds nonzero terms
-            m_run = tmax;
-            l_run *= alpha;
+        for (int j = 0; j < kPfRows / 16; ++j) {
+            const int rr = j * 16 + (tid >> 4), c = tid & 15;
+            const size_t qrow = size_t(blk * p.bq + (rr & 63)) * p.Hq + g * G + 2 * pair + rr / 64;
+            cp_async16(smem_u32(sh.q) + tile_off(rr, c), p.Q + qrow * 128 + c * 8, true);
         }
-
-        // P(t-1) V(t-1) is complete: P, O and its V buffer are free
-        ok = t == 0 || wait_bar(&sh.bar_o, ph_o);
-        if (t > 0 && ok) pend_o = false;
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-            // tcgen05.ld / st are warp-collective: a warp rescales when any of its rows needs it,
-            // the other rows by 1
-            if (__any_sync(0xffffffffu, rescale)) {
-                const float a = rescale ? alpha : 1.f;
+        // rows of tiles 0..2; tile t + 3 is staged during iteration t
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
+        for (int t = 0; t < 3; ++t) stage_rows(t, tid < kPfKeys ? key_row(t, tid) : -1);
+        soft_sync();
+        gather_k(0);
+        gather_k(1);
+        gather_v(0);
+        cp_async_wait_group<2>();                              // Q and K(0)
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.k_ready);
+        const uint32_t t_my_o = t_oa + uint32_t(half) * 128 + lane_off;
+
+        for (int t = 0; t < n_tiles; ++t) {
+            // S(t) is complete: its K buffer takes tile t + 2 (ok is made warp-uniform: the
+            // stores below hold warp votes)
+            bool ok = !my_to && wait_bar(&sh.bar_s, ph_s);
+            if (ok) ++seen_s;
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) gather_k(t + 2);
+            else cp_async_commit();
+            cp_async_wait_group<2>();                          // K(t + 1) has landed
+            if (ok && t + 1 < n_tiles) {                       // ... for the issuer's S(t + 1)
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sh.k_ready);
+            }
+            // rows of tile t + 3: the load is issued now and stored before the next barrier
+            const int row_pf = (tid < kPfKeys && t + 3 < n_tiles) ? key_row(t + 3, tid) : -1;
+
+            bool rescale = false;
+            float alpha = 1.f;
+            float s[64];
+            if (ok) {
+                // this thread's 64 logits of S(t) -> the tile's maximum
+                {
                     float v[32];
-                    tmem_ld32(t_my_o + cb * 32, v);
+                    const uint32_t ta = tmem + uint32_t(t & 1) * 128 + uint32_t(half) * 64 + lane_off;
+                    tmem_ld32(ta, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] *= a;
-                    tmem_st32(t_my_o + cb * 32, v);
+                    for (int i = 0; i < 32; ++i) s[i] = v[i];
+                    tmem_ld32(ta + 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[32 + i] = v[i];
                 }
-                tmem_wait_st();
-            }
-            // P = 2^(sl2 s - m) as bf16 hi + lo, stored 8 keys at a time (masked keys give
-            // 2^-inf = 0; while no key has been seen m is -inf and every logit is -inf, so the
-            // reference 0 gives P = 0)
-            const float mu = m_run == -INFINITY ? 0.f : m_run;
-            const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
-            float add4[4] = {0.f, 0.f, 0.f, 0.f};
+                tc_fence_before();
+                // raw logits; masked keys become -inf.  A full tile of support keys (every tile
+                // but the last partial one and the diagonal) needs no mask: the test is warp-uniform
+                const uint32_t vm0 = sh.valid[t & 3][2 * half], vm1 = sh.valid[t & 3][2 * half + 1];
+                if (!(t < n_gather && (vm0 & vm1) == 0xffffffffu)) {
+                    const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int i = c8 * 8 + 2 * j;
-                    const float p0 = ex2_approx(fmaf(s[i], sl2, -mu));
-                    const float p1 = ex2_approx(fmaf(s[i + 1], sl2, -mu));
-                    add4[(2 * j) & 3] += p0;
-                    add4[(2 * j + 1) & 3] += p1;
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    const float2 hf = __bfloat1622float2(h);
-                    const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-                    hw[j] = *reinterpret_cast<const uint32_t*>(&h);
-                    lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
+                    for (int i = 0; i < 64; ++i) {
+                        const bool valid = (((i < 32 ? vm0 : vm1) >> (i & 31)) & 1u) && i <= causal;
+                        s[i] = valid ? s[i] : -INFINITY;
+                    }
                 }
-                const uint32_t off = tile_off(r, half * 8 + c8);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[0]), "r"(hw[1]),
-                             "r"(hw[2]), "r"(hw[3]));
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[0]), "r"(lw[1]),
-                             "r"(lw[2]), "r"(lw[3]));
+                // tile maximum in four independent chains, then in log2 units (sm_scale > 0)
+                float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+                for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+                const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+                if (tmax > m_run + kRescaleLog2) {             // also the first finite maximum
+                    alpha = ex2_approx(m_run - tmax);
+                    rescale = m_run != -INFINITY;               // O of this half holds nonzero terms
+                    m_run = tmax;
+                    l_run *= alpha;
+                }
             }
-            l_run += (add4[0] + add4[1]) + (add4[2] + add4[3]);
-            gather_v(t + 1);
-        } else {
-            cp_async_commit();
+
+            // P(t-1) V(t-1) is complete: P, O and its V buffer are free
+            bool ok2 = ok && (t == 0 || wait_bar(&sh.bar_o, ph_o));
+            if (ok2 && t > 0) ++seen_o;
+            ok2 = __all_sync(0xffffffffu, ok2);
+            if (ok2) {
+                // tcgen05.ld / st are warp-collective: a warp rescales when any of its rows needs
+                // it, the other rows by 1
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float a = rescale ? alpha : 1.f;
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        float v[32];
+                        tmem_ld32(t_my_o + cb * 32, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= a;
+                        tmem_st32(t_my_o + cb * 32, v);
+                    }
+                    tmem_wait_st();
+                }
+                // P = 2^(sl2 s - m) as bf16 hi + lo, stored 8 keys at a time (masked keys give
+                // 2^-inf = 0; while no key has been seen m is -inf and every logit is -inf, so the
+                // reference 0 gives P = 0)
+                const float mu = m_run == -INFINITY ? 0.f : m_run;
+                const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
+                float add4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int i = c8 * 8 + 2 * j;
+                        const float p0 = ex2_approx(fmaf(s[i], sl2, -mu));
+                        const float p1 = ex2_approx(fmaf(s[i + 1], sl2, -mu));
+                        add4[(2 * j) & 3] += p0;
+                        add4[(2 * j + 1) & 3] += p1;
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                        const float2 hf = __bfloat1622float2(h);
+                        const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                        hw[j] = *reinterpret_cast<const uint32_t*>(&h);
+                        lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
+                    }
+                    const uint32_t off = tile_off(r, half * 8 + c8);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[0]), "r"(hw[1]),
+                                 "r"(hw[2]), "r"(hw[3]));
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[0]), "r"(lw[1]),
+                                 "r"(lw[2]), "r"(lw[3]));
+                }
+                l_run += (add4[0] + add4[1]) + (add4[2] + add4[3]);
+                gather_v(t + 1);
+            } else {
+                cp_async_commit();
+            }
+            stage_rows(t + 3, row_pf);                         // slot of tile t - 1, no longer read
+            cp_async_wait_group<2>();                          // V(t) has landed
+            if (ok2) {                                         // ... for the issuer's P(t) V(t)
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sh.p_ready);
+            }
+            if (soft_sync_or(my_to)) break;                    // staged rows visible; a give-up stops all
         }
-        stage_rows(t + 3, row_pf);                             // slot of tile t - 1, no longer read
-        cp_async_wait_group<2>();                              // V(t) has landed
-        fence_async_smem();
-        tc_fence_before();
-        stopped = __syncthreads_or(my_to) != 0;
-        tc_fence_after();
-        if (stopped) break;
-        if (tid == 0) issue_pv(t);
-        pend_o = true;
+        // the last P V
+        if (!my_to && wait_bar(&sh.bar_o, ph_o)) ++seen_o;
     }
 
-    // the last P V, then no copy is left in flight
-    if (!stopped && pend_o && wait_bar(&sh.bar_o, ph_o)) pend_o = false;
+    // ---- epilogue: every thread's copies have landed; the halves' (m, l) meet in shared memory
     cp_async_wait_all();
     tc_fence_before();
     const bool good = __syncthreads_or(my_to) == 0;
     float* ex = reinterpret_cast<float*>(sh.p_hi);            // [half][m | l][row]
-    if (good) {
+    if (good && !issuer_warp) {
         ex[half * 256 + r] = m_run;
         ex[half * 256 + 128 + r] = l_run;
     }
     __syncthreads();
     tc_fence_after();
-    if (good) {
+    if (good && !issuer_warp) {
         const float ma = ex[r], la = ex[128 + r], mb = ex[256 + r], lb = ex[384 + r];
         const float m = fmaxf(ma, mb);
         float sa = 0.f, sb = 0.f;
@@ -482,30 +528,33 @@ prefill_attend_kernel(PrefillAttendParams p) {
                 }
             }
         }
-    } else if (tid == 0) {
+    } else if (!good && tid == 0) {
         raise_status(p.status, SPA_ERR_TIMEOUT);
     }
     tc_fence_before();
     __syncthreads();
-    // after a give-up, an issued MMA may still be running: wait once more (bounded); TMEM is
-    // freed only when no commit is owed (a CTA that exits holding TMEM is the remaining hazard
-    // of a wait that never completes)
-    if (pend_s) {
-        uint32_t it = 0;
-        while (!mbar_try_wait(&sh.bar_s, ph_s) && ++it < spin_limit) {
+    // commits the issuer made that warp 0 has not seen complete (at most one per barrier, as the
+    // issuer waits for the softmax warps' hand-off before each): wait once more (bounded); TMEM is
+    // freed only when nothing is owed (a CTA that exits holding TMEM is the remaining hazard of a
+    // wait that never completes)
+    if (warp == 0) {
+        bool owed = false;
+        if (sh.n_s > seen_s) {
+            uint32_t it = 0;
+            while (!mbar_try_wait(&sh.bar_s, ph_s) && ++it < spin_limit) {
+            }
+            owed = owed || it >= spin_limit;
         }
-        pend_s = it >= spin_limit;
-    }
-    if (pend_o) {
-        uint32_t it = 0;
-        while (!mbar_try_wait(&sh.bar_o, ph_o) && ++it < spin_limit) {
+        if (sh.n_o > seen_o) {
+            uint32_t it = 0;
+            while (!mbar_try_wait(&sh.bar_o, ph_o) && ++it < spin_limit) {
+            }
+            owed = owed || it >= spin_limit;
         }
-        pend_o = it >= spin_limit;
-    }
-    // (the free is warp-collective: warp 0 frees only when none of its lanes still sees a debt)
-    if (warp == 0 && !__any_sync(0xffffffffu, pend_s || pend_o)) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if (!__any_sync(0xffffffffu, owed)) {
+            tc_fence_after();
+            tmem_dealloc(tmem, 512);
+        }
     }
 }
 
