@@ -157,6 +157,20 @@ struct PfShared {
 };
 static_assert(sizeof(PfShared) <= 227 * 1024, "prefill attention: shared memory over the per-CTA limit");
 
+// paired fp32 arithmetic (one instruction for two lanes of a 64-bit register pair)
+__device__ __forceinline__ void ffma2(float& r0, float& r1, float a0, float a1, float b0, float b1, float c0, float c1) {
+    asm("{\n .reg .b64 a, b, c, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n mov.b64 c, {%6, %7};\n"
+        " fma.rn.f32x2 d, a, b, c;\n mov.b64 {%0, %1}, d;\n}\n"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n .reg .b64 a, b, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n add.f32x2 d, a, b;\n"
+        " mov.b64 {%0, %1}, d;\n}\n"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // named barrier 1 of the 256 softmax threads (the issuing warp never joins it)
 __device__ __forceinline__ void soft_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
 // the same barrier, returning the OR of v over the 256 threads
@@ -437,20 +451,23 @@ prefill_attend_kernel(PrefillAttendParams p) {
                 // reference 0 gives P = 0)
                 const float mu = m_run == -INFINITY ? 0.f : m_run;
                 const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
-                float add4[4] = {0.f, 0.f, 0.f, 0.f};
+                float add4[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of running sums
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     uint32_t hw[4], lw[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int i = c8 * 8 + 2 * j;
-                        const float p0 = ex2_approx(fmaf(s[i], sl2, -mu));
-                        const float p1 = ex2_approx(fmaf(s[i + 1], sl2, -mu));
-                        add4[(2 * j) & 3] += p0;
-                        add4[(2 * j + 1) & 3] += p1;
+                        float x0, x1;
+                        ffma2(x0, x1, s[i], s[i + 1], sl2, sl2, -mu, -mu);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        const int a = (j & 1) * 2;
+                        fadd2(add4[a], add4[a + 1], add4[a], add4[a + 1], p0, p1);
                         const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                         const float2 hf = __bfloat1622float2(h);
-                        const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                        float r0, r1;
+                        fadd2(r0, r1, p0, p1, -hf.x, -hf.y);
+                        const __nv_bfloat162 lo = __floats2bfloat162_rn(r0, r1);
                         hw[j] = *reinterpret_cast<const uint32_t*>(&h);
                         lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
                     }
