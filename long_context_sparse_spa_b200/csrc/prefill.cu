@@ -389,35 +389,36 @@ prefill_attend_kernel(PrefillAttendParams p) {
 
             bool rescale = false;
             float alpha = 1.f;
-            float s[64];
-            if (ok) {
-                // this thread's 64 logits of S(t) -> the tile's maximum
-                {
-                    float v[32];
-                    const uint32_t ta = tmem + uint32_t(t & 1) * 128 + uint32_t(half) * 64 + lane_off;
-                    tmem_ld32(ta, v);
+            // this thread's 64 logits of S(t) are read from TMEM twice, 32 at a time: for the
+            // tile's maximum now, and for P after P(t-1) V(t-1) is complete (the issuer rewrites
+            // the buffer only after this thread's next arrival on k_ready)
+            const uint32_t ta = tmem + uint32_t(t & 1) * 128 + uint32_t(half) * 64 + lane_off;
+            const uint32_t vm0 = sh.valid[t & 3][2 * half], vm1 = sh.valid[t & 3][2 * half + 1];
+            // masked keys become -inf.  A full tile of support keys (every tile but the last partial
+            // one and the diagonal) needs no mask: the test is warp-uniform
+            const bool full = t < n_gather && (vm0 & vm1) == 0xffffffffu;
+            const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
+            auto logits32 = [&](int q2, float (&v)[32]) {
+                tmem_ld32(ta + uint32_t(q2) * 32, v);
+                if (!full) {
+                    const uint32_t vm = q2 ? vm1 : vm0;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[i] = v[i];
-                    tmem_ld32(ta + 32, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[32 + i] = v[i];
-                }
-                tc_fence_before();
-                // raw logits; masked keys become -inf.  A full tile of support keys (every tile
-                // but the last partial one and the diagonal) needs no mask: the test is warp-uniform
-                const uint32_t vm0 = sh.valid[t & 3][2 * half], vm1 = sh.valid[t & 3][2 * half + 1];
-                if (!(t < n_gather && (vm0 & vm1) == 0xffffffffu)) {
-                    const int causal = t < n_gather ? kPfKeys : qi - half * 64;   // diagonal tile: key c <= qi
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const bool valid = (((i < 32 ? vm0 : vm1) >> (i & 31)) & 1u) && i <= causal;
-                        s[i] = valid ? s[i] : -INFINITY;
+                    for (int i = 0; i < 32; ++i) {
+                        const bool valid = ((vm >> i) & 1u) && q2 * 32 + i <= causal;
+                        v[i] = valid ? v[i] : -INFINITY;
                     }
                 }
+            };
+            if (ok) {
                 // tile maximum in four independent chains, then in log2 units (sm_scale > 0)
-                float mx4[4] = {s[0], s[1], s[2], s[3]};
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float v[32];
+                    logits32(q2, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], v[i]);
+                }
                 const float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
                 if (tmax > m_run + kRescaleLog2) {             // also the first finite maximum
                     alpha = ex2_approx(m_run - tmax);
@@ -453,30 +454,36 @@ prefill_attend_kernel(PrefillAttendParams p) {
                 const uint32_t ph = smem_u32(sh.p_hi), pl = smem_u32(sh.p_lo);
                 float add4[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of running sums
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    uint32_t hw[4], lw[4];
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float s[32];
+                    logits32(q2, s);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int i = c8 * 8 + 2 * j;
-                        float x0, x1;
-                        ffma2(x0, x1, s[i], s[i + 1], sl2, sl2, -mu, -mu);
-                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                        const int a = (j & 1) * 2;
-                        fadd2(add4[a], add4[a + 1], add4[a], add4[a + 1], p0, p1);
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                        const float2 hf = __bfloat1622float2(h);
-                        float r0, r1;
-                        fadd2(r0, r1, p0, p1, -hf.x, -hf.y);
-                        const __nv_bfloat162 lo = __floats2bfloat162_rn(r0, r1);
-                        hw[j] = *reinterpret_cast<const uint32_t*>(&h);
-                        lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int i = c4 * 8 + 2 * j;
+                            float x0, x1;
+                            ffma2(x0, x1, s[i], s[i + 1], sl2, sl2, -mu, -mu);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const int a = (j & 1) * 2;
+                            fadd2(add4[a], add4[a + 1], add4[a], add4[a + 1], p0, p1);
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                            const float2 hf = __bfloat1622float2(h);
+                            float r0, r1;
+                            fadd2(r0, r1, p0, p1, -hf.x, -hf.y);
+                            const __nv_bfloat162 lo = __floats2bfloat162_rn(r0, r1);
+                            hw[j] = *reinterpret_cast<const uint32_t*>(&h);
+                            lw[j] = *reinterpret_cast<const uint32_t*>(&lo);
+                        }
+                        const uint32_t off = tile_off(r, half * 8 + q2 * 4 + c4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[0]),
+                                     "r"(hw[1]), "r"(hw[2]), "r"(hw[3]));
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[0]),
+                                     "r"(lw[1]), "r"(lw[2]), "r"(lw[3]));
                     }
-                    const uint32_t off = tile_off(r, half * 8 + c8);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(ph + off), "r"(hw[0]), "r"(hw[1]),
-                                 "r"(hw[2]), "r"(hw[3]));
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(pl + off), "r"(lw[0]), "r"(lw[1]),
-                                 "r"(lw[2]), "r"(lw[3]));
                 }
+                tc_fence_before();
                 l_run += (add4[0] + add4[1]) + (add4[2] + add4[3]);
                 gather_v(t + 1);
             } else {
@@ -523,12 +530,12 @@ prefill_attend_kernel(PrefillAttendParams p) {
         uint16_t* orow = p.out + qrow * 128 + half * 64;
         float* frow = p.out_f32 ? p.out_f32 + qrow * 128 + half * 64 : nullptr;
 #pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-            float va[32], vb[32];
-            tmem_ld32(t_oa + uint32_t(half * 64 + cb * 32) + lane_off, va);
-            tmem_ld32(t_oa + 128 + uint32_t(half * 64 + cb * 32) + lane_off, vb);
+        for (int cb = 0; cb < 4; ++cb) {
+            float va[16], vb[16];
+            tmem_ld16(t_oa + uint32_t(half * 64 + cb * 16) + lane_off, va);
+            tmem_ld16(t_oa + 128 + uint32_t(half * 64 + cb * 16) + lane_off, vb);
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
+            for (int i = 0; i < 16; i += 8) {
                 float o[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) o[k] = va[i + k] * sa + vb[i + k] * sb;
@@ -538,10 +545,10 @@ prefill_attend_kernel(PrefillAttendParams p) {
                     const __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
                     w[k] = *reinterpret_cast<const uint32_t*>(&h);
                 }
-                *reinterpret_cast<uint4*>(orow + cb * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(orow + cb * 16 + i) = make_uint4(w[0], w[1], w[2], w[3]);
                 if (frow) {
-                    *reinterpret_cast<float4*>(frow + cb * 32 + i) = make_float4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<float4*>(frow + cb * 32 + i + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                    *reinterpret_cast<float4*>(frow + cb * 16 + i) = make_float4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<float4*>(frow + cb * 16 + i + 4) = make_float4(o[4], o[5], o[6], o[7]);
                 }
             }
         }
