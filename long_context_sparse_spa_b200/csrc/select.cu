@@ -180,6 +180,7 @@ select_kernel(SelectParams p, int chunk, int resident_launch) {
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
     const int rank = int(cluster.block_rank());
+    const bool solo = C == 1;
     const int u = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -363,24 +364,27 @@ select_kernel(SelectParams p, int chunk, int resident_launch) {
                 for (int i = tid; i < n; i += kSelThreads) add(__ldg(srow + i));
             }
             __syncthreads();
-            // the unit's merged histogram: every CTA adds its nonzero bins with global
-            // reductions (integer sums: the result does not depend on their order)
+            auto local_mass = [&](int i) -> u64 {
+                return wide ? hist_wide[i]
+                            : u64(sh.hist_part[0][i]) + (u64(sh.hist_part[1][i]) << 14) +
+                                  (u64(sh.hist_part[2][i]) << 28);
+            };
+            // the unit's merged histogram.  A lone CTA's shared histogram already is the merged
+            // one; in a cluster every CTA adds its nonzero bins with global reductions (integer
+            // sums: the result does not depend on their order)
             const int goff = level == 1 ? 0 : kBins;
             uint32_t* gcnt = p.hist.lvl_cnt + size_t(u) * kLvlBins + goff;
             u64* gmass = p.hist.lvl_mass + size_t(u) * kLvlBins + goff;
-            for (int i = tid; i < nb; i += kSelThreads) {
-                const uint32_t c = sh.hist_cnt[i];
-                if (c) {
-                    atomicAdd(gcnt + i, c);
-                    if (TOPP) {
-                        const u64 m = wide ? hist_wide[i]
-                                           : u64(sh.hist_part[0][i]) + (u64(sh.hist_part[1][i]) << 14) +
-                                                 (u64(sh.hist_part[2][i]) << 28);
-                        atomicAdd(gmass + i, m);
+            if (!solo) {
+                for (int i = tid; i < nb; i += kSelThreads) {
+                    const uint32_t c = sh.hist_cnt[i];
+                    if (c) {
+                        atomicAdd(gcnt + i, c);
+                        if (TOPP) atomicAdd(gmass + i, local_mass(i));
                     }
                 }
+                cluster.sync();   // every CTA's reductions are performed (release / acquire at cluster scope)
             }
-            cluster.sync();   // every CTA's reductions are performed (release / acquire at cluster scope)
 
             const int per = nb / kSelThreads;    // bins per thread, descending
             uint32_t vc[kPerMax];
@@ -392,8 +396,13 @@ select_kernel(SelectParams p, int chunk, int resident_launch) {
                 vc[j] = 0; vm[j] = 0;
                 if (j < per) {
                     const int bin = nb - 1 - (tid * per + j);
-                    vc[j] = __ldcg(gcnt + bin);
-                    if (TOPP) vm[j] = __ldcg(gmass + bin);
+                    if (solo) {
+                        vc[j] = sh.hist_cnt[bin];
+                        if (TOPP) vm[j] = local_mass(bin);
+                    } else {
+                        vc[j] = __ldcg(gcnt + bin);
+                        if (TOPP) vm[j] = __ldcg(gmass + bin);
+                    }
                     sc += vc[j];
                     sm += vm[j];
                 }
@@ -637,9 +646,12 @@ select_kernel(SelectParams p, int chunk, int resident_launch) {
             p.hist.cnt[size_t(u) * kBins + i] = 0;
             p.hist.mass[size_t(u) * kBins + i] = 0;
         }
-        for (int i = tid; i < kLvlBins; i += kSelThreads) {
-            p.hist.lvl_cnt[size_t(u) * kLvlBins + i] = 0;
-            p.hist.lvl_mass[size_t(u) * kLvlBins + i] = 0;
+        // (a lone CTA never wrote the level 1 and 2 bins)
+        if (!solo) {
+            for (int i = tid; i < kLvlBins; i += kSelThreads) {
+                p.hist.lvl_cnt[size_t(u) * kLvlBins + i] = 0;
+                p.hist.lvl_mass[size_t(u) * kLvlBins + i] = 0;
+            }
         }
         if (tid == 0) {
             p.hist.max_key[u] = 0;
