@@ -7,7 +7,9 @@
 //
 // Work split: every unit (one support) has R_u gathered rows, cut into tiles of 16
 // rows.  The tiles of all units form one list, split evenly over all CTAs (two per SM),
-// so every SM streams the same number of K/V bytes whatever the support sizes.  Inside
+// so every SM streams about the same number of K/V bytes whatever the support sizes; each
+// unit is charged a fixed segment cost on top of its tiles, so that a CTA whose share spans
+// several units (and pays their start-up and merge) gets fewer tiles.  Inside
 // a CTA the four warps take a unit's tiles round-robin; each warp gathers its tiles
 // with cp.async (16-byte copies, bounds-checked, zero-filled when the index is out of
 // range) into a private multi-stage ring in shared memory.
@@ -40,6 +42,12 @@ constexpr int kRows = 16;           // rows per tile (the mma N-extent of the sc
 constexpr int kStages = 3;          // cp.async ring depth per warp
 constexpr int kMaxUnits = 8192;
 constexpr int kWinTiles = 128;      // tiles whose row indices are staged in shared memory at once
+// Fixed cost of a segment (one unit's share of a CTA's range) in tiles: draining the gathers,
+// the merge of the warps, the partial's store, the next unit's query and index loads and the
+// refill of the rings.  Measured on B200 at 5-8 us per extra segment against about 0.5 us per
+// tile of a CTA, so it is charged as 12 tiles at the head of every non-empty unit when the tiles
+// are split over the CTAs: a CTA whose range crosses unit boundaries gets fewer tiles.
+constexpr int kSegCost = 12;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -82,7 +90,7 @@ struct Tile {
     static constexpr int NT = D / 8;                  // 8-wide output column tiles
 };
 
-// owner CTA of tile x when TT tiles are split over G CTAs as [TT*c/G, TT*(c+1)/G)
+// owner CTA of (weighted) tile x when TT tiles are split over G CTAs as [TT*c/G, TT*(c+1)/G)
 __device__ __forceinline__ int tile_owner(long long x, long long TT, int G) {
     return int(((x + 1) * G - 1) / TT);
 }
@@ -115,6 +123,7 @@ attend_kernel(AttendParams p, int U, int nh) {
             int c = p.count[u];
             c = c < 0 ? 0 : (c > p.cap ? p.cap : c);
             t = (c * p.unit_tokens + kRows - 1) / kRows;
+            if (t > 0) t += kSegCost;   // the unit's tiles, weighted by the fixed cost of a segment
         }
         int incl = t;
 #pragma unroll
@@ -137,8 +146,10 @@ attend_kernel(AttendParams p, int U, int nh) {
     __syncthreads();
     const long long TT = running;
     const int cta = blockIdx.x;
-    // Tiles are split over G = min(grid, TT) CTAs so that every range is non-empty (the
-    // partial accounting counts CTAs); the rest only serve empty supports.
+    // Weighted tiles are split over G = min(grid, TT) CTAs so that every range is non-empty;
+    // the rest only serve empty supports.  A range may hold only a unit's cost share: the CTA
+    // then produces nothing for that unit, and the combine kernel takes the unit's partials
+    // from the CTAs that own its first to its last real tile.
     const int G = int(TT < (long long)gridDim.x ? TT : (long long)gridDim.x);
 
     // ---- empty supports: out = 0, lse = -inf
@@ -159,7 +170,7 @@ attend_kernel(AttendParams p, int U, int nh) {
         for (int v = tid; v < U; v += kAtThreads) {
             int lo = -1, hi = -1;
             if (s_prefix[v + 1] > s_prefix[v]) {
-                lo = tile_owner(s_prefix[v], TT, G);
+                lo = tile_owner(s_prefix[v] + kSegCost, TT, G);   // owner of the first real tile
                 hi = tile_owner(s_prefix[v + 1] - 1, TT, G);
                 if (lo == hi && !RLA) lo = hi = -1;
             }
@@ -185,9 +196,14 @@ attend_kernel(AttendParams p, int U, int nh) {
     while (x < t1) {
         while (s_prefix[u + 1] <= x) ++u;
         const long long seg_end = min(t1, (long long)s_prefix[u + 1]);
-        const int a = int(x - s_prefix[u]);
-        const int bnd = int(seg_end - s_prefix[u]);
-        const int tiles_u = s_prefix[u + 1] - s_prefix[u];
+        // the unit's weighted range is its segment cost, then its tiles: [a, bnd) are real tiles
+        const int a = max(int(x - s_prefix[u]) - kSegCost, 0);
+        const int bnd = max(int(seg_end - s_prefix[u]) - kSegCost, 0);
+        const int tiles_u = s_prefix[u + 1] - s_prefix[u] - kSegCost;
+        if (a >= bnd) {   // only the cost share of the unit (uniform over the CTA)
+            x = seg_end;
+            continue;
+        }
         const UnitGeom ug = unit_geom(p, u, nh);
 
         // Q^T as the B operand of S^T = K Q^T: b0/b1 of k-step kk, head tile nt hold
