@@ -22,7 +22,9 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 // so the result does not depend on the order of accumulation).
 constexpr int kLrThreads = 256;
 constexpr int kLrUnroll = 8;
-constexpr int kLrChunk = 2048;
+// At most 4080 rows per item: each 32-bit half of an item's fixed-point bin masses takes at most
+// 2^20 per row (masses are at most 2^40), so no half can overflow below 4096 rows.
+constexpr int kLrChunk = 4080;
 
 template <int NQ, bool HIST, bool MASS>
 __global__ void __launch_bounds__(kLrThreads)
@@ -128,7 +130,7 @@ lowrank_scores_kernel(const uint16_t* __restrict__ qidx, const uint4* __restrict
                             atomicAdd(&h_cnt[bin], 1u);
                             if (MASS) {
                                 // the 41-bit fixed-point mass as two 32-bit halves (20 low
-                                // bits, the rest high): with <= kLrChunk = 2048 rows per work
+                                // bits, the rest high): with <= kLrChunk < 4096 rows per work
                                 // item neither half can overflow
                                 const unsigned long long e = fixed_mass(sc, bin_top_score(bin));
                                 atomicAdd(&h_mhi[bin], uint32_t(e >> 20));
@@ -453,24 +455,24 @@ int grid_for(int items, int per_sm) {
     return items < cap ? (items > 0 ? items : 1) : cap;
 }
 
-// Rows per work item of the low-rank scorer, at most kLrChunk.  A grid with fewer items than SMs
-// (a short cache: 4K tokens make two 2048-row items per unit) is split into more, shorter items,
-// about one wave of the CTAs the SMs hold at once, each of at least min_rows rows (a histogram item
-// clears and flushes 2048 bins).  Larger grids keep 2048-row items: splitting them further was
-// measured slower (more clears and flushes, for a partial last wave that the next kernel's launch
-// overlaps anyway).
+// Rows per work item of the low-rank scorer, at most kLrChunk.  The grid is made a whole number
+// of waves of the CTAs the SMs hold at once: the fewest waves for which items of at most
+// kLrChunk rows cover every unit, with every unit cut into the same number of items.  A partial
+// last wave (1024 items of 2048 rows for 592 resident CTAs at a 128K-token cache) leaves most of
+// the SMs idle while it runs.  Short caches are cut into items of at least min_rows rows (a
+// histogram item clears and flushes 2048 bins).
 template <typename Kern>
 int lr_chunk_rows(Kern kern, int units, int M, int min_rows) {
-    const int base = (M + kLrChunk - 1) / kLrChunk;
     const int sms = device_info().num_sms;
-    if ((long long)units * base >= sms) return kLrChunk;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLrThreads, 0) != cudaSuccess || per_sm <= 0) {
         cudaGetLastError();
         per_sm = 1;
     }
     const long long resident = (long long)per_sm * sms;
-    const long long per_unit = (resident + units - 1) / units;   // chunks per unit for about one wave
+    const long long fewest = (long long)units * ((M + kLrChunk - 1) / kLrChunk);   // items at kLrChunk rows
+    const long long waves = (fewest + resident - 1) / resident;
+    const long long per_unit = (waves * resident + units - 1) / units;             // items per unit
     int rows = int((M + per_unit - 1) / per_unit);
     rows = (rows + 15) / 16 * 16;
     rows = rows < min_rows ? min_rows : rows;
