@@ -33,9 +33,12 @@ namespace cg = cooperative_groups;
 namespace spa {
 namespace {
 
-constexpr int kSelThreads = 512;
-constexpr int kPerMax = 2048 / kSelThreads;   // histogram bins per thread in a scan
-constexpr int kSelWarps = kSelThreads / 32;
+// Threads per selection CTA: 512 when the chunk is resident in shared memory, 1024 when it is
+// streamed from L2 on every level (twice the loads in flight; measured on B200 at 1M scores per
+// unit in clusters of 16: 111 -> 86 us).  Resident chunks are faster with 512.
+constexpr int kSelThreadsResident = 512;
+constexpr int kSelThreadsStream = 1024;
+constexpr int kMaxSelWarps = kSelThreadsStream / 32;
 constexpr int kBins = 2048;
 constexpr int kMaxCluster = 16;   // 16 is a non-portable cluster size, allowed on sm_100
 constexpr double kInvMassScale = 1.0 / 1099511627776.0;   // 2^-40
@@ -52,9 +55,9 @@ constexpr int kBulkPiece = 32768;               // bytes per bulk copy of the ch
 struct SelShared {
     uint32_t hist_cnt[kBins];     // local histogram of the current level (levels 1 and 2)
     uint32_t hist_part[3][kBins];
-    uint32_t warp_u32[kSelWarps];
-    u64 warp_u64[kSelWarps];
-    double warp_f64[kSelWarps];
+    uint32_t warp_u32[kMaxSelWarps];
+    u64 warp_u64[kMaxSelWarps];
+    double warp_f64[kMaxSelWarps];
     uint32_t sel_of[kMaxCluster];   // selected count of every CTA of the cluster (pushed by each)
     double fmass_of[kMaxCluster];   // mass of every CTA's forced-only elements (pushed by each)
     u64 load_bar;                   // completion of the chunk's bulk copy
@@ -66,8 +69,9 @@ struct SelShared {
     Level0Shared l0;
 };
 
-// Block-wide exclusive scan of (a, b) in thread order; totals returned too.  Fixed order.
-template <typename TB>
+// Block-wide exclusive scan of (a, b) in thread order over NW warps; totals returned too.
+// Fixed order.
+template <int NW, typename TB>
 __device__ __forceinline__ void block_exscan(uint32_t a, TB b, uint32_t& ea, TB& eb, uint32_t& ta, TB& tb,
                                              uint32_t* wa_s, TB* wb_s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -84,7 +88,7 @@ __device__ __forceinline__ void block_exscan(uint32_t a, TB b, uint32_t& ea, TB&
     uint32_t wa = 0, sa = 0;
     TB wb = 0, sb = 0;
 #pragma unroll
-    for (int w = 0; w < kSelWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
         const uint32_t va = wa_s[w];
         const TB vb = wb_s[w];
         if (w < warp) { wa += va; wb += vb; }
@@ -173,9 +177,12 @@ hist0_kernel(SelectParams p, int chunks_per_unit, int n_items) {
 }
 
 // ============================================================================ selection
-template <bool TOPP>
-__global__ void __launch_bounds__(kSelThreads, 2)
+template <bool TOPP, int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT)
 select_kernel(SelectParams p, int chunk, int resident_launch) {
+    constexpr int kSelThreads = NT;
+    constexpr int kSelWarps = NT / 32;
+    constexpr int kPerMax = 2048 / NT;   // histogram bins per thread in a scan
     pdl_enter();
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
@@ -409,7 +416,7 @@ select_kernel(SelectParams p, int chunk, int resident_launch) {
             }
             uint32_t ec, tc;
             u64 em, tm;
-            block_exscan<u64>(sc, sm, ec, em, tc, tm, sh.warp_u32, sh.warp_u64);
+            block_exscan<kSelWarps, u64>(sc, sm, ec, em, tc, tm, sh.warp_u32, sh.warp_u64);
             if (tid == 0) {   // defaults if rounding left no crossing: the last non-empty bin
                 sh.found_bin = 0;
                 sh.found_above_cnt = cum_c;
@@ -672,9 +679,10 @@ struct SelectConfig {
     int chunk;
     int resident;
     size_t smem;
+    int nt;   // threads per CTA
 };
 
-template <bool TOPP>
+template <bool TOPP, int NT>
 int max_active_clusters(int C, size_t smem) {
     // cached per (device, C, smem bucket)
     static thread_local int cache_dev = -1;
@@ -690,7 +698,7 @@ int max_active_clusters(int C, size_t smem) {
     if (v < 0) {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(C, 1, 1);
-        cfg.blockDim = dim3(kSelThreads, 1, 1);
+        cfg.blockDim = dim3(NT, 1, 1);
         cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -700,7 +708,7 @@ int max_active_clusters(int C, size_t smem) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, select_kernel<TOPP>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, select_kernel<TOPP, NT>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -719,13 +727,20 @@ int max_active_clusters(int C, size_t smem) {
 constexpr double kSelFixed = 40960.0;
 constexpr double kSelStreamCost = 3.0;
 template <bool TOPP>
+using SelectKernel = void (*)(SelectParams, int, int);
+
+template <bool TOPP>
+SelectKernel<TOPP> select_kernel_for(int nt) {
+    return nt == kSelThreadsStream ? select_kernel<TOPP, kSelThreadsStream> : select_kernel<TOPP, kSelThreadsResident>;
+}
+
+template <bool TOPP>
 SelectConfig choose(int U, int M) {
     const DeviceInfo& di = device_info();
     const size_t fixed = align_up(sizeof(SelShared), 16);
     SelectConfig best{};
     best.C = 0;
     double best_cost = 0.0;
-    cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     for (int C = kMaxCluster; C >= 1; C /= 2) {
         if (C > 1 && (M + C - 1) / C < 2048) continue;
         const int chunk = ((M + C - 1) / C + 3) / 4 * 4;
@@ -735,14 +750,17 @@ SelectConfig choose(int U, int M) {
             resident = 0;
             smem = fixed;
         }
-        cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        const int nt = resident ? kSelThreadsResident : kSelThreadsStream;
+        const SelectKernel<TOPP> kern = select_kernel_for<TOPP>(nt);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         int active = 0;   // units whose CTAs run at once
         if (C > 1) {
-            active = max_active_clusters<TOPP>(C, smem);
+            active = resident ? max_active_clusters<TOPP, kSelThreadsResident>(C, smem)
+                              : max_active_clusters<TOPP, kSelThreadsStream>(C, smem);
         } else {
             int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<TOPP>, kSelThreads, smem) !=
-                cudaSuccess) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem) != cudaSuccess) {
                 cudaGetLastError();
                 per_sm = 1;
             }
@@ -752,11 +770,11 @@ SelectConfig choose(int U, int M) {
         const double waves = double((U + active - 1) / active);
         const double cost = waves * (double(chunk) * (resident ? 1.0 : kSelStreamCost) + kSelFixed);
         if (best.C == 0 || cost < best_cost) {
-            best = SelectConfig{C, chunk, resident, smem};
+            best = SelectConfig{C, chunk, resident, smem, nt};
             best_cost = cost;
         }
     }
-    if (best.C == 0) best = SelectConfig{1, M, 0, fixed};
+    if (best.C == 0) best = SelectConfig{1, M, 0, fixed, kSelThreadsStream};
     return best;
 }
 
@@ -765,11 +783,12 @@ spa_status launch_t(const SelectParams& p0, cudaStream_t st) {
     SelectParams p = p0;
     p.test_stall = test_stall_bits();
     const SelectConfig c = choose<TOPP>(p.U, p.M);
-    SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-    SPA_CUDA_TRY(cudaFuncSetAttribute(select_kernel<TOPP>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)));
+    const SelectKernel<TOPP> kern = select_kernel_for<TOPP>(c.nt);
+    SPA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    SPA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(c.C, p.U, 1);
-    cfg.blockDim = dim3(kSelThreads, 1, 1);
+    cfg.blockDim = dim3(c.nt, 1, 1);
     cfg.dynamicSmemBytes = c.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -781,7 +800,7 @@ spa_status launch_t(const SelectParams& p0, cudaStream_t st) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    SPA_CUDA_TRY(cudaLaunchKernelEx(&cfg, select_kernel<TOPP>, p, c.chunk, c.resident));
+    SPA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, p, c.chunk, c.resident));
     return SPA_OK;
 }
 
