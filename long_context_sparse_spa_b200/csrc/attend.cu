@@ -45,9 +45,10 @@ constexpr int kWinTiles = 128;      // tiles whose row indices are staged in sha
 // Fixed cost of a segment (one unit's share of a CTA's range) in tiles: draining the gathers,
 // the merge of the warps, the partial's store, the next unit's query and index loads and the
 // refill of the rings.  Measured on B200 at 5-8 us per extra segment against about 0.5 us per
-// tile of a CTA, so it is charged as 12 tiles at the head of every non-empty unit when the tiles
-// are split over the CTAs: a CTA whose range crosses unit boundaries gets fewer tiles.
-constexpr int kSegCost = 12;
+// tile of a CTA (10-16 tiles), and charged as 20 tiles at the head of every non-empty unit when
+// the tiles are split over the CTAs, so that a CTA whose range crosses unit boundaries gets
+// fewer tiles (8, 12 and 20 were timed: 20 was the fastest or level on every decode workload).
+constexpr int kSegCost = 20;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
