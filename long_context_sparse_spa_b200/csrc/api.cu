@@ -1,7 +1,9 @@
 // Host side of the C ABI declared in include/spa.h: argument validation, workspace
 // layout and kernel launches.  No entry point allocates device memory.
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <string>
 #include <vector>
 
@@ -43,6 +45,66 @@ const DeviceInfo& device_info() {
         d.device = dev;
     }
     return d;
+}
+
+namespace {
+std::mutex g_memo_mu;
+struct AttrKey {
+    int dev;
+    const void* func;
+    int attr;
+    bool operator<(const AttrKey& o) const {
+        return std::tie(dev, func, attr) < std::tie(o.dev, o.func, o.attr);
+    }
+};
+struct OccKey {
+    int dev;
+    const void* func;
+    int threads;
+    size_t smem;
+    bool operator<(const OccKey& o) const {
+        return std::tie(dev, func, threads, smem) < std::tie(o.dev, o.func, o.threads, o.smem);
+    }
+};
+std::map<AttrKey, int> g_attr;
+std::map<OccKey, int> g_occ;
+}  // namespace
+
+cudaError_t set_func_attr(const void* func, cudaFuncAttribute attr, int value) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const AttrKey key{dev, func, int(attr)};
+    {
+        std::lock_guard<std::mutex> lk(g_memo_mu);
+        auto it = g_attr.find(key);
+        if (it != g_attr.end() && it->second == value) return cudaSuccess;
+    }
+    const cudaError_t e = cudaFuncSetAttribute(func, attr, value);
+    std::lock_guard<std::mutex> lk(g_memo_mu);
+    if (e == cudaSuccess) g_attr[key] = value;
+    else g_attr.erase(key);
+    return e;
+}
+
+int occupancy_blocks(const void* func, int threads, size_t smem) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const OccKey key{dev, func, threads, smem};
+    {
+        std::lock_guard<std::mutex> lk(g_memo_mu);
+        auto it = g_occ.find(key);
+        if (it != g_occ.end()) return it->second;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;   // not memoised: the query may succeed once the attributes allow this size
+    }
+    if (n <= 0) return 0;   // not memoised either (an attribute may still be below this size)
+    std::lock_guard<std::mutex> lk(g_memo_mu);
+    if (g_occ.size() > 4096) g_occ.clear();
+    g_occ[key] = n;
+    return n;
 }
 
 namespace {

@@ -703,12 +703,12 @@ spa_status launch_attend(const AttendParams& p, cudaStream_t st) {
 #define SPA_AT_CASE(DD, H8, R)                                                                                   \
     if (p.d == DD && (nh + 7) / 8 == H8 && rla == R) {                                                          \
         const size_t sm = attend_smem<DD>(U);                                                                   \
-        SPA_CUDA_TRY(cudaFuncSetAttribute(attend_kernel<DD, H8, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                          int(sm)));                                                            \
+        SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(attend_kernel<DD, H8, R>),                     \
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));                     \
         SPA_CUDA_TRY(launch_pdl(attend_kernel<DD, H8, R>, dim3(grid), dim3(kAtThreads), sm, st, p, U, nh));      \
         const size_t cs = size_t(kCombRecs) * (DD + 2) * 4;                                                    \
-        SPA_CUDA_TRY(cudaFuncSetAttribute(combine_kernel<DD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
-                                          int(cs)));                                                            \
+        SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(combine_kernel<DD, R>),                        \
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(cs)));                     \
         SPA_CUDA_TRY(launch_pdl(combine_kernel<DD, R>, dim3(U, nh), dim3(256), cs, st, p, nh, U + grid));         \
         return SPA_OK;                                                                                          \
     }

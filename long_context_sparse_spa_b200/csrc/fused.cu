@@ -1201,7 +1201,8 @@ int fused_ctas() {
     const DeviceInfo& di = device_info();
     if (dev != di.device) {
         int per_sm = 0;
-        cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fused_smem()));
+        set_func_attr(reinterpret_cast<const void*>(decode_fused_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                      int(fused_smem()));
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel, kFThreads, fused_smem()) !=
                 cudaSuccess ||
             per_sm < 1) {
@@ -1293,7 +1294,8 @@ spa_status launch_fused_decode(const spa_decode_args* a, void* ws_after_header, 
     p.n_sel = U < 16 ? U : 16;
     if (p.NR > 1024) return SPA_ERR_UNSUPPORTED_SHAPE;
     const size_t smem = fused_smem();
-    SPA_CUDA_TRY(cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(decode_fused_kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
     SPA_CUDA_TRY(launch_pdl(decode_fused_kernel, dim3(n_ctas), dim3(kFThreads), smem, st, p));
     if (events) {

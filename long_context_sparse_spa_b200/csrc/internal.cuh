@@ -27,6 +27,13 @@ struct DeviceInfo {
 // Cached per device; safe to call from several host threads.
 const DeviceInfo& device_info();
 
+// Kernel attributes and occupancy queries are driver calls of microseconds each, made with the
+// same values on every launch; both are memoised per device (safe from several host threads).
+// set_func_attr calls cudaFuncSetAttribute only when the value differs from the last one set.
+cudaError_t set_func_attr(const void* func, cudaFuncAttribute attr, int value);
+// CTAs of func per SM at this block size and dynamic shared memory (0 if the query fails).
+int occupancy_blocks(const void* func, int threads, size_t smem);
+
 // Records the CUDA error (thread-local text for spa_last_cuda_error) and maps it to a status.
 spa_status cuda_fail(cudaError_t e);
 

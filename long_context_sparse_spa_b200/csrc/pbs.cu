@@ -606,10 +606,10 @@ static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, voi
 #define SPA_PB_IMP(NMT)                                                                                         \
     if (nmt == NMT) {                                                                                           \
         const size_t sm = sizeof(ImShared<NMT>);                                                                \
-        SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_importance_tc_kernel<NMT, 0>,                                     \
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));               \
-        SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_importance_tc_kernel<NMT, 1>,                                     \
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));               \
+        SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(pbs_importance_tc_kernel<NMT, 0>),            \
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));                     \
+        SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(pbs_importance_tc_kernel<NMT, 1>),            \
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)));                     \
         SPA_CUDA_TRY(launch_pdl(pbs_importance_tc_kernel<NMT, 0>, dim3(nchunk, a->Hkv), dim3(128 * NMT), sm, st,  \
                                 p, status));                                                                    \
         SPA_CUDA_TRY(launch_pdl(pbs_rowcombine_kernel, dim3((p.R + kPbThreads - 1) / kPbThreads, a->Hkv),        \
@@ -622,18 +622,21 @@ static spa_status pbs_impl(const spa_pbs_args* a, void* ws, size_t ws_bytes, voi
     // 2. permutation inside segments
     int P = 1;
     while (P < a->S) P <<= 1;
-    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P * 8)));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(pbs_sort_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(P * 8)));
     SPA_CUDA_TRY(launch_pdl(pbs_sort_kernel, dim3((a->T + a->S - 1) / a->S, a->Hkv), dim3(1024), size_t(P) * 8, st, p));
     // 3. block means, block scores, top-k blocks
     SPA_CUDA_TRY(launch_pdl(pbs_means_kernel, dim3(nblk, a->Hkv, 2), dim3(kPbD), 0, st, p));
     SPA_CUDA_TRY(launch_pdl(pbs_scores_kernel, dim3((nblk + kPbJ - 1) / kPbJ, a->Hkv), dim3(kPbThreads), 0, st, p));
     int Pk = 1;
     while (Pk < nblk) Pk <<= 1;
-    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Pk * 8)));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(pbs_topk_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(Pk * 8)));
     SPA_CUDA_TRY(launch_pdl(pbs_topk_kernel, dim3(U), dim3(kPbThreads), size_t(Pk) * 8, st, p, a->topk));
     // 4. rows of the attention, then the tcgen05 attention
     const size_t bitmap = size_t((a->T + 31) / 32) * 4;
-    SPA_CUDA_TRY(cudaFuncSetAttribute(pbs_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bitmap)));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(pbs_expand_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(bitmap)));
     SPA_CUDA_TRY(launch_pdl(pbs_expand_kernel, dim3(U), dim3(kPbThreads), bitmap, st, p));
     PrefillAttendParams pp{a->Q, a->K, a->V, p.aidx, p.acount, p.acap, a->Hq, a->Hkv, a->T, a->b, 0, a->sm_scale,
                            a->out, a->out_f32, status};

@@ -624,7 +624,8 @@ spa_status launch_prefill_attend(const PrefillAttendParams& pp0, int U, cudaStre
     PrefillAttendParams pp = pp0;
     pp.test_stall = test_stall_bits();
     const size_t smem = sizeof(PfShared);
-    SPA_CUDA_TRY(cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(prefill_attend_kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
     SPA_CUDA_TRY(launch_pdl(prefill_attend_kernel, dim3(U, pp.Hq / pp.Hkv / 2), dim3(kPfThreads), smem, st, pp));
     if (events) SPA_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));

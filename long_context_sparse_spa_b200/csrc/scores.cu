@@ -464,11 +464,8 @@ int grid_for(int items, int per_sm) {
 template <typename Kern>
 int lr_chunk_rows(Kern kern, int units, int M, int min_rows) {
     const int sms = device_info().num_sms;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLrThreads, 0) != cudaSuccess || per_sm <= 0) {
-        cudaGetLastError();
-        per_sm = 1;
-    }
+    int per_sm = occupancy_blocks(reinterpret_cast<const void*>(kern), kLrThreads, 0);
+    if (per_sm <= 0) per_sm = 1;
     const long long resident = (long long)per_sm * sms;
     const long long fewest = (long long)units * ((M + kLrChunk - 1) / kLrChunk);   // items at kLrChunk rows
     const long long waves = (fewest + resident - 1) / resident;

@@ -24,6 +24,10 @@
 // (ballot + popc prefix) and packs the selected positions in place in shared memory; a
 // block scan and a cluster-wide prefix of the CTA counts give every list its offset in the
 // ascending support, and the lists are copied out coalesced.
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include <cooperative_groups.h>
 
 #include "internal.cuh"
@@ -736,7 +740,16 @@ SelectKernel<TOPP> select_kernel_for(int nt) {
 
 template <bool TOPP>
 SelectConfig choose(int U, int M) {
+    // memoised per (device, U, M): the choice depends on nothing else
+    static std::mutex memo_mu;
+    static std::map<std::tuple<int, int, int>, SelectConfig> memo;
     const DeviceInfo& di = device_info();
+    const std::tuple<int, int, int> key{di.device, U, M};
+    {
+        std::lock_guard<std::mutex> lk(memo_mu);
+        auto it = memo.find(key);
+        if (it != memo.end()) return it->second;
+    }
     const size_t fixed = align_up(sizeof(SelShared), 16);
     SelectConfig best{};
     best.C = 0;
@@ -752,18 +765,15 @@ SelectConfig choose(int U, int M) {
         }
         const int nt = resident ? kSelThreadsResident : kSelThreadsStream;
         const SelectKernel<TOPP> kern = select_kernel_for<TOPP>(nt);
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        set_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        set_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         int active = 0;   // units whose CTAs run at once
         if (C > 1) {
             active = resident ? max_active_clusters<TOPP, kSelThreadsResident>(C, smem)
                               : max_active_clusters<TOPP, kSelThreadsStream>(C, smem);
         } else {
-            int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem) != cudaSuccess) {
-                cudaGetLastError();
-                per_sm = 1;
-            }
+            int per_sm = occupancy_blocks(reinterpret_cast<const void*>(kern), nt, smem);
+            if (per_sm <= 0) per_sm = 1;
             active = per_sm * di.num_sms;
         }
         if (active <= 0) continue;
@@ -775,6 +785,9 @@ SelectConfig choose(int U, int M) {
         }
     }
     if (best.C == 0) best = SelectConfig{1, M, 0, fixed, kSelThreadsStream};
+    std::lock_guard<std::mutex> lk(memo_mu);
+    if (memo.size() > 4096) memo.clear();
+    memo[key] = best;
     return best;
 }
 
@@ -784,8 +797,9 @@ spa_status launch_t(const SelectParams& p0, cudaStream_t st) {
     p.test_stall = test_stall_bits();
     const SelectConfig c = choose<TOPP>(p.U, p.M);
     const SelectKernel<TOPP> kern = select_kernel_for<TOPP>(c.nt);
-    SPA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-    SPA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    SPA_CUDA_TRY(set_func_attr(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(c.smem)));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(c.C, p.U, 1);
     cfg.blockDim = dim3(c.nt, 1, 1);

@@ -115,6 +115,7 @@ SELECT_CASES = [
     ("needles", 64, 2048, 32, 1, 2),
     ("gauss", 1, 1, 1, 1, 1),
     ("gauss", 3, 50003, 5000, 600, 600),  # forced ranges overlapping the top set
+    ("gauss", 2, 1000003, 5000, 4, 128),  # chunks streamed from L2 (1024-thread CTAs), ragged tail
 ]
 
 
@@ -151,7 +152,8 @@ TOPP_CASES = [
     ("equal", 2, 1000, 0.5, 0, 0),
     ("gauss", 2, 3000, 1.0, 0, 0),
     ("gauss", 2, 3000, 1e-6, 3, 3),
-    ("needles", 2, 262144, 0.9, 4, 256),   # streaming (keys not resident in shared memory)
+    ("needles", 2, 262144, 0.9, 4, 256),   # clusters of 16 CTAs
+    ("needles", 1, 1048583, 0.9, 4, 256),  # chunks streamed from L2 (1024-thread CTAs), ragged tail
 ]
 
 
