@@ -15,10 +15,13 @@
 //            count reaches k, or the cumulative mass (scaled to the unit's maximum, fp64,
 //            fixed order) reaches p times the total -- is found by one block scan.
 //   levels 1, 2: one thread-block cluster of C CTAs per unit.  Each CTA holds a contiguous
-//            chunk of the unit's scores in shared memory; only elements of B0 are
-//            histogrammed (masses relative to the same bin reference, so they sum exactly to
-//            the level-0 mass of B0); the peers' histograms are merged over distributed
-//            shared memory in a fixed peer order and scanned from the top.
+//            chunk of the unit's scores in shared memory (512 threads), or streams it from L2
+//            on every level when it is too long for shared memory (1024 threads); only
+//            elements of B0 are histogrammed (masses relative to the same bin reference, so
+//            they sum exactly to the level-0 mass of B0).  The CTAs add their nonzero bins to
+//            the unit's merged histogram in global memory with integer reductions (order-free),
+//            meet at one cluster barrier and scan the merged bins from the top; a lone CTA
+//            (C = 1) scans its own shared histogram.
 // The result is the threshold key tau and the quota q of elements equal to tau, taken in
 // ascending position.  Compaction walks each warp's slice of the chunk in ascending order
 // (ballot + popc prefix) and packs the selected positions in place in shared memory; a
