@@ -294,6 +294,9 @@ select_kernel(SelectParams p, int chunk, int resident_launch) {
     }
     const float r0 = bin_top_score(b0);                       // mass reference inside B0
     const double scale0 = TOPP ? kInvMassScale * exp(double(r0) - double(m)) : 0.0;
+    // Thread 0 initialised the chunk barrier: level 0's block barriers order that before every
+    // thread's first poll; a unit without level 0 (all or none selected) needs this one.
+    if (bulk && !thresholded) __syncthreads();
     wait_chunk();
 
     // ---- levels 1 and 2 inside B0
